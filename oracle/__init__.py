@@ -1,0 +1,130 @@
+"""CPU oracle for MiniMax Sparse Attention (MSA) -- TEST INFRASTRUCTURE ONLY.
+
+This package wraps ``msa_oracle.c``: a plain, slow, double-precision C
+restatement of the method (index branch: one index query per GQA group, plain
+dot product with every visible index key, block max-pool over 128-token
+blocks, top-k with the own block kept and ties to the lower id; sparse branch:
+exact softmax attention over the kept blocks, shared by the group's heads).
+The sources are the cloud.tencent.com MSA article, sections 二 and 六, and the
+mlqm.cn guide's configuration-file passage.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never imports, links
+or calls it, and this package imports nothing from the CUDA library.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "msa_oracle.c")
+_SO = os.path.join(_HERE, "libmsa_oracle.so")
+_lib = None
+
+GCC_FLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-pthread", "-ffp-contract=off"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        tmp = _SO + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *GCC_FLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _SO)
+    return _SO
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        L = ctypes.c_int64
+        lib.oracle_index_topk.argtypes = [I, I, I, I, I, I, P, P, P, P, L, P, L, P, P, P, I, P, I]
+        lib.oracle_index_topk.restype = I
+        lib.oracle_sparse_attention.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, P, L,
+                                                ctypes.c_double, P, L, P, P, I]
+        lib.oracle_sparse_attention.restype = I
+        _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:  # pragma: no cover
+        return max(1, os.cpu_count() or 1)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def index_topk(q_idx, k_idx, lens, kv_offsets, *, block=128, top_k=16, rows=None,
+               want_all_scores=False, n_threads=None):
+    """Index branch.  Shapes: q_idx [B,Sq,H_kv,D] (bf16 bits as uint16),
+    k_idx [T,H_kv,D] (packed caches), lens [B] int32, kv_offsets [B] int64.
+    ``rows`` selects flattened query rows r = b*Sq + i (default: all).
+    Returns dict(block_ids [R,H_kv,k] int32, block_scores [R,H_kv,k] float32,
+    boundary [R,H_kv,2] float64, and all_scores [R,H_kv,nb_max] if asked)."""
+    q_idx = _c(q_idx, np.uint16)
+    k_idx = _c(k_idx, np.uint16)
+    lens = _c(lens, np.int32)
+    kv_offsets = _c(kv_offsets, np.int64)
+    B, Sq, H_kv, D = q_idx.shape
+    T = k_idx.shape[0]
+    assert k_idx.shape[1:] == (H_kv, D)
+    rows_a = None if rows is None else _c(rows, np.int64)
+    R = B * Sq if rows_a is None else rows_a.shape[0]
+    ids = np.empty((R, H_kv, top_k), np.int32)
+    sc = np.empty((R, H_kv, top_k), np.float32)
+    bnd = np.empty((R, H_kv, 2), np.float64)
+    nb_max = int((int(lens.max()) + block - 1) // block)
+    allsc = np.empty((R, H_kv, nb_max), np.float64) if want_all_scores else None
+    rc = _load().oracle_index_topk(B, Sq, H_kv, D, block, top_k, _ptr(q_idx), _ptr(k_idx),
+                                   _ptr(lens), _ptr(kv_offsets), T, _ptr(rows_a), R,
+                                   _ptr(ids), _ptr(sc), _ptr(allsc), nb_max, _ptr(bnd),
+                                   n_threads or default_threads())
+    if rc != 0:
+        raise ValueError(f"oracle_index_topk rejected its input (code {rc})")
+    res = dict(block_ids=ids, block_scores=sc, boundary=bnd)
+    if want_all_scores:
+        res["all_scores"] = allsc
+    return res
+
+
+def sparse_attention(q, k, v, block_ids, lens, kv_offsets, *, block=128, scale=None,
+                     rows=None, want_wsum=False, n_threads=None):
+    """Sparse branch.  Shapes: q [B,Sq,H_q,D], k/v [T,H_kv,D] (uint16 bf16 bits),
+    block_ids [B*Sq, H_kv, k] (indexed by the flattened row r, whatever rows
+    are requested).  Returns out [R,H_q,D] float64 (and wsum [R,H_q])."""
+    q = _c(q, np.uint16)
+    k = _c(k, np.uint16)
+    v = _c(v, np.uint16)
+    lens = _c(lens, np.int32)
+    kv_offsets = _c(kv_offsets, np.int64)
+    B, Sq, H_q, D = q.shape
+    T, H_kv, _ = k.shape
+    ids = _c(block_ids, np.int32).reshape(B * Sq, H_kv, -1)
+    top_k = ids.shape[-1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    rows_a = None if rows is None else _c(rows, np.int64)
+    R = B * Sq if rows_a is None else rows_a.shape[0]
+    out = np.empty((R, H_q, D), np.float64)
+    ws = np.empty((R, H_q), np.float64) if want_wsum else None
+    rc = _load().oracle_sparse_attention(B, Sq, H_q, H_kv, D, block, top_k, _ptr(q), _ptr(k),
+                                         _ptr(v), _ptr(ids), _ptr(lens), _ptr(kv_offsets), T,
+                                         float(scale), _ptr(rows_a), R, _ptr(out), _ptr(ws),
+                                         n_threads or default_threads())
+    if rc != 0:
+        raise ValueError(f"oracle_sparse_attention rejected its input (code {rc})")
+    return (out, ws) if want_wsum else out
