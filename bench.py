@@ -1,0 +1,392 @@
+"""Benchmark of the MSA hot path on B200: one step = the whole decode path
+(index score + block max-pool, top-k, sparse attention with split-K merge)
+for one batch, through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode_1m]
+                    [--impl msa|reference] [--no-cpu-baseline] [--no-e2e]
+
+Prints ONE JSON line (rank 0).  N > 1 runs under torchrun: every rank runs
+its own independent batch (weak scaling, no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MSA decode HBM GB/s (% of 8 TB/s) & prefill sparse-attn TFLOP/s, 128k/1M"
+DOMINANT = "index_score_maxpool_decode"
+DOMINANT_SRC = os.path.join(ROOT, "block_sparse_attention_43_b200", "csrc", "index_decode.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="decode_1m",
+                    choices=["decode_1m", "decode_32k", "decode_ragged"])
+    ap.add_argument("--impl", default="msa", choices=["msa", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- bytes
+def decode_step_bytes(w, ids_host):
+    """Bytes the decode path must move per step: every index key of every
+    sequence, the valid tokens of the kept K/V blocks, q, q_idx, out, ids and
+    scores."""
+    lens = np.asarray(w.lens_host, np.int64)
+    k_idx = int(lens.sum()) * w.H_kv * w.d_idx * 2
+    kv = 0
+    ids = ids_host.reshape(w.B, w.H_kv, w.top_k)
+    for b in range(w.B):
+        L = int(lens[b])
+        for g in range(w.H_kv):
+            for j in ids[b, g]:
+                if j >= 0:
+                    kv += min(128, L - 128 * int(j))
+    kv *= w.D * 2 * 2
+    small = w.B * w.H_q * w.D * 2 * 2 + w.B * w.H_kv * w.d_idx * 2 + w.B * w.H_kv * w.top_k * 8
+    return k_idx + kv + small, k_idx
+
+
+def index_kernel_bytes(w):
+    lens = np.asarray(w.lens_host, np.int64)
+    nb = (lens + 127) // 128
+    return int(lens.sum()) * w.H_kv * w.d_idx * 2 + w.B * w.H_kv * w.d_idx * 2 + int(nb.sum()) * w.H_kv * 4
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- helpers
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_traffic():
+    """Per-launch DRAM bytes of the dominant kernel from the last ncu capture,
+    or None when the kernel source changed since."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    d = json.load(open(TRAFFIC_FILE)).get(DOMINANT)
+    if not d:
+        return None
+    h = hashlib.sha256(open(DOMINANT_SRC, "rb").read()).hexdigest()
+    if d.get("source_sha256") != h:
+        return None
+    return d
+
+
+def dist_setup(args):
+    if args.gpus > 1 or "RANK" in os.environ:
+        import datetime
+        import torch.distributed as dist
+        rank = int(os.environ.get("RANK", 0))
+        local = int(os.environ.get("LOCAL_RANK", 0))
+        world = int(os.environ.get("WORLD_SIZE", 1))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return dist, rank, local, world
+    return None, 0, 0, 1
+
+
+def cores_used():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+def oracle_sample(w, dev_inputs=True):
+    """The oracle, as it stands, on sequence 0 of the workload (index branch
+    over all its index keys + sparse branch), on the host's cores.  Returns
+    (GB/s of that sequence's algorithmic bytes, seconds, threads, note)."""
+    import oracle
+    from synthetic import bf16_bits
+    L = w.lens_host[0]
+    off = int(w.kv_offsets[0])
+    sl = slice(off, off + L)
+    q_idx = bf16_bits(w.q_idx[:1])
+    k_idx = bf16_bits(w.k_idx[sl])
+    q = bf16_bits(w.q[:1])
+    k = bf16_bits(w.k[sl])
+    v = bf16_bits(w.v[sl])
+    lens = np.array([L], np.int32)
+    offs = np.zeros(1, np.int64)
+    threads = oracle.default_threads()
+    t0 = time.perf_counter()
+    sel = oracle.index_topk(q_idx, k_idx, lens, offs, top_k=w.top_k, n_threads=threads)
+    oracle.sparse_attention(q, k, v, sel["block_ids"], lens, offs, n_threads=threads)
+    dt = time.perf_counter() - t0
+    nbytes = L * w.H_kv * w.d_idx * 2
+    kv = sum(min(128, L - 128 * int(j)) for j in sel["block_ids"].ravel() if j >= 0) * w.D * 4
+    gbs = (nbytes + kv) / dt / 1e9
+    # The oracle spreads (row, group) work over threads: one decode row has
+    # H_kv index jobs and H_q attention jobs.
+    used = min(threads, w.H_kv)
+    return gbs, dt, used, f"sequence 0 of {w.name} ({L} tokens, all {w.H_kv} groups, both stages)"
+
+
+def run_reference(args):
+    dist, rank, local, world = dist_setup(args)
+    if rank != 0:
+        return
+    from synthetic import make_workload
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    w = make_workload(args.workload, dev)
+    vals = []
+    for i in range(args.warmup + args.steps):
+        gbs, dt, used, note = oracle_sample(w)
+        if i >= args.warmup:
+            vals.append((gbs, dt))
+    gbs = float(np.mean([v[0] for v in vals]))
+    ms = float(np.mean([v[1] for v in vals])) * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "sample": note},
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": used, "kind": "oracle",
+                             "sample": note},
+            "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- main arm
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    import block_sparse_attention_43_b200 as msa
+    from synthetic import make_workload
+
+    dist, rank, local, world = dist_setup(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = make_workload(args.workload, dev)
+    if world > 1:
+        # independent batch per rank: perturb q so ranks differ
+        w.q_idx.mul_(1.0 + 0.001 * rank)
+    stream = torch.cuda.Stream(device=dev)
+    eng = msa.MSA(batch=w.B, q_len=1, max_kv_len=max(w.lens_host), num_q_heads=w.H_q,
+                  num_kv_heads=w.H_kv, top_k=w.top_k, kv_capacity=w.kv_capacity, device=dev)
+    torch.cuda.synchronize()
+
+    def step():
+        eng.index_topk(w.q_idx, w.k_idx, w.lens, w.kv_offsets, stream)
+        eng.sparse_attention(w.q, w.k, w.v, w.lens, w.kv_offsets, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize()
+    status = eng.device_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status {msa.STATUS_NAMES.get(status, status)} after warm-up")
+    ids_host = eng.block_ids.cpu().numpy()
+    step_bytes, kidx_bytes = decode_step_bytes(w, ids_host)
+
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    msa.msa_trace_enable(True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ms_total = ev0.elapsed_time(ev1)
+    trace = msa.msa_trace_read()
+    msa.msa_trace_enable(False)
+    clk = clocks.stop()
+
+    launches = len(trace)
+    dom = [t for n, t in trace if n == DOMINANT]
+    dom_ms = float(np.mean(dom)) if dom else float("nan")
+    shares = {}
+    for n, t in trace:
+        shares[n] = shares.get(n, 0.0) + t
+
+    if dist is not None:
+        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    value = step_bytes * world / (ms_step / 1e3) / 1e9
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(w, eng, stream, args, step_bytes, world, dist)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, dt, used, note = oracle_sample(w)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": used, "kind": "oracle", "sample": note,
+               "seconds": dt}
+
+    peak, peak_kind = measured_peaks()
+    kb = index_kernel_bytes(w)
+    achieved = kb / (dom_ms / 1e3) / 1e9
+    tr = kernel_traffic()
+    traffic = None
+    if tr is not None:
+        traffic = tr["dram_bytes_per_unit"] * (kb / tr["bytes_per_unit_basis"])
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "batch": w.B, "context": max(w.lens_host),
+                       "H_q": w.H_q, "H_kv": w.H_kv, "top_k": w.top_k, "block": 128,
+                       "step_bytes": step_bytes, "index_key_bytes": kidx_bytes,
+                       "pct_of_8TBps": 100.0 * value / world / 8000.0,
+                       "l2": "inputs larger than L2 (index keys %.1f GiB per GPU)" % (kidx_bytes / 2**30),
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "roofline": {"bound": "hbm", "kernel": DOMINANT, "achieved": achieved, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": traffic, "algorithmic_bytes": kb,
+                         "avg_launch_ms": dom_ms},
+            "kernel_ms": {k: v / args.steps for k, v in shares.items()},
+            "gpu_launches": launches,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def run_e2e(w, eng, stream, args, step_bytes, world, dist):
+    """Same step through the public API from pinned host buffers: per step the
+    new query (q, q_idx) and the new token's k/v/k_idx rows go host->device
+    (the token is appended at position L-1 of every sequence's resident cache),
+    the two calls run, and out + block ids + block scores come back."""
+    B = w.B
+    pos = [int(w.kv_offsets[b]) + w.lens_host[b] - 1 for b in range(B)]
+    h_q = w.q.cpu().pin_memory()
+    h_qi = w.q_idx.cpu().pin_memory()
+    h_tok = {n: torch.stack([getattr(w, n)[p] for p in pos]).cpu().pin_memory()
+             for n in ("k", "v", "k_idx")}
+    h_out = torch.empty(eng.out.shape, dtype=eng.out.dtype).pin_memory()
+    h_ids = torch.empty(eng.block_ids.shape, dtype=torch.int32).pin_memory()
+    h_sc = torch.empty(eng.block_scores.shape, dtype=torch.float32).pin_memory()
+    d_q = torch.empty_like(w.q)
+    d_qi = torch.empty_like(w.q_idx)
+    h2d = h_q.numel() * 2 + h_qi.numel() * 2 + sum(t.numel() * 2 for t in h_tok.values())
+    d2h = h_out.numel() * 2 + h_ids.numel() * 4 + h_sc.numel() * 4
+
+    def one():
+        with torch.cuda.stream(stream):
+            d_q.copy_(h_q, non_blocking=True)
+            d_qi.copy_(h_qi, non_blocking=True)
+            for n, t in h_tok.items():
+                dst = getattr(w, n)
+                for b, p in enumerate(pos):
+                    dst[p].copy_(t[b], non_blocking=True)
+            eng.index_topk(d_qi, w.k_idx, w.lens, w.kv_offsets, stream)
+            eng.sparse_attention(d_q, w.k, w.v, w.lens, w.kv_offsets, stream=stream)
+            h_out.copy_(eng.out, non_blocking=True)
+            h_ids.copy_(eng.block_ids, non_blocking=True)
+            h_sc.copy_(eng.block_scores, non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(max(3, args.warmup // 4)):
+        one()
+    n = max(10, args.steps // 4)
+    if dist is not None:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(n):
+        one()
+    dt = (time.perf_counter() - t0) / n
+    if dist is not None:
+        t = torch.tensor([dt], dtype=torch.float64, device=w.q.device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dt = float(t.item())
+    return {"value": step_bytes * world / dt / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": dt * 1e3, "steps": n}
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,243 @@
+// msa_api.cu -- the C ABI declared in include/msa.h: argument checks,
+// workspace layout, launch sequence and the device status word.
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "msa.h"
+#include "msa_device.cuh"
+#include "msa_internal.h"
+
+namespace msa {
+
+int device_sm_count() {
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+        v = 148;
+    cache[dev].store(v, std::memory_order_relaxed);
+    return v;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool encode_kv_tensor_map(CUtensorMap *map, const void *base, int H_kv, long long capacity) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDim), static_cast<cuuint64_t>(H_kv),
+                                static_cast<cuuint64_t>(capacity)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDim) * 2,
+                                   static_cast<cuuint64_t>(kDim) * 2 * H_kv};
+    const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kBlock)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace msa
+
+using namespace msa;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool pow2_le16(int x) { return x == 1 || x == 2 || x == 4 || x == 8 || x == 16; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Shape checks shared by both calls.
+msa_status_t check_shape(const msa_shape_t *s) {
+    if (!s) return MSA_ERR_INVALID_ARG;
+    if (s->batch < 1 || s->q_len < 1 || s->max_kv_len < 1 || s->num_q_heads < 1 ||
+        s->num_kv_heads < 1 || s->top_k < 1 || s->kv_capacity < 1 || s->head_dim < 1 ||
+        s->index_dim < 1 || s->block_size < 1)
+        return MSA_ERR_INVALID_ARG;
+    if (s->num_q_heads % s->num_kv_heads) return MSA_ERR_INVALID_ARG;
+    if (s->q_len > s->max_kv_len) return MSA_ERR_INVALID_ARG;
+    if (s->head_dim != kDim || s->index_dim != kDim || s->block_size != kBlock)
+        return MSA_ERR_UNSUPPORTED;
+    if (s->top_k > 64 || !pow2_le16(s->num_kv_heads) ||
+        !pow2_le16(s->num_q_heads / s->num_kv_heads))
+        return MSA_ERR_UNSUPPORTED;
+    if (s->batch > 4096 || s->max_kv_len > (1 << 27) || s->kv_capacity >= (1LL << 31))
+        return MSA_ERR_UNSUPPORTED;
+    return MSA_OK;
+}
+
+long long rows_of(const msa_shape_t *s) { return static_cast<long long>(s->batch) * s->q_len; }
+
+int nb_max_of(const msa_shape_t *s) { return (s->max_kv_len + kBlock - 1) / kBlock; }
+
+size_t index_ws_bytes(const msa_shape_t *s) {
+    return kWsHeaderBytes +
+           round_up(static_cast<size_t>(rows_of(s)) * s->num_kv_heads * nb_max_of(s) * sizeof(float));
+}
+
+struct AttnLayout {
+    int nsplit;
+    size_t tickets_off, tickets_bytes, partials_off, total;
+};
+
+AttnLayout attn_layout(const msa_shape_t *s) {
+    AttnLayout L;
+    const long long pairs = rows_of(s) * s->num_kv_heads;
+    L.nsplit = attn_rows_nsplit(pairs, s->top_k);
+    const int G = s->num_q_heads / s->num_kv_heads;
+    L.tickets_off = kWsHeaderBytes;
+    L.tickets_bytes = L.nsplit > 1 ? round_up(static_cast<size_t>(pairs) * sizeof(int)) : 0;
+    L.partials_off = L.tickets_off + L.tickets_bytes;
+    const size_t part = L.nsplit > 1 ? static_cast<size_t>(pairs) * L.nsplit * G * (kDim + 2) * 4 : 0;
+    L.total = L.partials_off + round_up(part);
+    return L;
+}
+
+msa_status_t check_ws(void *ws, size_t have, size_t need) {
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) || have < need)
+        return MSA_ERR_WORKSPACE;
+    return MSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t msa_index_topk_workspace_size(const msa_shape_t *shape) {
+    if (check_shape(shape) != MSA_OK) return 0;
+    return index_ws_bytes(shape);
+}
+
+size_t msa_sparse_attention_workspace_size(const msa_shape_t *shape) {
+    if (check_shape(shape) != MSA_OK) return 0;
+    return attn_layout(shape).total;
+}
+
+msa_status_t msa_index_topk(const msa_shape_t *shape, const void *q_idx, const void *k_idx,
+                            const int32_t *lens, const int64_t *kv_offsets, int32_t *block_ids,
+                            float *block_scores, void *workspace, size_t workspace_bytes,
+                            msa_stream_t stream) {
+    msa_status_t st = check_shape(shape);
+    if (st != MSA_OK) return st;
+    if (!q_idx || !k_idx || !lens || !kv_offsets || !block_ids || !block_scores)
+        return MSA_ERR_INVALID_ARG;
+    if (!aligned16(q_idx) || !aligned16(k_idx)) return MSA_ERR_MISALIGNED;
+    st = check_ws(workspace, workspace_bytes, index_ws_bytes(shape));
+    if (st != MSA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int *status = reinterpret_cast<int *>(ws);
+    float *scores = reinterpret_cast<float *>(ws + kWsHeaderBytes);
+    const int nb_max = nb_max_of(shape);
+
+    if (cudaMemsetAsync(ws, 0, kWsHeaderBytes, s) != cudaSuccess) return MSA_ERR_CUDA;
+    cudaError_t e;
+    if (shape->q_len == 1) {
+        IndexDecodeArgs a;
+        a.q_idx = q_idx; a.k_idx = k_idx; a.lens = lens; a.kv_offsets = kv_offsets;
+        a.scores = scores; a.status = status;
+        a.B = shape->batch; a.H_kv = shape->num_kv_heads; a.nb_max = nb_max;
+        a.max_kv_len = shape->max_kv_len; a.capacity = shape->kv_capacity;
+        e = launch_index_decode(a, s);
+    } else {
+        IndexRowsArgs a;
+        a.q_idx = q_idx; a.k_idx = k_idx; a.lens = lens; a.kv_offsets = kv_offsets;
+        a.scores = scores; a.status = status;
+        a.B = shape->batch; a.Sq = shape->q_len; a.H_kv = shape->num_kv_heads; a.nb_max = nb_max;
+        a.max_kv_len = shape->max_kv_len; a.capacity = shape->kv_capacity;
+        e = launch_index_rows_simt(a, s);
+    }
+    if (e != cudaSuccess) return MSA_ERR_CUDA;
+    TopkArgs t;
+    t.scores = scores; t.lens = lens; t.kv_offsets = kv_offsets; t.ids = block_ids;
+    t.out_scores = block_scores; t.status = status;
+    t.B = shape->batch; t.Sq = shape->q_len; t.H_kv = shape->num_kv_heads; t.nb_max = nb_max;
+    t.K = shape->top_k; t.max_kv_len = shape->max_kv_len; t.capacity = shape->kv_capacity;
+    if (launch_topk(t, s) != cudaSuccess) return MSA_ERR_CUDA;
+    return MSA_OK;
+}
+
+msa_status_t msa_sparse_attention(const msa_shape_t *shape, const void *q, const void *k_cache,
+                                  const void *v_cache, const int32_t *block_ids,
+                                  const int32_t *lens, const int64_t *kv_offsets,
+                                  float softmax_scale, void *out, void *workspace,
+                                  size_t workspace_bytes, msa_stream_t stream) {
+    msa_status_t st = check_shape(shape);
+    if (st != MSA_OK) return st;
+    if (!q || !k_cache || !v_cache || !block_ids || !lens || !kv_offsets || !out)
+        return MSA_ERR_INVALID_ARG;
+    if (!(softmax_scale == softmax_scale) || softmax_scale == INFINITY || softmax_scale == -INFINITY)
+        return MSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return MSA_ERR_MISALIGNED;
+    const AttnLayout L = attn_layout(shape);
+    st = check_ws(workspace, workspace_bytes, L.total);
+    if (st != MSA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    if (cudaMemsetAsync(ws, 0, kWsHeaderBytes + L.tickets_bytes, s) != cudaSuccess)
+        return MSA_ERR_CUDA;
+    AttnRowsArgs a;
+    a.q = q; a.k_cache = k_cache; a.v_cache = v_cache; a.ids = block_ids; a.lens = lens;
+    a.kv_offsets = kv_offsets; a.out = out;
+    a.partials = reinterpret_cast<float *>(ws + L.partials_off);
+    a.tickets = reinterpret_cast<int *>(ws + L.tickets_off);
+    a.status = reinterpret_cast<int *>(ws);
+    a.B = shape->batch; a.Sq = shape->q_len; a.H_q = shape->num_q_heads;
+    a.H_kv = shape->num_kv_heads; a.K = shape->top_k; a.nsplit = L.nsplit;
+    a.max_kv_len = shape->max_kv_len; a.capacity = shape->kv_capacity;
+    a.softmax_scale = softmax_scale;
+    if (launch_attn_rows(a, s) != cudaSuccess) return MSA_ERR_CUDA;
+    return MSA_OK;
+}
+
+msa_status_t msa_read_device_status(const void *workspace, msa_stream_t stream) {
+    if (!workspace) return MSA_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MSA_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MSA_ERR_CUDA;
+    if (word & kStatusTimeout) return MSA_ERR_DEVICE_TIMEOUT;
+    if (word & kStatusBadLens) return MSA_ERR_BAD_LENS;
+    return MSA_OK;
+}
+
+const char *msa_status_string(msa_status_t status) {
+    switch (status) {
+        case MSA_OK: return "MSA_OK";
+        case MSA_ERR_INVALID_ARG: return "MSA_ERR_INVALID_ARG: null pointer or invalid size";
+        case MSA_ERR_UNSUPPORTED: return "MSA_ERR_UNSUPPORTED: size not handled by this build";
+        case MSA_ERR_WORKSPACE: return "MSA_ERR_WORKSPACE: workspace missing, short or misaligned";
+        case MSA_ERR_CUDA: return "MSA_ERR_CUDA: a CUDA call or launch failed";
+        case MSA_ERR_DEVICE_TIMEOUT: return "MSA_ERR_DEVICE_TIMEOUT: a device wait gave up";
+        case MSA_ERR_BAD_LENS: return "MSA_ERR_BAD_LENS: lens, offsets or block ids out of range";
+        case MSA_ERR_MISALIGNED: return "MSA_ERR_MISALIGNED: tensor not 16-byte aligned";
+    }
+    return "MSA_ERR_UNKNOWN";
+}
+
+}  // extern "C"

@@ -1,0 +1,95 @@
+// msa_internal.h -- host-side launchers of the MSA kernels (not exported).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "msa.h"
+
+namespace msa {
+
+// Number of SMs of the current device (cached per device).
+int device_sm_count();
+
+// Records a CUDA event pair around the kernel launched in its scope when the
+// trace is enabled (msa_trace_enable); a no-op otherwise.
+class TraceScope {
+  public:
+    TraceScope(cudaStream_t s, const char *name);
+    ~TraceScope();
+
+  private:
+    cudaStream_t stream_;
+    int slot_;
+};
+
+// Block max-pooled index scores for decode (one query row per sequence):
+// scores[b][g][j] = max over tokens t of block j (t < lens[b]) of
+// dot(q_idx[b][0][g], k_idx[kv_offsets[b] + t][g]).
+struct IndexDecodeArgs {
+    const void *q_idx;
+    const void *k_idx;
+    const int32_t *lens;
+    const int64_t *kv_offsets;
+    float *scores;          // [B][H_kv][nb_max]
+    int *status;
+    int B, H_kv, nb_max, max_kv_len;
+    long long capacity;
+};
+cudaError_t launch_index_decode(const IndexDecodeArgs &a, cudaStream_t s);
+
+// Block max-pooled index scores for q_len >= 1 query rows per sequence
+// (prefill), causal: scores[r][g][j] for every visible block j <= own(r).
+struct IndexRowsArgs {
+    const void *q_idx;      // [B][Sq][H_kv][128]
+    const void *k_idx;
+    const int32_t *lens;
+    const int64_t *kv_offsets;
+    float *scores;          // [B*Sq][H_kv][nb_max]
+    int *status;
+    int B, Sq, H_kv, nb_max, max_kv_len;
+    long long capacity;
+};
+cudaError_t launch_index_rows_simt(const IndexRowsArgs &a, cudaStream_t s);
+// Same contract, tcgen05 tensor-core path.
+cudaError_t launch_index_rows_tc(const IndexRowsArgs &a, cudaStream_t s);
+
+// Top-k block selection per (row, group) from a block-score buffer.
+struct TopkArgs {
+    const float *scores;    // [B*Sq][H_kv][nb_max]
+    const int32_t *lens;
+    const int64_t *kv_offsets;
+    int32_t *ids;           // [B*Sq][H_kv][K]
+    float *out_scores;      // [B*Sq][H_kv][K]
+    int *status;
+    int B, Sq, H_kv, nb_max, K, max_kv_len;
+    long long capacity;
+};
+cudaError_t launch_topk(const TopkArgs &a, cudaStream_t s);
+
+// Sparse attention, one CTA per (row, group, split) over the kept blocks.
+struct AttnRowsArgs {
+    const void *q;          // [B][Sq][H_q][128]
+    const void *k_cache;
+    const void *v_cache;
+    const int32_t *ids;     // [B*Sq][H_kv][K]
+    const int32_t *lens;
+    const int64_t *kv_offsets;
+    void *out;              // [B][Sq][H_q][128]
+    float *partials;        // [B*Sq][H_kv][nsplit][G*(128+2)]
+    int *tickets;           // [B*Sq][H_kv]
+    int *status;
+    int B, Sq, H_q, H_kv, K, nsplit, max_kv_len;
+    long long capacity;
+    float softmax_scale;
+};
+cudaError_t launch_attn_rows(const AttnRowsArgs &a, cudaStream_t s);
+// Splits used by launch_attn_rows for this shape (workspace sizing too).
+int attn_rows_nsplit(long long rows_x_groups, int top_k);
+
+// Encodes a [capacity, H_kv, 128] bf16 cache as a 3-D TMA tensor map whose
+// box is (64 dims, 1 group, 128 tokens) with 128-byte swizzling.
+bool encode_kv_tensor_map(CUtensorMap *map, const void *base, int H_kv, long long capacity);
+
+}  // namespace msa

@@ -1,0 +1,161 @@
+/*
+ * msa.h -- C ABI of the B200 (sm_100a) MiniMax Sparse Attention library.
+ *
+ * MiniMax Sparse Attention (MSA) runs attention in two stages:
+ *
+ *   index branch  ("百万token上下文提速近10倍，MiniMax M3的稀疏注意力凭什么这么快",
+ *                 cloud.tencent.com, section 二): one lightweight index query
+ *                 per GQA group is dotted with a per-token index key; the
+ *                 scores are max-pooled over each 128-token KV block ("Block
+ *                 Max Pool") and the top-k blocks are kept ("Top-k").
+ *   sparse branch (same section): full softmax attention runs over the kept
+ *                 blocks only.  Every query head of a GQA group uses the
+ *                 group's one block set (same article, section 六).
+ *
+ * Block size 128, top-k 16 and index dimension 128 are the configuration the
+ * mlqm.cn MiniMax-M3 guide prints ("sparse_block_size", "sparse_topk_blocks",
+ * "sparse_index_dim").  The pages give no formula; this library fixes:
+ *   - index score s[t] = dot(q_idx[b,i,g,:], k_idx[t,g,:]), no scale;
+ *   - block score S[j] = max of s[t] over the tokens t of block j with
+ *     t <= p, where p = lens[b] - q_len + i is the query's position;
+ *   - the query's own block floor(p/128) is always kept; the other k-1 slots
+ *     go to the highest block scores among blocks j < own, ties to the lower
+ *     block id; with at most k visible blocks all are kept;
+ *   - sparse branch: softmax(softmax_scale * q.k) over the keys t <= p of the
+ *     kept blocks, applied to v; head h belongs to group h / (H_q / H_kv).
+ *
+ * Layouts (all row-major, head dim innermost, bf16 = IEEE bfloat16 bits):
+ *   q_idx  [B, q_len, H_kv, index_dim]     q   [B, q_len, H_q, head_dim]
+ *   k_idx, k_cache, v_cache: packed [kv_capacity, H_kv, dim]; sequence b
+ *          owns rows kv_offsets[b] .. kv_offsets[b] + lens[b] - 1 (a padded
+ *          cache is the case kv_offsets[b] = b * stride).
+ *   block_ids [B, q_len, H_kv, top_k] int32, ascending, -1 padded
+ *   block_scores: same shape, float32, -inf padded
+ *   out    [B, q_len, H_q, head_dim] bf16 (round to nearest even)
+ *
+ * Ownership: every pointer is caller-owned device memory (lens and
+ * kv_offsets included) and stays caller-owned; the library allocates no
+ * device memory and keeps no pointer after a call returns.  Work is enqueued
+ * on the caller's stream; no call synchronises except
+ * msa_read_device_status.  The workspace must hold at least the bytes the
+ * matching *_workspace_size call returns, 256-byte aligned, and must not be
+ * shared by calls that may run concurrently.
+ *
+ * Errors: problems visible on the host (null pointers, unsupported sizes, a
+ * short or misaligned workspace, misaligned tensors) return a status before
+ * anything is launched.  A failed launch returns MSA_ERR_CUDA.  Problems that
+ * only the device can see (lens[b] < q_len, lens[b] > max_kv_len, a sequence
+ * that runs past kv_capacity, a bounded wait that gave up) set a status word
+ * inside the workspace: the affected outputs are written as -1 / -inf / NaN,
+ * nothing outside the caller's buffers is touched, and
+ * msa_read_device_status reports the word.  The library never traps.
+ */
+#ifndef MSA_H
+#define MSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MSA_API __attribute__((visibility("default")))
+#else
+#define MSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; 0 is the legacy default stream. */
+typedef struct CUstream_st *msa_stream_t;
+
+typedef enum {
+    MSA_OK = 0,
+    MSA_ERR_INVALID_ARG = 1,    /* null pointer, non-positive size, H_q % H_kv != 0 */
+    MSA_ERR_UNSUPPORTED = 2,    /* a size this build does not handle (see below) */
+    MSA_ERR_WORKSPACE = 3,      /* workspace missing, too small or not 256-byte aligned */
+    MSA_ERR_CUDA = 4,           /* a CUDA call or kernel launch failed */
+    MSA_ERR_DEVICE_TIMEOUT = 5, /* a bounded device-side wait gave up (device status) */
+    MSA_ERR_BAD_LENS = 6,       /* lens/kv_offsets out of range (device status) */
+    MSA_ERR_MISALIGNED = 7      /* a tensor pointer is not 16-byte aligned */
+} msa_status_t;
+
+/* Problem shape.  Supported by this build: head_dim == index_dim == 128,
+ * block_size == 128, 1 <= top_k <= 64, num_kv_heads in {1, 2, 4, 8, 16},
+ * num_q_heads / num_kv_heads in {1, 2, 4, 8, 16}, batch <= 4096,
+ * max_kv_len <= 2^27, kv_capacity < 2^31. */
+typedef struct {
+    int32_t batch;        /* B */
+    int32_t q_len;        /* query rows per sequence: 1 = decode, lens[b] = full prefill */
+    int32_t max_kv_len;   /* upper bound on every lens[b] */
+    int32_t num_q_heads;  /* H_q */
+    int32_t num_kv_heads; /* H_kv = number of GQA groups = number of index queries */
+    int32_t head_dim;     /* D */
+    int32_t index_dim;    /* d_idx */
+    int32_t block_size;   /* tokens per KV block */
+    int32_t top_k;        /* blocks kept per (query row, group), own block included */
+    int64_t kv_capacity;  /* rows in the packed k_idx / k_cache / v_cache */
+} msa_shape_t;
+
+/* Bytes of workspace msa_index_topk needs for this shape (0 on bad shape). */
+MSA_API size_t msa_index_topk_workspace_size(const msa_shape_t *shape);
+
+/* Index branch: block max-pooled index scores and the top-k block ids of
+ * every (query row, group).  See the header comment for the definition.
+ *   q_idx        device bf16 [B, q_len, H_kv, index_dim]
+ *   k_idx        device bf16 [kv_capacity, H_kv, index_dim]
+ *   lens         device int32 [B], each in [q_len, max_kv_len]
+ *   kv_offsets   device int64 [B], row of token 0 of sequence b
+ *   block_ids    device int32 [B, q_len, H_kv, top_k]   (written)
+ *   block_scores device float [B, q_len, H_kv, top_k]   (written)
+ *   workspace    device, >= msa_index_topk_workspace_size(shape) bytes */
+MSA_API msa_status_t msa_index_topk(const msa_shape_t *shape, const void *q_idx, const void *k_idx,
+                            const int32_t *lens, const int64_t *kv_offsets,
+                            int32_t *block_ids, float *block_scores,
+                            void *workspace, size_t workspace_bytes, msa_stream_t stream);
+
+/* Bytes of workspace msa_sparse_attention needs for this shape (0 on bad shape). */
+MSA_API size_t msa_sparse_attention_workspace_size(const msa_shape_t *shape);
+
+/* Sparse branch: exact softmax attention of every query head over the keys
+ * of its group's kept blocks (ids as written by msa_index_topk; -1 entries
+ * are skipped; every id must be a visible block, the own block included).
+ *   q            device bf16 [B, q_len, H_q, head_dim]
+ *   k_cache      device bf16 [kv_capacity, H_kv, head_dim]
+ *   v_cache      device bf16 [kv_capacity, H_kv, head_dim]
+ *   block_ids    device int32 [B, q_len, H_kv, top_k]
+ *   softmax_scale  multiplies q.k before the softmax (1/sqrt(head_dim) usual)
+ *   out          device bf16 [B, q_len, H_q, head_dim]  (written)
+ *   workspace    device, >= msa_sparse_attention_workspace_size(shape) bytes */
+MSA_API msa_status_t msa_sparse_attention(const msa_shape_t *shape, const void *q, const void *k_cache,
+                                  const void *v_cache, const int32_t *block_ids,
+                                  const int32_t *lens, const int64_t *kv_offsets,
+                                  float softmax_scale, void *out,
+                                  void *workspace, size_t workspace_bytes, msa_stream_t stream);
+
+/* Waits for `stream`, then returns the device status word that the last call
+ * using this workspace left (MSA_OK, MSA_ERR_BAD_LENS or
+ * MSA_ERR_DEVICE_TIMEOUT), or MSA_ERR_CUDA if the wait or copy failed.  Every
+ * call clears the word when it starts. */
+MSA_API msa_status_t msa_read_device_status(const void *workspace, msa_stream_t stream);
+
+/* Kernel timing trace (off by default).  After msa_trace_enable(1), every
+ * call records a pair of CUDA events around each kernel it launches, on that
+ * call's stream, from a pool of events created by msa_trace_enable (up to
+ * 4096 kernels between reads; later launches go unrecorded).
+ * msa_trace_read waits for the recorded events, copies out up to
+ * max_entries records in launch order (kernel name, milliseconds between the
+ * pair) and forgets every record; it returns the number copied, or -1 if a
+ * CUDA call failed.  Names are static strings.  msa_trace_enable(0) stops
+ * recording and drops unread records. */
+MSA_API msa_status_t msa_trace_enable(int on);
+MSA_API int msa_trace_read(const char **names, float *ms, int max_entries);
+
+/* Static, human-readable name of a status code. */
+MSA_API const char *msa_status_string(msa_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H */

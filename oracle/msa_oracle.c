@@ -98,8 +98,8 @@ static int int_cmp(const void *a, const void *b)
     return (x > y) - (x < y);
 }
 
-/* Index branch for one query row, all groups. */
-static void index_row(job_t *J, int64_t rr)
+/* Index branch for one (query row, group). */
+static void index_row(job_t *J, int64_t rr, int g)
 {
     int64_t r = J->rows ? J->rows[rr] : rr;
     int b; int64_t p;
@@ -113,7 +113,7 @@ static void index_row(job_t *J, int64_t rr)
     double *S = (double *)malloc(sizeof(double) * nvis);
     cand_t *c = (cand_t *)malloc(sizeof(cand_t) * (nvis > 0 ? nvis : 1));
     int *sel = (int *)malloc(sizeof(int) * (K + 1));
-    for (int g = 0; g < J->H_kv; ++g) {
+    {
         const uint16_t *qi = J->q_idx + (r * J->H_kv + g) * (int64_t)Di;
         /* Step 1+2: per-token index score (plain dot product of the group's
          * index query with the token's index key, no scale), then the block
@@ -164,10 +164,10 @@ static void index_row(job_t *J, int64_t rr)
     free(S); free(c); free(sel);
 }
 
-/* Sparse branch for one query row, all heads: exact softmax attention over
- * the keys of the selected blocks (causal inside the own block), shared by
- * every head of the group. */
-static void attn_row(job_t *J, int64_t rr)
+/* Sparse branch for one (query row, head): exact softmax attention over the
+ * keys of the selected blocks (causal inside the own block); the block set is
+ * the one of the head's group, shared by every head of the group. */
+static void attn_row(job_t *J, int64_t rr, int h)
 {
     int64_t r = J->rows ? J->rows[rr] : rr;
     int b; int64_t p;
@@ -178,7 +178,7 @@ static void attn_row(job_t *J, int64_t rr)
     int64_t max_keys = (int64_t)K * blk;
     int64_t *keys = (int64_t *)malloc(sizeof(int64_t) * max_keys);
     double *z = (double *)malloc(sizeof(double) * max_keys);
-    for (int h = 0; h < J->H_q; ++h) {
+    {
         const int g = h / G;                 /* contiguous head -> group map */
         const int32_t *ids = J->block_ids_in + (r * J->H_kv + g) * (int64_t)K;
         int64_t nk = 0;
@@ -225,9 +225,13 @@ static void attn_row(job_t *J, int64_t rr)
 static void *worker(void *arg)
 {
     slice_t *s = (slice_t *)arg;
-    for (int64_t rr = s->first; rr < s->job->n_rows; rr += s->stride) {
-        if (s->kind == 0) index_row(s->job, rr);
-        else attn_row(s->job, rr);
+    /* A job is one (row, group) of the index branch or one (row, head) of
+     * the sparse branch; rows are independent, so jobs are too. */
+    const int per = s->kind == 0 ? s->job->H_kv : s->job->H_q;
+    const int64_t n_jobs = s->job->n_rows * per;
+    for (int64_t jb = s->first; jb < n_jobs; jb += s->stride) {
+        if (s->kind == 0) index_row(s->job, jb / per, (int)(jb % per));
+        else attn_row(s->job, jb / per, (int)(jb % per));
     }
     return NULL;
 }
@@ -236,10 +240,13 @@ static int run(job_t *J, int kind, int n_threads)
 {
     if (n_threads < 1) n_threads = 1;
     if (n_threads > 512) n_threads = 512;
-    if (n_threads > J->n_rows) n_threads = (int)(J->n_rows > 0 ? J->n_rows : 1);
+    {
+        int64_t n_jobs = J->n_rows * (kind == 0 ? J->H_kv : J->H_q);
+        if (n_threads > n_jobs) n_threads = (int)(n_jobs > 0 ? n_jobs : 1);
+    }
     pthread_t th[512];
     slice_t sl[512];
-    /* Rows are dealt round-robin so long and short rows spread evenly. */
+    /* Jobs are dealt round-robin so long and short rows spread evenly. */
     for (int t = 0; t < n_threads; ++t) {
         sl[t].job = J; sl[t].kind = kind;
         sl[t].first = t; sl[t].stride = n_threads;

@@ -1,0 +1,97 @@
+"""Shared parity checks: the CUDA library (through its C ABI) against the CPU
+oracle on the same seeded inputs.
+
+Tolerances (written here, used by every GPU test):
+  - block ids: bit-exact, except at a near tie, where the oracle's last kept
+    and first dropped non-own block scores differ by <= 1e-5 relative; there
+    the kept sets may differ in that one slot, and the outputs are compared
+    with the oracle run on the GPU's own selection;
+  - block scores: |gpu - oracle| <= 1e-5 * max(|oracle|, 1) (fp32 sums of
+    128 exact bf16 products against a double sum);
+  - outputs (bf16): max-abs <= 2e-2 and relative L2 <= 5e-3 against the
+    oracle's double result.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import block_sparse_attention_43_b200 as msa
+from synthetic import bf16_bits
+
+NEAR_TIE_REL = 1e-5
+SCORE_REL = 1e-5
+OUT_MAX_ABS = 2e-2
+OUT_REL_L2 = 5e-3
+
+
+def run_gpu(w, *, stream=None):
+    """Both stages through the C ABI on the workload's device tensors."""
+    m = msa.MSA(batch=w.B, q_len=w.Sq, max_kv_len=max(w.lens_host), num_q_heads=w.H_q,
+                num_kv_heads=w.H_kv, top_k=w.top_k, kv_capacity=w.kv_capacity, device=w.q.device)
+    m.index_topk(w.q_idx, w.k_idx, w.lens, w.kv_offsets, stream)
+    m.sparse_attention(w.q, w.k, w.v, w.lens, w.kv_offsets, stream=stream)
+    torch.cuda.synchronize()
+    st = m.device_status()
+    return m, st
+
+
+def host_inputs(w):
+    return dict(q_idx=bf16_bits(w.q_idx), k_idx=bf16_bits(w.k_idx), q=bf16_bits(w.q),
+                k=bf16_bits(w.k), v=bf16_bits(w.v), lens=w.lens.cpu().numpy(),
+                kv_offsets=w.kv_offsets.cpu().numpy())
+
+
+def compare(oracle_mod, w, gpu_ids, gpu_scores, gpu_out, rows=None, host=None):
+    """Checks one run against the oracle on `rows` (flattened b*Sq+i; None = all).
+    Returns a small report dict; raises AssertionError on a mismatch."""
+    a = host if host is not None else host_inputs(w)
+    R = w.B * w.Sq
+    rows_a = np.arange(R, dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
+    ref = oracle_mod.index_topk(a["q_idx"], a["k_idx"], a["lens"], a["kv_offsets"],
+                                block=w.block, top_k=w.top_k, rows=rows_a)
+    g_ids = gpu_ids.reshape(R, w.H_kv, w.top_k)[rows_a]
+    g_sc = gpu_scores.reshape(R, w.H_kv, w.top_k)[rows_a]
+    o_ids, o_sc, bnd = ref["block_ids"], ref["block_scores"], ref["boundary"]
+
+    same = (g_ids == o_ids).all(axis=-1)
+    ties = 0
+    for r, g in zip(*np.nonzero(~same)):
+        last_in, first_out = bnd[r, g]
+        gap = abs(last_in - first_out)
+        tol = NEAR_TIE_REL * max(abs(last_in), abs(first_out))
+        assert np.isfinite(first_out) and gap <= tol, (
+            f"block ids differ at row {rows_a[r]} group {g}: gpu {g_ids[r, g].tolist()} "
+            f"oracle {o_ids[r, g].tolist()} (boundary {last_in} vs {first_out})")
+        diff = set(g_ids[r, g].tolist()) ^ set(o_ids[r, g].tolist())
+        assert len(diff) == 2, (rows_a[r], g, diff)
+        ties += 1
+    # Scores of the ids both sides kept.
+    m = same[..., None] & (o_ids >= 0)
+    err = np.abs(g_sc[m].astype(np.float64) - o_sc[m].astype(np.float64))
+    lim = SCORE_REL * np.maximum(np.abs(o_sc[m].astype(np.float64)), 1.0)
+    assert (err <= lim).all(), f"block scores off by up to {err.max()}"
+    assert (g_sc[~(o_ids >= 0) & same[..., None]] == -np.inf).all()
+
+    # Outputs: oracle attention on the GPU's own selection (identical to the
+    # oracle's except at near ties).
+    full_ids = np.full((R, w.H_kv, w.top_k), -1, np.int32)
+    full_ids[rows_a] = g_ids
+    o_out = oracle_mod.sparse_attention(a["q"], a["k"], a["v"], full_ids, a["lens"],
+                                        a["kv_offsets"], block=w.block, scale=w.scale, rows=rows_a)
+    g_out = gpu_out.reshape(R, w.H_q, w.D)[rows_a].astype(np.float64)
+    assert np.isfinite(g_out).all(), "non-finite output"
+    d = np.abs(g_out - o_out)
+    max_abs = float(d.max())
+    rel_l2 = float(np.linalg.norm(g_out - o_out) / max(np.linalg.norm(o_out), 1e-30))
+    assert max_abs <= OUT_MAX_ABS, f"max-abs {max_abs}"
+    assert rel_l2 <= OUT_REL_L2, f"rel-L2 {rel_l2}"
+    return dict(rows=len(rows_a), near_ties=ties, max_abs=max_abs, rel_l2=rel_l2,
+                score_err=float(err.max()) if err.size else 0.0)
+
+
+def to_host(m):
+    ids = m.block_ids.cpu().numpy()
+    sc = m.block_scores.cpu().numpy()
+    out = m.out.float().cpu().numpy()
+    return ids, sc, out

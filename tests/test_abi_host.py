@@ -1,0 +1,87 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/msa.h declares, sizes workspaces, and rejects bad
+arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def m():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_msa_build", os.path.join(ROOT, "block_sparse_attention_43_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    b.build()
+    import block_sparse_attention_43_b200 as mod
+    return mod
+
+
+def _declared():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", f)).read()
+            names |= set(re.findall(r"MSA_API\s+[\w\s\*]*?\b(msa_\w+)\s*\(", txt))
+    return names
+
+
+def test_every_declared_symbol_is_exported(m):
+    decl = _declared()
+    assert {"msa_index_topk", "msa_sparse_attention"} <= decl
+    lib = ctypes.CDLL(m.LIB_PATH)
+    for name in decl:
+        assert hasattr(lib, name), name
+    assert decl == set(m.EXPORTS)
+
+
+def _shape(m, **kw):
+    base = dict(batch=4, q_len=1, max_kv_len=1 << 20, num_q_heads=64, num_kv_heads=8, top_k=16,
+                kv_capacity=4 << 20)
+    base.update(kw)
+    return m.make_shape(**base)
+
+
+def test_workspace_sizes(m):
+    s = _shape(m)
+    nb = (1 << 20) // 128
+    assert m.msa_index_topk_workspace_size(s) == 256 + 4 * 8 * nb * 4
+    assert m.msa_sparse_attention_workspace_size(s) > 256
+    assert m.msa_index_topk_workspace_size(_shape(m, head_dim=64)) == 0
+    assert m.msa_index_topk_workspace_size(_shape(m, num_q_heads=63)) == 0
+    assert m.msa_sparse_attention_workspace_size(_shape(m, top_k=65)) == 0
+
+
+def _call_index(m, s, ptrs, ws=0x100000, wsb=1 << 40):
+    P = ctypes.c_void_p
+    return m.lib.msa_index_topk(ctypes.byref(s), *[P(x) for x in ptrs], P(ws), wsb, None)
+
+
+def test_bad_arguments_are_rejected_before_launch(m):
+    s = _shape(m)
+    good = [0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 0x60000]
+    assert _call_index(m, s, [0] + good[1:]) == 1                 # null q_idx
+    assert _call_index(m, s, [0x10001] + good[1:]) == 7           # misaligned q_idx
+    assert _call_index(m, s, good, ws=0x100010) == 3              # misaligned workspace
+    assert _call_index(m, s, good, wsb=100) == 3                  # short workspace
+    assert _call_index(m, _shape(m, block_size=64), good) == 2
+    assert _call_index(m, _shape(m, num_kv_heads=3, num_q_heads=9), good) == 2
+    assert _call_index(m, _shape(m, q_len=0), good) == 1
+    assert _call_index(m, _shape(m, q_len=10, max_kv_len=5), good) == 1
+    P = ctypes.c_void_p
+    r = m.lib.msa_sparse_attention(ctypes.byref(s), P(0x10000), P(0x20000), P(0x30000),
+                                   P(0x40000), P(0x50000), P(0x60000), ctypes.c_float(float("nan")),
+                                   P(0x70000), P(0x100000), 1 << 40, None)
+    assert r == 1
+    assert m.lib.msa_read_device_status(None, None) == 1
+
+
+def test_status_strings(m):
+    for code in range(8):
+        assert m.msa_status_string(code).startswith(m.STATUS_NAMES[code])
+    assert m.msa_status_string(99) == "MSA_ERR_UNKNOWN"
