@@ -24,7 +24,8 @@ STATUS_NAMES = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
 # Every entry point include/msa.h declares.
 EXPORTS = ("msa_index_topk_workspace_size", "msa_index_topk",
            "msa_sparse_attention_workspace_size", "msa_sparse_attention",
-           "msa_read_device_status", "msa_trace_enable", "msa_trace_read",
+           "msa_index_topk_static", "msa_read_device_status", "msa_trace_enable",
+           "msa_trace_read",
            "msa_status_string")
 
 
@@ -56,6 +57,8 @@ def _load():
     lib.msa_index_topk.restype = ctypes.c_int
     lib.msa_sparse_attention.argtypes = [S, P, P, P, P, P, P, ctypes.c_float, P, P, Z, P]
     lib.msa_sparse_attention.restype = ctypes.c_int
+    lib.msa_index_topk_static.argtypes = [S, P, P, P, P, P, P, P]
+    lib.msa_index_topk_static.restype = ctypes.c_int
     lib.msa_read_device_status.argtypes = [P, P]
     lib.msa_read_device_status.restype = ctypes.c_int
     lib.msa_trace_enable.argtypes = [ctypes.c_int]
@@ -122,6 +125,16 @@ def msa_sparse_attention(shape, q, k_cache, v_cache, block_ids, lens, kv_offsets
                                     float(softmax_scale), _ptr(out), _ptr(workspace),
                                     workspace.numel(), _stream(stream)),
            "msa_sparse_attention")
+
+
+def msa_index_topk_static(shape, q_idx, k_idx, lens, kv_offsets, block_ids, block_scores,
+                          stream=None) -> None:
+    """Index branch with the library's fixed device scratch instead of a
+    workspace (for callers that cannot allocate); see include/msa.h."""
+    _check(lib.msa_index_topk_static(ctypes.byref(shape), _ptr(q_idx), _ptr(k_idx), _ptr(lens),
+                                     _ptr(kv_offsets), _ptr(block_ids), _ptr(block_scores),
+                                     _stream(stream)),
+           "msa_index_topk_static")
 
 
 def msa_read_device_status(workspace, stream=None) -> int:

@@ -133,6 +133,30 @@ MSA_API msa_status_t msa_sparse_attention(const msa_shape_t *shape, const void *
                                   float softmax_scale, void *out,
                                   void *workspace, size_t workspace_bytes, msa_stream_t stream);
 
+/* msa_index_topk without a workspace argument, for callers that cannot
+ * allocate device memory or hand over a workspace (plugin hosts that pass a
+ * kernel only its inputs and outputs, processes whose device memory belongs
+ * to another allocator, loops that must not stall on cudaMalloc).  The paper
+ * has no counterpart; this is a library convenience.
+ *   Scratch: a file-scope device array of 256 B + 4 MiB that every GPU which
+ *   loads the library holds until the process exits.  Shapes whose
+ *   msa_index_topk_workspace_size exceeds that (batch * q_len * num_kv_heads
+ *   * ceil(max_kv_len / 128) > 1,048,576 block scores) are rejected with
+ *   MSA_ERR_WORKSPACE; nothing is launched and nothing is allocated.
+ *   Set-up: the first call on each device looks up the array's device
+ *   address with cudaGetSymbolAddress (that device must be current); make
+ *   that first call before any stream capture.
+ *   Sharing: every call on a device uses the same array and it keeps the last
+ *   call's contents; calls that may overlap on the GPU (different streams,
+ *   no ordering) race on it and must be serialised by the caller.
+ *   Device-detected errors leave -1 / -inf in the outputs; the status word
+ *   stays inside the library's array and is not reported by this call.
+ * Other arguments, layouts and results are those of msa_index_topk. */
+MSA_API msa_status_t msa_index_topk_static(const msa_shape_t *shape, const void *q_idx,
+                                           const void *k_idx, const int32_t *lens,
+                                           const int64_t *kv_offsets, int32_t *block_ids,
+                                           float *block_scores, msa_stream_t stream);
+
 /* Waits for `stream`, then returns the device status word that the last call
  * using this workspace left (MSA_OK, MSA_ERR_BAD_LENS or
  * MSA_ERR_DEVICE_TIMEOUT), or MSA_ERR_CUDA if the wait or copy failed.  Every
