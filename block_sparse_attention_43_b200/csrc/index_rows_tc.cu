@@ -1,0 +1,277 @@
+// index_rows_tc.cu -- MSA index branch for prefill on the fifth-generation
+// tensor cores: block max-pooled causal index scores as a tiled bf16 GEMM.
+//
+// Method: "百万token上下文提速近10倍，MiniMax M3的稀疏注意力凭什么这么快"
+// (cloud.tencent.com), section 二 -- one index query per GQA group dotted with
+// the index keys of every visible token, "Block Max Pool" per 128-token KV
+// block.  For q_len query rows this is, per (sequence, group), the causal
+// product Q_idx (rows x 128) . K_idx^T (128 x tokens) reduced by a max over
+// each 128-column block: a real dense contraction, so it runs on tcgen05.
+//
+// Tiling: a work unit is (sequence, group, 128 query rows).  The unit's index
+// queries (32 KiB) sit in shared memory; its visible key blocks stream through
+// a 3-stage ring two blocks (64 KiB) at a time.  One thread issues
+// tcgen05.mma kind::f16 M=128, N=256 (or 128 for a lone last block), K=128 as
+// eight K=16 steps into one of two 256-column fp32 TMEM accumulators, and
+// commits to mbarriers.  Four epilogue warps (one TMEM lane = one query row
+// per thread) read the accumulator with tcgen05.ld, apply the causal mask
+// where the block reaches past the row's position and write one block score
+// per (row, block).  Units are dealt to a persistent grid in snake order of
+// decreasing length.
+//
+// Roles: warp 0 = TMA producer, warp 1 = MMA issuer, warp 2 = TMEM owner,
+// warps 4-7 = epilogue (warp % 4 selects its 32 TMEM lanes).
+#include "msa_device.cuh"
+#include "msa_internal.h"
+
+namespace msa {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kStages = 3;
+constexpr int kQBytes = 2 * 16384;          // 128 rows x 128 dims, two swizzled halves
+constexpr int kStageBytes = 2 * 32768;      // two key blocks: [256 rows x 128 B] per half
+constexpr uint32_t kTmemCols = 512;         // two 256-column accumulators
+
+struct Smem {
+    uint8_t q[kQBytes];
+    uint8_t ring[kStages][kStageBytes];
+    uint64_t k_full[kStages], k_empty[kStages];
+    uint64_t q_full, q_empty;
+    uint64_t acc_full[2], acc_empty[2];
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+struct Unit {
+    int b, g, i0, nrows, L;
+    long long off, p_first;
+    int jmax;        // last visible key block of the tile
+    bool valid;
+};
+
+__device__ __forceinline__ Unit unit_at(const IndexRowsArgs &P, long long u, int ntiles) {
+    // Unit u -> (query tile, counted from the last one, sequence, group).
+    Unit x;
+    const long long per_tile = static_cast<long long>(P.B) * P.H_kv;
+    const int t = ntiles - 1 - static_cast<int>(u / per_tile);
+    const int rem = static_cast<int>(u % per_tile);
+    x.b = rem / P.H_kv;
+    x.g = rem % P.H_kv;
+    x.i0 = t * 128;
+    x.nrows = min(128, P.Sq - x.i0);
+    x.L = P.lens[x.b];
+    x.off = P.kv_offsets[x.b];
+    x.valid = x.L >= P.Sq && x.L >= 1 && x.L <= P.max_kv_len && x.off >= 0 &&
+              x.off + x.L <= P.capacity;
+    x.p_first = static_cast<long long>(x.L) - P.Sq + x.i0;
+    x.jmax = x.valid ? static_cast<int>((x.p_first + x.nrows - 1) / kBlock) : -1;
+    return x;
+}
+
+// The r-th unit of this CTA in snake order over rounds of gridDim.x units.
+__device__ __forceinline__ long long unit_index(int r) {
+    const long long G = gridDim.x;
+    const long long c = (r & 1) ? (G - 1 - blockIdx.x) : blockIdx.x;
+    return static_cast<long long>(r) * G + c;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    index_rows_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                         const __grid_constant__ CUtensorMap tmK, const IndexRowsArgs P) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem &S = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                        ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ntiles = (P.Sq + 127) / 128;
+    const long long nunits = static_cast<long long>(ntiles) * P.B * P.H_kv;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&S.k_full[s], 1);
+            mbar_init(&S.k_empty[s], 1);
+        }
+        mbar_init(&S.q_full, 1);
+        mbar_init(&S.q_empty, 1);
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&S.acc_full[a], 1);
+            mbar_init(&S.acc_empty[a], 4);
+        }
+        S.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 2) {
+        tmem_alloc(&S.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+    volatile int *abort_flag = &S.abort_flag;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------ TMA producer
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmK);
+        int itk = 0, nq = 0;
+        bool ok = true;
+        for (int r = 0; ok; ++r) {
+            const long long u = unit_index(r);
+            if (u >= nunits) break;
+            const Unit x = unit_at(P, u, ntiles);
+            if (!x.valid) {
+                if (x.i0 == 0 && x.g == 0) set_status(P.status, kStatusBadLens);
+                continue;
+            }
+            if (nq > 0 && (*abort_flag || !mbar_wait(&S.q_empty, (nq - 1) & 1, P.status))) {
+                ok = false;
+                break;
+            }
+            const int qrow = x.b * P.Sq + x.i0;
+            mbar_arrive_expect_tx(&S.q_full, kQBytes);
+            tma_load_3d(S.q, &tmQ, 0, x.g, qrow, &S.q_full);
+            tma_load_3d(S.q + 16384, &tmQ, 64, x.g, qrow, &S.q_full);
+            ++nq;
+            for (int j = 0; j <= x.jmax; j += 2, ++itk) {
+                const int s = itk % kStages;
+                if (itk >= kStages &&
+                    (*abort_flag || !mbar_wait(&S.k_empty[s], ((itk / kStages) - 1) & 1, P.status))) {
+                    ok = false;
+                    break;
+                }
+                const int nb = min(2, x.jmax - j + 1);
+                mbar_arrive_expect_tx(&S.k_full[s], nb * 32768);
+                for (int jj = 0; jj < nb; ++jj) {
+                    const int tok = static_cast<int>(x.off + (long long)(j + jj) * kBlock);
+                    tma_load_3d(S.ring[s] + jj * 16384, &tmK, 0, x.g, tok, &S.k_full[s]);
+                    tma_load_3d(S.ring[s] + 32768 + jj * 16384, &tmK, 64, x.g, tok, &S.k_full[s]);
+                }
+            }
+        }
+        if (!ok) *abort_flag = 1;
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------ MMA issuer
+        int itk = 0, ita = 0, nq = 0;
+        bool ok = true;
+        for (int r = 0; ok; ++r) {
+            const long long u = unit_index(r);
+            if (u >= nunits) break;
+            const Unit x = unit_at(P, u, ntiles);
+            if (!x.valid) continue;
+            if (*abort_flag || !mbar_wait(&S.q_full, nq & 1, P.status)) { ok = false; break; }
+            ++nq;
+            tc_fence_after();
+            const uint32_t qa = smem_u32(S.q);
+            for (int j = 0; j <= x.jmax; j += 2, ++itk, ++ita) {
+                const int s = itk % kStages, a = ita & 1;
+                if (*abort_flag || !mbar_wait(&S.k_full[s], (itk / kStages) & 1, P.status)) {
+                    ok = false;
+                    break;
+                }
+                if (ita >= 2 && (*abort_flag || !mbar_wait(&S.acc_empty[a], ((ita >> 1) - 1) & 1,
+                                                           P.status))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int nb = min(2, x.jmax - j + 1);
+                const uint32_t idesc = umma_idesc_bf16(128, nb * 128);
+                const uint32_t kb = smem_u32(S.ring[s]);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t ad = umma_desc_sw128(qa + (kk >> 2) * 16384 + (kk & 3) * 32);
+                    const uint64_t bd = umma_desc_sw128(kb + (kk >> 2) * 32768 + (kk & 3) * 32);
+                    umma_bf16_ss(tmem + a * 256, ad, bd, idesc, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&S.k_empty[s]);
+                umma_commit(&S.acc_full[a]);
+                if (j + 2 > x.jmax) umma_commit(&S.q_empty);
+            }
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            // Let every MMA already issued finish before TMEM is released.
+            if (ita > 0) mbar_wait(&S.acc_full[(ita - 1) & 1], ((ita - 1) >> 1) & 1, nullptr);
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------ epilogue
+        const int r = tid - 128;                     // TMEM lane = tile row
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        int ita = 0;
+        bool ok = true;
+        for (int rr = 0; ok; ++rr) {
+            const long long u = unit_index(rr);
+            if (u >= nunits) break;
+            const Unit x = unit_at(P, u, ntiles);
+            if (!x.valid) continue;
+            const long long p = x.p_first + r;        // this row's query position
+            const int own = static_cast<int>(p / kBlock);
+            const bool row_ok = r < x.nrows;
+            float *dst = P.scores + ((static_cast<long long>(x.b) * P.Sq + x.i0 + r) * P.H_kv + x.g) *
+                                        static_cast<long long>(P.nb_max);
+            for (int j = 0; j <= x.jmax; j += 2, ++ita) {
+                const int a = ita & 1;
+                bool have = !*abort_flag && mbar_wait(&S.acc_full[a], (ita >> 1) & 1, P.status);
+                have = __all_sync(0xffffffffu, have);
+                if (!have) { ok = false; break; }
+                tc_fence_after();
+                const int nb = min(2, x.jmax - j + 1);
+                for (int jj = 0; jj < nb; ++jj) {
+                    const int J = j + jj;
+                    const long long t0 = static_cast<long long>(J) * kBlock;
+                    const bool full = t0 + kBlock - 1 <= x.p_first;     // no masking for any row
+                    float m = -INFINITY;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        float v[32];
+                        tmem_ld32(lane_addr + a * 256 + jj * 128 + c * 32, v);
+                        tmem_ld_wait();
+                        if (full) {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) m = fmaxf(m, v[e]);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                if (t0 + c * 32 + e <= p) m = fmaxf(m, v[e]);
+                        }
+                    }
+                    if (row_ok && J <= own) dst[J] = m;
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.acc_empty[a]);
+            }
+        }
+        if (!ok) *abort_flag = 1;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_index_rows_tc(const IndexRowsArgs &a, cudaStream_t s) {
+    static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "shared memory budget");
+    CUtensorMap tq, tk;
+    if (!encode_kv_tensor_map(&tq, a.q_idx, a.H_kv, static_cast<long long>(a.B) * a.Sq) ||
+        !encode_kv_tensor_map(&tk, a.k_idx, a.H_kv, a.capacity))
+        return cudaErrorInvalidValue;
+    const size_t smem = sizeof(Smem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(index_rows_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const long long ntiles = (a.Sq + 127) / 128;
+    const long long units = ntiles * a.B * a.H_kv;
+    const long long grid = units < device_sm_count() ? units : device_sm_count();
+    TraceScope trace(s, "index_score_maxpool_rows_tc");
+    index_rows_tc_kernel<<<static_cast<unsigned>(grid), kThreads, smem, s>>>(tq, tk, a);
+    return cudaGetLastError();
+}
+
+}  // namespace msa

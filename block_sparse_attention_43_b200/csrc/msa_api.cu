@@ -168,7 +168,7 @@ msa_status_t msa_index_topk(const msa_shape_t *shape, const void *q_idx, const v
         a.scores = scores; a.status = status;
         a.B = shape->batch; a.Sq = shape->q_len; a.H_kv = shape->num_kv_heads; a.nb_max = nb_max;
         a.max_kv_len = shape->max_kv_len; a.capacity = shape->kv_capacity;
-        e = launch_index_rows_simt(a, s);
+        e = launch_index_rows_tc(a, s);
     }
     if (e != cudaSuccess) return MSA_ERR_CUDA;
     TopkArgs t;

@@ -51,8 +51,7 @@ struct IndexRowsArgs {
     int B, Sq, H_kv, nb_max, max_kv_len;
     long long capacity;
 };
-cudaError_t launch_index_rows_simt(const IndexRowsArgs &a, cudaStream_t s);
-// Same contract, tcgen05 tensor-core path.
+// tcgen05 tensor-core kernel (index_rows_tc.cu).
 cudaError_t launch_index_rows_tc(const IndexRowsArgs &a, cudaStream_t s);
 
 // Top-k block selection per (row, group) from a block-score buffer.

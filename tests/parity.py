@@ -42,9 +42,9 @@ def host_inputs(w):
                 kv_offsets=w.kv_offsets.cpu().numpy())
 
 
-def compare(oracle_mod, w, gpu_ids, gpu_scores, gpu_out, rows=None, host=None):
-    """Checks one run against the oracle on `rows` (flattened b*Sq+i; None = all).
-    Returns a small report dict; raises AssertionError on a mismatch."""
+def compare_index(oracle_mod, w, gpu_ids, gpu_scores, rows=None, host=None):
+    """Block ids and scores of `rows` (flattened b*Sq+i; None = all) against
+    the oracle's index branch.  Returns (rows, gpu ids of those rows, report)."""
     a = host if host is not None else host_inputs(w)
     R = w.B * w.Sq
     rows_a = np.arange(R, dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
@@ -72,6 +72,16 @@ def compare(oracle_mod, w, gpu_ids, gpu_scores, gpu_out, rows=None, host=None):
     lim = SCORE_REL * np.maximum(np.abs(o_sc[m].astype(np.float64)), 1.0)
     assert (err <= lim).all(), f"block scores off by up to {err.max()}"
     assert (g_sc[~(o_ids >= 0) & same[..., None]] == -np.inf).all()
+    return rows_a, g_ids, dict(rows=len(rows_a), near_ties=ties,
+                               score_err=float(err.max()) if err.size else 0.0)
+
+
+def compare(oracle_mod, w, gpu_ids, gpu_scores, gpu_out, rows=None, host=None):
+    """Checks one run (ids, scores, outputs) against the oracle on `rows`.
+    Returns a small report dict; raises AssertionError on a mismatch."""
+    a = host if host is not None else host_inputs(w)
+    R = w.B * w.Sq
+    rows_a, g_ids, rep = compare_index(oracle_mod, w, gpu_ids, gpu_scores, rows=rows, host=a)
 
     # Outputs: oracle attention on the GPU's own selection (identical to the
     # oracle's except at near ties).
@@ -86,8 +96,16 @@ def compare(oracle_mod, w, gpu_ids, gpu_scores, gpu_out, rows=None, host=None):
     rel_l2 = float(np.linalg.norm(g_out - o_out) / max(np.linalg.norm(o_out), 1e-30))
     assert max_abs <= OUT_MAX_ABS, f"max-abs {max_abs}"
     assert rel_l2 <= OUT_REL_L2, f"rel-L2 {rel_l2}"
-    return dict(rows=len(rows_a), near_ties=ties, max_abs=max_abs, rel_l2=rel_l2,
-                score_err=float(err.max()) if err.size else 0.0)
+    rep.update(max_abs=max_abs, rel_l2=rel_l2)
+    return rep
+
+
+def sample_rows(n, count, seed):
+    """`count` seeded distinct rows of [0, n) plus the block-edge rows."""
+    g = np.random.default_rng(seed)
+    pick = set(g.choice(n, size=min(count, n), replace=False).tolist())
+    pick |= {x for x in (0, 1, 127, 128, 129, 2047, 2048, n - 1) if 0 <= x < n}
+    return np.array(sorted(pick), np.int64)
 
 
 def to_host(m):

@@ -84,6 +84,25 @@ def test_named_workload_full_parity(msa_lib, oracle_mod, name):
     print(name, rep)
 
 
+def test_prefill_128k_index_sampled_rows(msa_lib, oracle_mod):
+    """128k-token prefill, index branch at full size on the GPU (tcgen05
+    path), 4096 seeded rows plus block-edge rows checked against the oracle."""
+    import block_sparse_attention_43_b200 as m
+    from parity import compare_index, sample_rows
+    from synthetic import bf16_bits, make_workload
+    w = make_workload("prefill_128k", DEV)
+    eng = m.MSA(batch=1, q_len=w.Sq, max_kv_len=w.Sq, num_q_heads=w.H_q, num_kv_heads=w.H_kv,
+                top_k=w.top_k, kv_capacity=w.kv_capacity, device=DEV)
+    eng.index_topk(w.q_idx, w.k_idx, w.lens, w.kv_offsets)
+    assert m.msa_read_device_status(eng.ws_index) == 0
+    host = dict(q_idx=bf16_bits(w.q_idx), k_idx=bf16_bits(w.k_idx), lens=w.lens.cpu().numpy(),
+                kv_offsets=w.kv_offsets.cpu().numpy())
+    rows = sample_rows(w.Sq, 4096, seed=2)
+    _, _, rep = compare_index(oracle_mod, w, eng.block_ids.cpu().numpy(),
+                              eng.block_scores.cpu().numpy(), rows=rows, host=host)
+    print("prefill_128k index", rep)
+
+
 def test_repeat_calls_are_bit_identical(msa_lib):
     from parity import run_gpu, to_host
     from synthetic import make_inputs
