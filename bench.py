@@ -1,9 +1,11 @@
 """Benchmark of the MSA hot path on B200: one step = the whole decode path
 (index score + block max-pool, top-k, sparse attention with split-K merge)
-for one batch, through the C ABI.
+for one batch, through the C ABI; a decode run also times one 128k-token
+prefill (index GEMM + fused top-k, sparse attention) as a sub-object.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode_1m]
                     [--impl msa|reference] [--no-cpu-baseline] [--no-e2e]
+                    [--no-prefill] [--prefill-steps S] [--prefill-len N]
 
 Prints ONE JSON line (rank 0).  N > 1 runs under torchrun: every rank runs
 its own independent batch (weak scaling, no data-path collective).
@@ -38,10 +40,16 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="decode_1m",
-                    choices=["decode_1m", "decode_32k", "decode_ragged"])
+                    choices=["decode_1m", "decode_32k", "decode_ragged", "prefill_128k",
+                             "prefill_2k"])
     ap.add_argument("--impl", default="msa", choices=["msa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the prefill_128k measurement attached to a decode run")
+    ap.add_argument("--prefill-steps", type=int, default=5)
+    ap.add_argument("--prefill-len", type=int, default=None,
+                    help="override the prefill length (profiling captures of a smaller case)")
     return ap.parse_args()
 
 
@@ -69,6 +77,85 @@ def index_kernel_bytes(w):
     lens = np.asarray(w.lens_host, np.int64)
     nb = (lens + 127) // 128
     return int(lens.sum()) * w.H_kv * w.d_idx * 2 + w.B * w.H_kv * w.d_idx * 2 + int(nb.sum()) * w.H_kv * 4
+
+
+def prefill_useful_flops(w, ids_host):
+    """Useful sparse-branch FLOPs: 4*D per (row, head, visible kept key)."""
+    ids = ids_host.reshape(w.B, w.Sq, w.H_kv, w.top_k).astype(np.int64)
+    keys = 0
+    for b in range(w.B):
+        L = w.lens_host[b]
+        p = np.arange(w.Sq, dtype=np.int64) + (L - w.Sq)
+        own = p // 128
+        idb = ids[b]
+        vis = np.where(idb == own[:, None, None], (p % 128 + 1)[:, None, None], 128)
+        keys += int((vis * (idb >= 0)).sum())
+    return keys * (w.H_q // w.H_kv) * 4 * w.D
+
+
+def prefill_index_flops(w):
+    """Index-branch FLOPs of the causal product: 2*d_idx per (row, group, visible token)."""
+    f = 0
+    for b in range(w.B):
+        L = w.lens_host[b]
+        p = np.arange(w.Sq, dtype=np.int64) + (L - w.Sq)
+        f += int((p + 1).sum())
+    return f * w.H_kv * 2 * w.d_idx
+
+
+def measure_prefill(name, dev, steps, warmup, seq_len=None):
+    """Times msa_index_topk + msa_sparse_attention on a prefill workload;
+    per-kernel times come from the library's CUDA-event trace."""
+    import block_sparse_attention_43_b200 as msa
+    from synthetic import WORKLOADS, make_inputs, make_workload
+    if seq_len is None:
+        w = make_workload(name, dev)
+    else:
+        c = WORKLOADS[name]
+        w = make_inputs(B=c["B"], Sq=seq_len, lens=[seq_len] * c["B"], H_q=c["H_q"],
+                        H_kv=c["H_kv"], top_k=c["top_k"], seed=c["seed"], device=dev,
+                        name=f"{name}@{seq_len}")
+    stream = torch.cuda.Stream(device=dev)
+    eng = msa.MSA(batch=w.B, q_len=w.Sq, max_kv_len=max(w.lens_host), num_q_heads=w.H_q,
+                  num_kv_heads=w.H_kv, top_k=w.top_k, kv_capacity=w.kv_capacity, device=dev)
+
+    def step():
+        eng.index_topk(w.q_idx, w.k_idx, w.lens, w.kv_offsets, stream)
+        eng.sparse_attention(w.q, w.k, w.v, w.lens, w.kv_offsets, stream=stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    st = eng.device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"prefill device status {msa.STATUS_NAMES.get(st, st)}")
+    useful = prefill_useful_flops(w, eng.block_ids.cpu().numpy())
+    idx_flops = prefill_index_flops(w)
+    msa.msa_trace_enable(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    trace = msa.msa_trace_read()
+    msa.msa_trace_enable(False)
+    ms_step = ev0.elapsed_time(ev1) / steps
+    per = {}
+    for n, t in trace:
+        per[n] = per.get(n, 0.0) + t / steps
+    idx_ms = sum(t for n, t in per.items() if n.startswith("index_"))
+    att_ms = sum(t for n, t in per.items() if n.startswith("prefill_") or n.startswith("sparse_"))
+    res = {"workload": w.name, "rows": w.B * w.Sq, "H_q": w.H_q, "H_kv": w.H_kv,
+           "top_k": w.top_k, "ms_per_step": ms_step,
+           "sparse_attn_useful_tflop": useful / 1e12,
+           "sparse_attn_ms": att_ms, "sparse_attn_tflops": useful / (att_ms / 1e3) / 1e12,
+           "index_tflop": idx_flops / 1e12, "index_ms": idx_ms,
+           "index_tflops": idx_flops / (idx_ms / 1e3) / 1e12,
+           "kernel_ms": per, "gpu_launches_per_step": len(trace) / steps}
+    del eng, w
+    torch.cuda.empty_cache()
+    return res
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -127,11 +214,13 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- helpers
 def measured_peaks():
+    """(HBM GB/s, bf16 burst TFLOP/s, bf16 sustained TFLOP/s, source)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return float(d["hbm_gbs"]), "measured"
-    return 6650.0, "fallback"
+        return (float(d["hbm_gbs"]), float(d["bf16_tflops"]),
+                float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured")
+    return 6650.0, 1590.0, 1400.0, "fallback"
 
 
 def kernel_traffic():
@@ -229,6 +318,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload.startswith("prefill"):
+        return run_prefill_headline(args)
     import block_sparse_attention_43_b200 as msa
     from synthetic import make_workload
 
@@ -304,7 +395,18 @@ def main():
         cpu = {"value": gbs, "unit": "GB/s", "cores": used, "kind": "oracle", "sample": note,
                "seconds": dt}
 
-    peak, peak_kind = measured_peaks()
+    prefill = None
+    if not args.no_prefill and world == 1:
+        del eng
+        torch.cuda.empty_cache()
+        prefill = measure_prefill("prefill_128k", dev, args.prefill_steps, 2)
+        _, tf_burst, tf_sus, _ = measured_peaks()
+        prefill["roofline"] = {"bound": "tensor", "unit": "TFLOP/s",
+                               "sparse_attn_frac_of_burst": prefill["sparse_attn_tflops"] / tf_burst,
+                               "index_frac_of_burst": prefill["index_tflops"] / tf_burst,
+                               "peak_burst": tf_burst, "peak_sustained": tf_sus}
+
+    peak, _, _, peak_kind = measured_peaks()
     kb = index_kernel_bytes(w)
     achieved = kb / (dom_ms / 1e3) / 1e9
     tr = kernel_traffic()
@@ -331,7 +433,38 @@ def main():
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "prefill_128k": prefill,
         }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def run_prefill_headline(args):
+    """--workload prefill_*: the step is one full prefill (index + sparse
+    branch); the value is the sparse branch's useful TFLOP/s."""
+    dist, rank, local, world = dist_setup(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    r = measure_prefill(args.workload, dev, args.steps, max(args.warmup, 1), args.prefill_len)
+    clk = clocks.stop()
+    _, tf_burst, tf_sus, kind = measured_peaks()
+    if rank == 0:
+        line = {"metric": METRIC, "value": r["sparse_attn_tflops"], "unit": "TFLOP/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": r["workload"], "rows": r["rows"], "H_q": r["H_q"],
+                           "H_kv": r["H_kv"], "top_k": r["top_k"],
+                           "l2": "inputs larger than L2"},
+                "roofline": {"bound": "tensor", "kernel": "prefill_attn_kv_outer",
+                             "achieved": r["sparse_attn_tflops"], "peak": tf_burst,
+                             "peak_kind": kind + " burst", "unit": "TFLOP/s",
+                             "frac": r["sparse_attn_tflops"] / tf_burst, "traffic": None},
+                "prefill": r, "clocks": clk, "gpu_launches": int(r["gpu_launches_per_step"] * args.steps),
+                "e2e": None, "cpu_baseline": None}
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()

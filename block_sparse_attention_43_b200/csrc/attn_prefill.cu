@@ -1,0 +1,758 @@
+// attn_prefill.cu -- MSA sparse branch for prefill (many query rows), on the
+// fifth-generation tensor cores, organised around the KV blocks.
+//
+// Method: "百万token上下文提速近10倍，MiniMax M3的稀疏注意力凭什么这么快"
+// (cloud.tencent.com), section 二 -- exact attention over the kept blocks
+// only; section 六 -- the heads of a GQA group share the group's block set,
+// so one K/V block tile serves every (row, head) of the group that kept it.
+// The dev.to MiniMax-M3 summary describes the KV tile as the outer loop with
+// each tile read once for every query that needs it; that is the organisation
+// used here for every kept block except the query's own one.
+//
+// Exactness: softmax is invariant to the shift subtracted before exp, so the
+// partial sums of different blocks can be added directly if they share one
+// shift per (row, head).  The shift is the row's exact max over its own block
+// (pass A).  It is safe (no overflow) whenever the Cauchy-Schwarz bound
+// scale*|q|*max|k| exceeds it by at most 64 (base 2); rows where the bound
+// does not prove that are flagged and get their exact max over all kept keys
+// from the fix-up pass before pass B adds anything.
+//
+// Passes (one stream, no host synchronisation):
+//   knorm      max token norm of k per (sequence, group)
+//   bucket_*   rows that kept block j (j != own) bucketed by (sequence, group,
+//              8192-row range, j); buckets become work items of <= 256 rows
+//   pass A     own block of every row (causal), query-outer: writes the
+//              partial output, sum and shift
+//   fixup      flagged (row, head) only: exact shift, rescale pass A's partials
+//   pass B     the other kept blocks, block-outer: partials reduced into the
+//              accumulator with red.global.add.v4.f32
+//   finalize   out = accumulator / sum, bf16
+//
+// Passes A and B share one kernel: per 16-row tile, 16 rows x 8 heads = 128
+// TMEM lanes; the tile's Q rows are gathered by TMA (one 8-head x 64-dim box
+// per row and half), S = Q K^T and O = P V run as tcgen05.mma kind::f16
+// (M=128, N=128, K=128; P is written to shared memory in the K-major
+// 128-byte-swizzled layout, V is read MN-major).  Roles: warp 0 TMA, warp 1
+// MMA issue, warp 2 TMEM owner, warps 4-7 softmax and epilogue.  The
+// accumulator interleaves the 8 heads of a row at 16-byte granularity so
+// that every warp-wide reduction covers whole 128-byte lines.
+#include "msa_device.cuh"
+#include "msa_internal.h"
+
+namespace msa {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kG = 8;                      // heads per group handled by this path
+constexpr int kTileRows = 128 / kG;        // query rows per 128-lane tile
+constexpr int kRange = 8192;               // query rows per bucket range
+constexpr int kItemRows = 256;             // max rows per pass-B work item
+constexpr uint32_t kTmemCols = 512;        // S[2] + O[2], 128 columns each
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kSafeLog2 = 64.f;          // max (bound - shift) accepted, base 2
+
+struct Smem {
+    uint8_t kv[2][65536];                  // K lo, K hi, V lo, V hi (16 KiB each)
+    uint8_t q[2][32768];                   // gathered Q tile, two swizzled halves
+    uint8_t p[32768];                      // P tile (bf16), two swizzled halves
+    uint64_t kv_full[2], kv_empty[2], q_full[2], q_empty[2];
+    uint64_t s_full[2], s_empty[2], o_full[2], o_empty[2];
+    uint64_t p_full, p_empty;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+
+__device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+                 "f"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool seq_ok(const PrefillArgs &P, int b, int &L, long long &off) {
+    L = P.lens[b];
+    off = P.kv_offsets[b];
+    return L >= P.Sq && L >= 1 && L <= P.max_kv_len && off >= 0 && off + L <= P.capacity;
+}
+
+// A work item: one key block j of one (sequence, group) and the rows that
+// use it.  Pass A: the rows whose own block is j (consecutive query rows).
+// Pass B: a slice of the bucket of rows that kept j as a non-own block.
+struct Item {
+    int b, g, j, n;         // n = number of rows
+    int i_lo;               // pass A: first query row
+    const int *rows;        // pass B: flattened rows (b*Sq + i)
+    long long off;
+    int L;
+    bool valid;
+};
+
+template <int MODE>
+__device__ __forceinline__ Item item_at(const PrefillArgs &P, long long it) {
+    Item x;
+    x.valid = false;
+    x.rows = nullptr;
+    x.i_lo = 0;
+    if (MODE == 0) {
+        const int nj = (P.Sq + 127) / 128 + 1;
+        x.b = static_cast<int>(it / (static_cast<long long>(P.H_kv) * nj));
+        const int rem = static_cast<int>(it % (static_cast<long long>(P.H_kv) * nj));
+        x.g = rem / nj;
+        const int jj = rem % nj;
+        if (!seq_ok(P, x.b, x.L, x.off)) { x.n = 0; return x; }
+        const long long p0 = static_cast<long long>(x.L) - P.Sq;   // position of row 0
+        x.j = static_cast<int>(p0 / 128) + jj;
+        const long long plo = max(p0, static_cast<long long>(x.j) * 128);
+        const long long phi = min(static_cast<long long>(x.L), static_cast<long long>(x.j) * 128 + 128);
+        x.n = phi > plo ? static_cast<int>(phi - plo) : 0;
+        x.i_lo = static_cast<int>(plo - p0);
+        x.valid = x.n > 0;
+    } else {
+        const long long bucket = P.item_bucket[it];
+        const int chunk = static_cast<int>(it - P.item_off[bucket]);
+        const int cnt = P.bucket_cnt[bucket];
+        x.j = static_cast<int>(bucket % P.nb_max);
+        long long t = bucket / P.nb_max;
+        t /= P.n_ranges;
+        x.g = static_cast<int>(t % P.H_kv);
+        x.b = static_cast<int>(t / P.H_kv);
+        x.n = min(kItemRows, cnt - chunk * kItemRows);
+        x.rows = P.bucket_rows + P.bucket_off[bucket] + static_cast<long long>(chunk) * kItemRows;
+        x.valid = x.n > 0 && seq_ok(P, x.b, x.L, x.off);
+    }
+    return x;
+}
+
+template <int MODE>
+__device__ __forceinline__ long long n_items(const PrefillArgs &P) {
+    if (MODE == 0) return static_cast<long long>(P.B) * P.H_kv * ((P.Sq + 127) / 128 + 1);
+    return *P.item_total;
+}
+
+// Flattened row (b*Sq + i) of row r of tile t of the item.
+__device__ __forceinline__ long long tile_row(const PrefillArgs &P, const Item &x, int r) {
+    return x.rows ? static_cast<long long>(x.rows[r])
+                  : static_cast<long long>(x.b) * P.Sq + x.i_lo + r;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_prefill_kernel(const __grid_constant__ CUtensorMap tmQ,
+                        const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const PrefillArgs P) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem &S = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                        ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long total = n_items<MODE>(P);
+
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&S.kv_full[i], 1);
+            mbar_init(&S.kv_empty[i], 1);
+            mbar_init(&S.q_full[i], 1);
+            // Pass A reads each Q tile once more (its norms) after the MMA: the
+            // four softmax warps release it; in pass B the MMA commit does.
+            mbar_init(&S.q_empty[i], MODE == 0 ? 4 : 1);
+            mbar_init(&S.s_full[i], 1);
+            mbar_init(&S.s_empty[i], 4);
+            mbar_init(&S.o_full[i], 1);
+            mbar_init(&S.o_empty[i], 4);
+        }
+        mbar_init(&S.p_full, 4);
+        mbar_init(&S.p_empty, 1);
+        S.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 2) {
+        tmem_alloc(&S.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+    volatile int *abort_flag = &S.abort_flag;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (whole warp:
+        // lane 0 owns the barriers, lane r gathers tile row r)
+        if (lane == 0) {
+            prefetch_tensormap(&tmQ);
+            prefetch_tensormap(&tmK);
+            prefetch_tensormap(&tmV);
+        }
+        int ki = 0, qt = 0;
+        bool ok = true;
+        for (long long it = blockIdx.x; it < total && ok; it += gridDim.x) {
+            const Item x = item_at<MODE>(P, it);
+            if (!x.valid) continue;
+            const int kvs = ki & 1;
+            if (lane == 0) {
+                if (ki >= 2 &&
+                    (*abort_flag || !mbar_wait(&S.kv_empty[kvs], ((ki >> 1) - 1) & 1, P.status))) {
+                    ok = false;
+                } else {
+                    const int tok = static_cast<int>(x.off + static_cast<long long>(x.j) * 128);
+                    mbar_arrive_expect_tx(&S.kv_full[kvs], 65536);
+                    tma_load_3d(S.kv[kvs], &tmK, 0, x.g, tok, &S.kv_full[kvs]);
+                    tma_load_3d(S.kv[kvs] + 16384, &tmK, 64, x.g, tok, &S.kv_full[kvs]);
+                    tma_load_3d(S.kv[kvs] + 32768, &tmV, 0, x.g, tok, &S.kv_full[kvs]);
+                    tma_load_3d(S.kv[kvs] + 49152, &tmV, 64, x.g, tok, &S.kv_full[kvs]);
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            ++ki;
+            for (int t0 = 0; t0 < x.n; t0 += kTileRows, ++qt) {
+                const int qs = qt & 1;
+                const int nr = min(kTileRows, x.n - t0);
+                // Row index of this lane's gather, loaded before the wait.
+                const int row = lane < nr ? static_cast<int>(tile_row(P, x, t0 + lane)) : 0;
+                if (lane == 0) {
+                    if (qt >= 2 &&
+                        (*abort_flag || !mbar_wait(&S.q_empty[qs], ((qt >> 1) - 1) & 1, P.status)))
+                        ok = false;
+                    else
+                        mbar_arrive_expect_tx(&S.q_full[qs], nr * 2 * 1024);
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                if (lane < nr) {
+                    tma_load_3d(S.q[qs] + lane * 1024, &tmQ, 0, x.g * kG, row, &S.q_full[qs]);
+                    tma_load_3d(S.q[qs] + 16384 + lane * 1024, &tmQ, 64, x.g * kG, row, &S.q_full[qs]);
+                }
+            }
+        }
+        if (!ok && lane == 0) *abort_flag = 1;
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------ MMA issuer
+        const uint32_t idesc_qk = umma_idesc_bf16(128, 128);
+        const uint32_t idesc_pv = umma_idesc_bf16(128, 128) | (1u << 16);   // B (V) MN-major
+        int ki = 0, qt = 0;
+        int pv_pending = -1, pv_kvs = 0, pv_last = 0;   // tile waiting for its PV
+        bool ok = true;
+        auto issue_pv = [&](int t, int kvs, int last_of_item) -> bool {
+            const int os = t & 1;
+            if (*abort_flag || !mbar_wait(&S.p_full, t & 1, P.status)) return false;
+            if (t >= 2 && (*abort_flag || !mbar_wait(&S.o_empty[os], ((t >> 1) - 1) & 1, P.status)))
+                return false;
+            tc_fence_after();
+            const uint32_t pa = smem_u32(S.p);
+            const uint32_t va = smem_u32(S.kv[kvs] + 32768);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint64_t ad = umma_desc(pa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                const uint64_t bd = umma_desc(va + kk * 2048, 16384, 1024);
+                umma_bf16_ss(tmem + 256 + os * 128, ad, bd, idesc_pv, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&S.o_full[os]);
+            umma_commit(&S.p_empty);
+            if (last_of_item) umma_commit(&S.kv_empty[kvs]);
+            return true;
+        };
+        for (long long it = blockIdx.x; it < total && ok; it += gridDim.x) {
+            const Item x = item_at<MODE>(P, it);
+            if (!x.valid) continue;
+            const int kvs = ki & 1;
+            if (*abort_flag || !mbar_wait(&S.kv_full[kvs], (ki >> 1) & 1, P.status)) { ok = false; break; }
+            ++ki;
+            const uint32_t ka = smem_u32(S.kv[kvs]);
+            for (int t0 = 0; t0 < x.n; t0 += kTileRows, ++qt) {
+                const int qs = qt & 1, ss = qt & 1;
+                if (*abort_flag || !mbar_wait(&S.q_full[qs], (qt >> 1) & 1, P.status)) { ok = false; break; }
+                if (qt >= 2 && (*abort_flag || !mbar_wait(&S.s_empty[ss], ((qt >> 1) - 1) & 1, P.status))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t qa = smem_u32(S.q[qs]);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t ad = umma_desc(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = umma_desc(ka + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                    umma_bf16_ss(tmem + ss * 128, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&S.s_full[ss]);
+                if (MODE == 1) umma_commit(&S.q_empty[qs]);
+                // PV of the previous tile runs behind this tile's QK.
+                if (pv_pending >= 0 && !issue_pv(pv_pending, pv_kvs, pv_last)) { ok = false; break; }
+                pv_pending = qt;
+                pv_kvs = kvs;
+                pv_last = t0 + kTileRows >= x.n;
+            }
+        }
+        if (ok && pv_pending >= 0 && !issue_pv(pv_pending, pv_kvs, pv_last)) ok = false;
+        if (!ok) *abort_flag = 1;
+        // Every MMA issued must finish before TMEM is released.
+        if (qt > 0) mbar_wait(&S.s_full[(qt - 1) & 1], ((qt - 1) >> 1) & 1, nullptr);
+        if (pv_pending >= 0) mbar_wait(&S.o_full[pv_pending & 1], (pv_pending >> 1) & 1, nullptr);
+    } else if (warp >= 4) {
+        // ------------------------------------------------ softmax + epilogue
+        const int m = tid - 128;                       // TMEM lane
+        const int ri = m / kG, h = m % kG;             // tile row, head in group
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        const float sl2 = P.softmax_scale * kLog2e;
+        int qt = 0;
+        bool ok = true;
+        // state of the tile whose output is still in TMEM
+        int prev = -1;
+        long long prev_row = 0;
+        int prev_g = 0;
+        bool prev_valid = false;
+        float prev_l = 0.f;
+
+        auto epilogue = [&](int t, long long row, int g, bool valid, float l) -> bool {
+            const int os = t & 1;
+            bool have = !*abort_flag && mbar_wait(&S.o_full[os], (t >> 1) & 1, P.status);
+            have = __all_sync(0xffffffffu, have);
+            if (!have) return false;
+            tc_fence_after();
+            float *acc = P.o_acc + (row * P.H_kv + g) * (kDim * kG) + h * 4;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float v[32];
+                tmem_ld32(lane_addr + 256 + os * 128 + c * 32, v);
+                tmem_ld_wait();
+                if (valid) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 8; ++q4) {
+                        float *dst = acc + (c * 8 + q4) * (4 * kG);
+                        if (MODE == 0)
+                            *reinterpret_cast<float4 *>(dst) =
+                                make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+                        else
+                            red_add_v4(dst, v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+                    }
+                }
+            }
+            if (valid) {
+                float *lp = P.l_acc + row * P.H_q + g * kG + h;
+                if (MODE == 0) *lp = l;
+                else atomicAdd(lp, l);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.o_empty[os]);
+            return true;
+        };
+
+        for (long long it = blockIdx.x; it < total && ok; it += gridDim.x) {
+            const Item x = item_at<MODE>(P, it);
+            if (!x.valid) continue;
+            for (int t0 = 0; t0 < x.n; t0 += kTileRows, ++qt) {
+                const int ss = qt & 1;
+                const bool valid = t0 + ri < x.n;
+                const long long row = valid ? tile_row(P, x, t0 + ri) : 0;
+                // Pass B's shift is known before S: fetch it while the MMA runs.
+                float shift_b = 0.f;
+                if (MODE == 1 && valid) shift_b = P.m_arr[row * P.H_q + x.g * kG + h];
+                bool have = !*abort_flag && mbar_wait(&S.s_full[ss], (qt >> 1) & 1, P.status);
+                have = __all_sync(0xffffffffu, have);
+                if (!have) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t sa = lane_addr + ss * 128;
+                float shift, l = 0.f;
+                long long p = 0;
+                if (MODE == 0) {
+                    // own block: causal mask t <= p, exact max of the visible logits
+                    p = static_cast<long long>(x.L) - P.Sq + (row - static_cast<long long>(x.b) * P.Sq);
+                    const long long lim = p - static_cast<long long>(x.j) * 128;   // last visible column
+                    float mx = -INFINITY;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        float v[32];
+                        tmem_ld32(sa + c * 32, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (c * 32 + e <= lim) mx = fmaxf(mx, v[e] * sl2);
+                    }
+                    shift = valid ? mx : 0.f;
+                } else {
+                    shift = shift_b;
+                }
+                // P buffer is free once the previous tile's PV has read it.
+                bool pfree = !*abort_flag && (qt == 0 || mbar_wait(&S.p_empty, (qt - 1) & 1, P.status));
+                pfree = __all_sync(0xffffffffu, pfree);
+                if (!pfree) { ok = false; break; }
+                const long long lim = MODE == 0 ? p - static_cast<long long>(x.j) * 128 : 127;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float v[32];
+                    tmem_ld32(sa + c * 32, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float z = v[e] * sl2 - shift;
+                        v[e] = (c * 32 + e <= lim && valid) ? exp2f(z) : 0.f;
+                        l += v[e];
+                    }
+                    // 32 tokens = 4 chunks of 8 in half c / 2
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8) {
+                        const int chunk = (c & 1) * 4 + q8;
+                        uint4 w;
+                        w.x = pack_bf16x2(v[8 * q8 + 0], v[8 * q8 + 1]);
+                        w.y = pack_bf16x2(v[8 * q8 + 2], v[8 * q8 + 3]);
+                        w.z = pack_bf16x2(v[8 * q8 + 4], v[8 * q8 + 5]);
+                        w.w = pack_bf16x2(v[8 * q8 + 6], v[8 * q8 + 7]);
+                        *reinterpret_cast<uint4 *>(S.p + (c >> 1) * 16384 + swz128(m, chunk)) = w;
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&S.s_empty[ss]);
+                    mbar_arrive(&S.p_full);
+                }
+                if (MODE == 0) {
+                    bool qok = !*abort_flag && mbar_wait(&S.q_full[qt & 1], (qt >> 1) & 1, P.status);
+                    qok = __all_sync(0xffffffffu, qok);
+                    if (!qok) { ok = false; break; }
+                }
+                if (MODE == 0 && valid) {
+                    // Shift of this (row, head) and the safety test of the bound.
+                    const uint8_t *qs = S.q[qt & 1];
+                    float nq = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const uint4 w = *reinterpret_cast<const uint4 *>(
+                            qs + (c >> 3) * 16384 + swz128(m, c & 7));
+                        const uint32_t a4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            nq = fmaf(bf16lo(a4[e]), bf16lo(a4[e]), nq);
+                            nq = fmaf(bf16hi(a4[e]), bf16hi(a4[e]), nq);
+                        }
+                    }
+                    const float bound = fabsf(sl2) * sqrtf(nq) * P.knorm[x.b * P.H_kv + x.g];
+                    const long long idx = row * P.H_q + x.g * kG + h;
+                    P.m_arr[idx] = shift;
+                    const uint8_t fl = !(bound - shift <= kSafeLog2);   // NaN-safe
+                    P.flags[idx] = fl;
+                    if (fl) atomicAdd(P.flag_count, 1);
+                }
+                if (MODE == 0) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.q_empty[qt & 1]);
+                }
+                // Output of the previous tile (its PV ran while this tile's QK did).
+                if (prev >= 0 && !epilogue(prev, prev_row, prev_g, prev_valid, prev_l)) { ok = false; break; }
+                prev = qt;
+                prev_row = row;
+                prev_g = x.g;
+                prev_valid = valid;
+                prev_l = l;
+            }
+        }
+        if (ok && prev >= 0 && !epilogue(prev, prev_row, prev_g, prev_valid, prev_l)) ok = false;
+        if (!ok) *abort_flag = 1;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- helpers
+// Max token norm of k per (sequence, group); one warp per (sequence, group,
+// 128-token block).
+__global__ void knorm_kernel(const PrefillArgs P) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    const int nb = P.nb_max;
+    const long long total = static_cast<long long>(P.B) * P.H_kv * nb;
+    for (long long w = warp; w < total; w += (static_cast<long long>(gridDim.x) * blockDim.x) >> 5) {
+        const int j = static_cast<int>(w % nb);
+        const int g = static_cast<int>((w / nb) % P.H_kv);
+        const int b = static_cast<int>(w / (static_cast<long long>(nb) * P.H_kv));
+        int L;
+        long long off;
+        if (!seq_ok(P, b, L, off) || j * 128 >= L) continue;
+        const __nv_bfloat16 *k = static_cast<const __nv_bfloat16 *>(P.k_cache);
+        float best = 0.f;
+        for (int t = j * 128 + lane; t < min(L, j * 128 + 128); t += 32) {
+            const uint4 *row = reinterpret_cast<const uint4 *>(k + ((off + t) * P.H_kv + g) * kDim);
+            float s = 0.f;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const uint4 v = row[c];
+                const uint32_t a4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    s = fmaf(bf16lo(a4[e]), bf16lo(a4[e]), s);
+                    s = fmaf(bf16hi(a4[e]), bf16hi(a4[e]), s);
+                }
+            }
+            best = fmaxf(best, sqrtf(s));
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
+        // Norms are >= 0, so their float bits order like ints (NaN -> flagged later).
+        if (lane == 0) atomicMax(reinterpret_cast<int *>(P.knorm) + b * P.H_kv + g, __float_as_int(best));
+    }
+}
+
+// Visits every (row, group, slot) whose block is kept and is not the row's own.
+template <int PHASE>
+__global__ void bucket_kernel(const PrefillArgs P) {
+    const long long total = static_cast<long long>(P.B) * P.Sq * P.H_kv * P.K;
+    for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+         e += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long pair = e / P.K;
+        const long long row = pair / P.H_kv;
+        const int g = static_cast<int>(pair % P.H_kv);
+        const int b = static_cast<int>(row / P.Sq), i = static_cast<int>(row % P.Sq);
+        int L;
+        long long off;
+        if (!seq_ok(P, b, L, off)) continue;
+        const int j = P.ids[e];
+        const long long p = static_cast<long long>(L) - P.Sq + i;
+        if (j < 0 || j >= p / 128) continue;            // padding, own block, or out of range
+        const long long bucket =
+            ((static_cast<long long>(b) * P.H_kv + g) * P.n_ranges + i / kRange) * P.nb_max + j;
+        if (PHASE == 0) {
+            atomicAdd(P.bucket_cnt + bucket, 1);
+        } else {
+            const int pos = atomicAdd(P.bucket_cur + bucket, 1);
+            P.bucket_rows[P.bucket_off[bucket] + pos] = static_cast<int>(row);
+        }
+    }
+}
+
+// Exclusive scans of the bucket counts (row offsets) and of their item counts.
+__global__ void __launch_bounds__(1024) bucket_scan_kernel(const PrefillArgs P) {
+    __shared__ long long part_rows[1024], part_items[1024];
+    const long long n = P.n_buckets;
+    const int tid = threadIdx.x;
+    const long long per = (n + 1023) / 1024;
+    const long long lo = min(n, tid * per), hi = min(n, lo + per);
+    long long sr = 0, si = 0;
+    for (long long k = lo; k < hi; ++k) {
+        const int c = P.bucket_cnt[k];
+        sr += c;
+        si += (c + kItemRows - 1) / kItemRows;
+    }
+    part_rows[tid] = sr;
+    part_items[tid] = si;
+    __syncthreads();
+    if (tid == 0) {
+        long long ar = 0, ai = 0;
+        for (int t = 0; t < 1024; ++t) {
+            const long long r = part_rows[t], q = part_items[t];
+            part_rows[t] = ar;
+            part_items[t] = ai;
+            ar += r;
+            ai += q;
+        }
+        P.bucket_off[n] = static_cast<int>(ar);
+        P.item_off[n] = ai;
+        *P.item_total = ai;
+    }
+    __syncthreads();
+    long long ar = part_rows[tid], ai = part_items[tid];
+    for (long long k = lo; k < hi; ++k) {
+        const int c = P.bucket_cnt[k];
+        const int ni = (c + kItemRows - 1) / kItemRows;
+        P.bucket_off[k] = static_cast<int>(ar);
+        P.item_off[k] = ai;
+        for (int q = 0; q < ni; ++q) P.item_bucket[ai + q] = static_cast<int>(k);
+        ar += c;
+        ai += ni;
+    }
+}
+
+// Flagged (row, head): exact max logit over the row's other kept keys, then
+// the own-block partials are rescaled to the new shift.  Exits at once when
+// no row was flagged.  One warp per (row, group).
+__global__ void fixup_kernel(const PrefillArgs P) {
+    if (*P.flag_count == 0) return;
+    const int lane = threadIdx.x & 31;
+    const long long total = static_cast<long long>(P.B) * P.Sq * P.H_kv;
+    const float sl2 = P.softmax_scale * kLog2e;
+    const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(P.q);
+    const __nv_bfloat16 *kb = static_cast<const __nv_bfloat16 *>(P.k_cache);
+    for (long long pair = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+         pair < total; pair += (static_cast<long long>(gridDim.x) * blockDim.x) >> 5) {
+        const long long row = pair / P.H_kv;
+        const int g = static_cast<int>(pair % P.H_kv);
+        const int b = static_cast<int>(row / P.Sq), i = static_cast<int>(row % P.Sq);
+        int L;
+        long long off;
+        if (!seq_ok(P, b, L, off)) continue;
+        const long long p = static_cast<long long>(L) - P.Sq + i;
+        for (int h = 0; h < kG; ++h) {
+            const long long idx = row * P.H_q + g * kG + h;
+            if (!P.flags[idx]) continue;
+            const __nv_bfloat16 *qh = qb + idx * kDim;
+            float mx = -INFINITY;
+            for (int s = 0; s < P.K; ++s) {
+                const int j = P.ids[pair * P.K + s];
+                if (j < 0 || j >= p / 128) continue;
+                for (int t = j * 128 + lane; t < j * 128 + 128; t += 32) {
+                    const __nv_bfloat16 *kt = kb + ((off + t) * P.H_kv + g) * kDim;
+                    float d = 0.f;
+                    for (int c = 0; c < kDim; ++c) d = fmaf(__bfloat162float(qh[c]), __bfloat162float(kt[c]), d);
+                    mx = fmaxf(mx, d * sl2);
+                }
+            }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            const float m_own = P.m_arr[idx];
+            const float m_new = fmaxf(m_own, mx);
+            const float sc = exp2f(m_own - m_new);
+            float *acc = P.o_acc + (row * P.H_kv + g) * (kDim * kG) + h * 4;
+            for (int c = lane; c < kDim / 4; c += 32) {
+                float4 *v = reinterpret_cast<float4 *>(acc + c * 4 * kG);
+                float4 x = *v;
+                x.x *= sc; x.y *= sc; x.z *= sc; x.w *= sc;
+                *v = x;
+            }
+            __syncwarp();
+            if (lane == 0) {
+                P.l_acc[idx] *= sc;
+                P.m_arr[idx] = m_new;
+            }
+        }
+    }
+}
+
+// out = accumulator / sum, bf16.  One warp per (row, group): lane = (head, 32 dims).
+__global__ void finalize_kernel(const PrefillArgs P) {
+    const int lane = threadIdx.x & 31;
+    const int h = lane >> 2, qd = lane & 3;
+    const long long total = static_cast<long long>(P.B) * P.Sq * P.H_kv;
+    for (long long pair = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+         pair < total; pair += (static_cast<long long>(gridDim.x) * blockDim.x) >> 5) {
+        const long long row = pair / P.H_kv;
+        const int g = static_cast<int>(pair % P.H_kv);
+        const int b = static_cast<int>(row / P.Sq);
+        int L;
+        long long off;
+        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(P.out) + (row * P.H_q + g * kG + h) * kDim + qd * 32;
+        if (!seq_ok(P, b, L, off)) {
+            for (int d = 0; d < 32; ++d) out[d] = __float2bfloat16(NAN);
+            continue;
+        }
+        const float inv = 1.f / P.l_acc[row * P.H_q + g * kG + h];
+        const float *acc = P.o_acc + pair * (kDim * kG) + h * 4;
+#pragma unroll
+        for (int c = 0; c < 8; c += 2) {
+            const float4 a = *reinterpret_cast<const float4 *>(acc + (qd * 8 + c) * 4 * kG);
+            const float4 bq = *reinterpret_cast<const float4 *>(acc + (qd * 8 + c + 1) * 4 * kG);
+            uint4 w;
+            w.x = pack_bf16x2(a.x * inv, a.y * inv);
+            w.y = pack_bf16x2(a.z * inv, a.w * inv);
+            w.z = pack_bf16x2(bq.x * inv, bq.y * inv);
+            w.w = pack_bf16x2(bq.z * inv, bq.w * inv);
+            *reinterpret_cast<uint4 *>(out + c * 4) = w;
+        }
+    }
+}
+
+template <int MODE>
+cudaError_t launch_pass(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                        const PrefillArgs &a, cudaStream_t s, const char *name) {
+    const size_t smem = sizeof(Smem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    TraceScope trace(s, name);
+    attn_prefill_kernel<MODE><<<device_sm_count(), kThreads, smem, s>>>(tq, tk, tv, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool prefill_attention_supported(int H_q, int H_kv) { return H_q / H_kv == kG; }
+
+size_t prefill_workspace_layout(int B, int Sq, int H_q, int H_kv, int K, int max_kv_len,
+                                PrefillLayout *L) {
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    const long long rows = static_cast<long long>(B) * Sq;
+    L->nb_max = (max_kv_len + 127) / 128;
+    L->n_ranges = (Sq + kRange - 1) / kRange;
+    L->n_buckets = static_cast<long long>(B) * H_kv * L->n_ranges * L->nb_max;
+    size_t o = kWsHeaderBytes;
+    L->knorm = o;        o += up(static_cast<size_t>(B) * H_kv * 4);
+    L->cnt = o;          o += up(static_cast<size_t>(L->n_buckets) * 4);
+    L->cur = o;          o += up(static_cast<size_t>(L->n_buckets) * 4);
+    L->zero_end = o;                                  // [knorm, zero_end) is cleared per call
+    L->off = o;          o += up(static_cast<size_t>(L->n_buckets + 1) * 4);
+    L->item_off = o;     o += up(static_cast<size_t>(L->n_buckets + 1) * 8);
+    L->item_bucket = o;
+    o += up((static_cast<size_t>(L->n_buckets) + static_cast<size_t>(rows) * H_kv * K / kItemRows + 1) * 4);
+    L->rows = o;         o += up(static_cast<size_t>(rows) * H_kv * (K > 1 ? K - 1 : 1) * 4);
+    L->o_acc = o;        o += up(static_cast<size_t>(rows) * H_q * kDim * 4);
+    L->l_acc = o;        o += up(static_cast<size_t>(rows) * H_q * 4);
+    L->m_arr = o;        o += up(static_cast<size_t>(rows) * H_q * 4);
+    L->flags = o;        o += up(static_cast<size_t>(rows) * H_q);
+    L->total = o;
+    return o;
+}
+
+cudaError_t launch_prefill_attention(const PrefillArgs &a0, uint8_t *ws, const PrefillLayout &L,
+                                     cudaStream_t s) {
+    PrefillArgs a = a0;
+    a.knorm = reinterpret_cast<float *>(ws + L.knorm);
+    a.bucket_cnt = reinterpret_cast<int *>(ws + L.cnt);
+    a.bucket_cur = reinterpret_cast<int *>(ws + L.cur);
+    a.bucket_off = reinterpret_cast<int *>(ws + L.off);
+    a.item_off = reinterpret_cast<long long *>(ws + L.item_off);
+    a.item_bucket = reinterpret_cast<int *>(ws + L.item_bucket);
+    a.bucket_rows = reinterpret_cast<int *>(ws + L.rows);
+    a.o_acc = reinterpret_cast<float *>(ws + L.o_acc);
+    a.l_acc = reinterpret_cast<float *>(ws + L.l_acc);
+    a.m_arr = reinterpret_cast<float *>(ws + L.m_arr);
+    a.flags = reinterpret_cast<uint8_t *>(ws + L.flags);
+    a.flag_count = reinterpret_cast<int *>(ws + 4);
+    a.item_total = reinterpret_cast<long long *>(ws + 8);
+    a.nb_max = L.nb_max;
+    a.n_ranges = L.n_ranges;
+    a.n_buckets = L.n_buckets;
+
+    CUtensorMap tq, tk, tv;
+    if (!encode_q_gather_map(&tq, a.q, a.H_q, static_cast<long long>(a.B) * a.Sq) ||
+        !encode_kv_tensor_map(&tk, a.k_cache, a.H_kv, a.capacity) ||
+        !encode_kv_tensor_map(&tv, a.v_cache, a.H_kv, a.capacity))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaMemsetAsync(ws + L.knorm, 0, L.zero_end - L.knorm, s);
+    if (e != cudaSuccess) return e;
+    const int sms = device_sm_count();
+    {
+        TraceScope t(s, "prefill_knorm");
+        knorm_kernel<<<sms * 4, 256, 0, s>>>(a);
+    }
+    {
+        TraceScope t(s, "prefill_bucket");
+        bucket_kernel<0><<<sms * 8, 256, 0, s>>>(a);
+        bucket_scan_kernel<<<1, 1024, 0, s>>>(a);
+        bucket_kernel<1><<<sms * 8, 256, 0, s>>>(a);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pass<0>(tq, tk, tv, a, s, "prefill_attn_own_block")) != cudaSuccess) return e;
+    {
+        TraceScope t(s, "prefill_fixup");
+        fixup_kernel<<<sms * 4, 256, 0, s>>>(a);
+    }
+    if ((e = launch_pass<1>(tq, tk, tv, a, s, "prefill_attn_kv_outer")) != cudaSuccess) return e;
+    {
+        TraceScope t(s, "prefill_finalize");
+        finalize_kernel<<<sms * 8, 256, 0, s>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace msa

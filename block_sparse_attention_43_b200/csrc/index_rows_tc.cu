@@ -16,8 +16,11 @@
 // commits to mbarriers.  Four epilogue warps (one TMEM lane = one query row
 // per thread) read the accumulator with tcgen05.ld, apply the causal mask
 // where the block reaches past the row's position and write one block score
-// per (row, block).  Units are dealt to a persistent grid in snake order of
-// decreasing length.
+// per (row, block) into a running top-k list the thread keeps in registers
+// (candidate blocks arrive in increasing order, so the list needs no
+// scores buffer and no second pass).  At the end of the unit each thread
+// writes its row's kept ids ascending, the own block last.  Units are dealt
+// to a persistent grid in snake order of decreasing length.
 //
 // Roles: warp 0 = TMA producer, warp 1 = MMA issuer, warp 2 = TMEM owner,
 // warps 4-7 = epilogue (warp % 4 selects its 32 TMEM lanes).
@@ -76,6 +79,34 @@ __device__ __forceinline__ long long unit_index(int r) {
     return static_cast<long long>(r) * G + c;
 }
 
+// Running top-(k-1) list of one query row: LIST keys sorted descending.
+// The first LIST-(k-1) slots hold a sentinel larger than any key, so the
+// smallest kept key is always L[LIST-1] and every index is static.
+template <int LIST>
+struct TopList {
+    unsigned long long L[LIST];
+    __device__ __forceinline__ void reset(int keep) {
+#pragma unroll
+        for (int i = 0; i < LIST; ++i) L[i] = (i < LIST - keep) ? ~0ull : 0ull;
+    }
+    __device__ __forceinline__ void offer(unsigned long long key) {
+        if (key <= L[LIST - 1]) return;
+        unsigned long long x = key;
+#pragma unroll
+        for (int i = 0; i < LIST; ++i) {
+            const unsigned long long hi = L[i] > x ? L[i] : x;
+            x = L[i] > x ? x : L[i];
+            L[i] = hi;
+        }
+    }
+};
+
+__device__ __forceinline__ float key_score(unsigned long long key) {
+    const uint32_t u = static_cast<uint32_t>(key >> 32);
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
+template <int LIST>
 __global__ void __launch_bounds__(kThreads, 1)
     index_rows_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK, const IndexRowsArgs P) {
@@ -198,18 +229,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------ epilogue
         const int r = tid - 128;                     // TMEM lane = tile row
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        const int keep = P.K - 1;                    // non-own blocks kept per row
+        TopList<LIST> top;
         int ita = 0;
         bool ok = true;
         for (int rr = 0; ok; ++rr) {
             const long long u = unit_index(rr);
             if (u >= nunits) break;
             const Unit x = unit_at(P, u, ntiles);
-            if (!x.valid) continue;
+            const bool row_ok = r < x.nrows;
+            const long long out_off =
+                ((static_cast<long long>(x.b) * P.Sq + x.i0 + r) * P.H_kv + x.g) * P.K;
+            if (!x.valid) {
+                if (row_ok)
+                    for (int q = 0; q < P.K; ++q) {
+                        P.ids[out_off + q] = -1;
+                        P.out_scores[out_off + q] = -INFINITY;
+                    }
+                continue;
+            }
             const long long p = x.p_first + r;        // this row's query position
             const int own = static_cast<int>(p / kBlock);
-            const bool row_ok = r < x.nrows;
-            float *dst = P.scores + ((static_cast<long long>(x.b) * P.Sq + x.i0 + r) * P.H_kv + x.g) *
-                                        static_cast<long long>(P.nb_max);
+            float s_own = -INFINITY;
+            top.reset(keep);
             for (int j = 0; j <= x.jmax; j += 2, ++ita) {
                 const int a = ita & 1;
                 bool have = !*abort_flag && mbar_wait(&S.acc_full[a], (ita >> 1) & 1, P.status);
@@ -236,11 +278,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 if (t0 + c * 32 + e <= p) m = fmaxf(m, v[e]);
                         }
                     }
-                    if (row_ok && J <= own) dst[J] = m;
+                    if (J < own) top.offer(topk_key(m, J));
+                    else if (J == own) s_own = m;
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.acc_empty[a]);
+            }
+            if (!ok || !row_ok) continue;
+            // Kept non-own blocks (all ids < own) ascending, then the own block.
+            // They sit in slots [LIST - keep, LIST - keep + n_other), best first.
+            const int n_other = min(own, keep);
+            const int lo = LIST - keep, hi = LIST - keep + n_other;
+            int32_t *ids_out = P.ids + out_off;
+            float *sc_out = P.out_scores + out_off;
+#pragma unroll
+            for (int i = 0; i < LIST; ++i) {
+                if (i < lo || i >= hi) continue;
+                const int id = topk_key_id(top.L[i]);
+                int rank = 0;
+#pragma unroll
+                for (int k2 = 0; k2 < LIST; ++k2)
+                    if (k2 >= lo && k2 < hi && topk_key_id(top.L[k2]) < id) ++rank;
+                ids_out[rank] = id;
+                sc_out[rank] = key_score(top.L[i]);
+            }
+            ids_out[n_other] = own;
+            sc_out[n_other] = s_own;
+            for (int q = n_other + 1; q < P.K; ++q) {
+                ids_out[q] = -1;
+                sc_out[q] = -INFINITY;
             }
         }
         if (!ok) *abort_flag = 1;
@@ -263,15 +330,21 @@ cudaError_t launch_index_rows_tc(const IndexRowsArgs &a, cudaStream_t s) {
         !encode_kv_tensor_map(&tk, a.k_idx, a.H_kv, a.capacity))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(Smem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(index_rows_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
     const long long ntiles = (a.Sq + 127) / 128;
     const long long units = ntiles * a.B * a.H_kv;
     const long long grid = units < device_sm_count() ? units : device_sm_count();
-    TraceScope trace(s, "index_score_maxpool_rows_tc");
-    index_rows_tc_kernel<<<static_cast<unsigned>(grid), kThreads, smem, s>>>(tq, tk, a);
-    return cudaGetLastError();
+    auto go = [&](auto kern) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        TraceScope trace(s, "index_score_maxpool_topk_rows_tc");
+        kern<<<static_cast<unsigned>(grid), kThreads, smem, s>>>(tq, tk, a);
+        return cudaGetLastError();
+    };
+    if (a.K <= 16) return go(index_rows_tc_kernel<16>);
+    if (a.K <= 32) return go(index_rows_tc_kernel<32>);
+    if (a.K <= 64) return go(index_rows_tc_kernel<64>);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace msa

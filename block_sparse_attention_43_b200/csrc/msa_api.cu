@@ -56,6 +56,20 @@ bool encode_kv_tensor_map(CUtensorMap *map, const void *base, int H_kv, long lon
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool encode_q_gather_map(CUtensorMap *map, const void *q, int H_q, long long rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDim), static_cast<cuuint64_t>(H_q),
+                                static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDim) * 2,
+                                   static_cast<cuuint64_t>(kDim) * 2 * H_q};
+    const cuuint32_t box[3] = {64, 8, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace msa
 
 using namespace msa;
@@ -93,18 +107,36 @@ long long rows_of(const msa_shape_t *s) { return static_cast<long long>(s->batch
 
 int nb_max_of(const msa_shape_t *s) { return (s->max_kv_len + kBlock - 1) / kBlock; }
 
+// Decode keeps one fp32 score per (sequence, group, block) for the top-k
+// pass; prefill selects inside the tensor-core kernel and needs only the header.
 size_t index_ws_bytes(const msa_shape_t *s) {
+    if (s->q_len > 1) return kWsHeaderBytes;
     return kWsHeaderBytes +
            round_up(static_cast<size_t>(rows_of(s)) * s->num_kv_heads * nb_max_of(s) * sizeof(float));
+}
+
+// Prefill rows with groups of 8 heads run the block-outer tensor-core path;
+// decode rows (and other group sizes) run one CTA per (row, group, split).
+bool use_prefill_path(const msa_shape_t *s) {
+    return s->q_len > 1 && prefill_attention_supported(s->num_q_heads, s->num_kv_heads);
 }
 
 struct AttnLayout {
     int nsplit;
     size_t tickets_off, tickets_bytes, partials_off, total;
+    PrefillLayout pre;
 };
 
 AttnLayout attn_layout(const msa_shape_t *s) {
     AttnLayout L;
+    if (use_prefill_path(s)) {
+        L.nsplit = 1;
+        L.tickets_off = L.partials_off = kWsHeaderBytes;
+        L.tickets_bytes = 0;
+        L.total = prefill_workspace_layout(s->batch, s->q_len, s->num_q_heads, s->num_kv_heads,
+                                           s->top_k, s->max_kv_len, &L.pre);
+        return L;
+    }
     const long long pairs = rows_of(s) * s->num_kv_heads;
     L.nsplit = attn_rows_nsplit(pairs, s->top_k);
     const int G = s->num_q_heads / s->num_kv_heads;
@@ -165,10 +197,10 @@ msa_status_t msa_index_topk(const msa_shape_t *shape, const void *q_idx, const v
     } else {
         IndexRowsArgs a;
         a.q_idx = q_idx; a.k_idx = k_idx; a.lens = lens; a.kv_offsets = kv_offsets;
-        a.scores = scores; a.status = status;
-        a.B = shape->batch; a.Sq = shape->q_len; a.H_kv = shape->num_kv_heads; a.nb_max = nb_max;
+        a.ids = block_ids; a.out_scores = block_scores; a.status = status;
+        a.B = shape->batch; a.Sq = shape->q_len; a.H_kv = shape->num_kv_heads; a.K = shape->top_k;
         a.max_kv_len = shape->max_kv_len; a.capacity = shape->kv_capacity;
-        e = launch_index_rows_tc(a, s);
+        return launch_index_rows_tc(a, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
     }
     if (e != cudaSuccess) return MSA_ERR_CUDA;
     TopkArgs t;
@@ -200,6 +232,15 @@ msa_status_t msa_sparse_attention(const msa_shape_t *shape, const void *q, const
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     if (cudaMemsetAsync(ws, 0, kWsHeaderBytes + L.tickets_bytes, s) != cudaSuccess)
         return MSA_ERR_CUDA;
+    if (use_prefill_path(shape)) {
+        PrefillArgs p;
+        p.q = q; p.k_cache = k_cache; p.v_cache = v_cache; p.ids = block_ids; p.lens = lens;
+        p.kv_offsets = kv_offsets; p.out = out; p.status = reinterpret_cast<int *>(ws);
+        p.B = shape->batch; p.Sq = shape->q_len; p.H_q = shape->num_q_heads;
+        p.H_kv = shape->num_kv_heads; p.K = shape->top_k; p.max_kv_len = shape->max_kv_len;
+        p.capacity = shape->kv_capacity; p.softmax_scale = softmax_scale;
+        return launch_prefill_attention(p, ws, L.pre, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+    }
     AttnRowsArgs a;
     a.q = q; a.k_cache = k_cache; a.v_cache = v_cache; a.ids = block_ids; a.lens = lens;
     a.kv_offsets = kv_offsets; a.out = out;

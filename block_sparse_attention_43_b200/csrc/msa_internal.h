@@ -39,16 +39,18 @@ struct IndexDecodeArgs {
 };
 cudaError_t launch_index_decode(const IndexDecodeArgs &a, cudaStream_t s);
 
-// Block max-pooled index scores for q_len >= 1 query rows per sequence
-// (prefill), causal: scores[r][g][j] for every visible block j <= own(r).
+// Index branch for q_len >= 1 query rows per sequence (prefill), causal:
+// block max-pooled scores of every visible block and the top-k selection,
+// written straight to ids / out_scores [B*Sq][H_kv][K].
 struct IndexRowsArgs {
     const void *q_idx;      // [B][Sq][H_kv][128]
     const void *k_idx;
     const int32_t *lens;
     const int64_t *kv_offsets;
-    float *scores;          // [B*Sq][H_kv][nb_max]
+    int32_t *ids;
+    float *out_scores;
     int *status;
-    int B, Sq, H_kv, nb_max, max_kv_len;
+    int B, Sq, H_kv, K, max_kv_len;
     long long capacity;
 };
 // tcgen05 tensor-core kernel (index_rows_tc.cu).
@@ -86,6 +88,45 @@ struct AttnRowsArgs {
 cudaError_t launch_attn_rows(const AttnRowsArgs &a, cudaStream_t s);
 // Splits used by launch_attn_rows for this shape (workspace sizing too).
 int attn_rows_nsplit(long long rows_x_groups, int top_k);
+
+// Prefill sparse attention organised around the KV blocks (attn_prefill.cu).
+struct PrefillArgs {
+    const void *q;          // [B][Sq][H_q][128]
+    const void *k_cache;
+    const void *v_cache;
+    const int32_t *ids;     // [B*Sq][H_kv][K]
+    const int32_t *lens;
+    const int64_t *kv_offsets;
+    void *out;
+    int *status;
+    int B, Sq, H_q, H_kv, K, max_kv_len;
+    long long capacity;
+    float softmax_scale;
+    // workspace views (filled by launch_prefill_attention)
+    float *knorm;
+    int *bucket_cnt, *bucket_cur, *bucket_off, *bucket_rows;
+    long long *item_off;
+    int *item_bucket;       // bucket of every pass-B work item
+    long long *item_total;
+    float *o_acc, *l_acc, *m_arr;
+    uint8_t *flags;
+    int *flag_count;
+    int nb_max, n_ranges;
+    long long n_buckets;
+};
+struct PrefillLayout {
+    size_t knorm, cnt, cur, zero_end, off, item_off, item_bucket, rows, o_acc, l_acc, m_arr, flags,
+        total;
+    int nb_max, n_ranges;
+    long long n_buckets;
+};
+bool prefill_attention_supported(int H_q, int H_kv);
+size_t prefill_workspace_layout(int B, int Sq, int H_q, int H_kv, int K, int max_kv_len,
+                                PrefillLayout *L);
+cudaError_t launch_prefill_attention(const PrefillArgs &a, uint8_t *ws, const PrefillLayout &L,
+                                     cudaStream_t s);
+// 3-D map over q [rows, H_q, 128] with an 8-head x 64-dim box (one row).
+bool encode_q_gather_map(CUtensorMap *map, const void *q, int H_q, long long rows);
 
 // Encodes a [capacity, H_kv, 128] bf16 cache as a 3-D TMA tensor map whose
 // box is (64 dims, 1 group, 128 tokens) with 128-byte swizzling.

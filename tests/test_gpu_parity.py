@@ -75,6 +75,37 @@ def test_prefill_small_shapes(msa_lib, oracle_mod, B, Sq, lens, H_q, H_kv, top_k
     _run_and_compare(oracle_mod, w)
 
 
+# Groups of 8 heads take the block-outer tensor-core prefill path.
+PREFILL_G8_CASES = [
+    (1, 1000, [1000], 64, 8, 16),     # every block kept (k >= blocks), ragged last block
+    (1, 4000, [4000], 16, 2, 8),      # real selection
+    (2, 700, [3000, 700], 16, 2, 4),  # unaligned chunk after a cached prefix + a full prefill
+    (1, 20000, [20000], 8, 1, 16),    # one group, three 8192-row bucket ranges
+]
+
+
+@pytest.mark.parametrize("B,Sq,lens,H_q,H_kv,top_k", PREFILL_G8_CASES)
+def test_prefill_block_outer_path(msa_lib, oracle_mod, B, Sq, lens, H_q, H_kv, top_k):
+    from parity import sample_rows
+    from synthetic import make_inputs
+    w = make_inputs(B=B, Sq=Sq, lens=lens, H_q=H_q, H_kv=H_kv, top_k=top_k, seed=400 + Sq,
+                    device=DEV)
+    rows = None if B * Sq <= 4000 else sample_rows(B * Sq, 3000, seed=5)
+    rep = _run_and_compare(oracle_mod, w, rows=rows)
+    print("prefill g8", (B, Sq, H_q, H_kv, top_k), rep)
+
+
+def test_prefill_large_logit_block_takes_exact_shift(msa_lib, oracle_mod):
+    """A kept non-own block whose keys are 40x larger: its logits dwarf the
+    own block's, the norm bound cannot prove the own-block shift safe, and the
+    fix-up pass must supply the exact shift."""
+    from synthetic import make_inputs
+    w = make_inputs(B=1, Sq=640, lens=[640], H_q=16, H_kv=2, top_k=5, seed=33, device=DEV)
+    w.k[128:256].mul_(40.0)
+    rep = _run_and_compare(oracle_mod, w)
+    print("large logits", rep)
+
+
 @pytest.mark.parametrize("name", ["prefill_2k", "decode_32k", "decode_ragged", "decode_1m"])
 def test_named_workload_full_parity(msa_lib, oracle_mod, name):
     """The workloads at full size, every row compared."""
@@ -101,6 +132,20 @@ def test_prefill_128k_index_sampled_rows(msa_lib, oracle_mod):
     _, _, rep = compare_index(oracle_mod, w, eng.block_ids.cpu().numpy(),
                               eng.block_scores.cpu().numpy(), rows=rows, host=host)
     print("prefill_128k index", rep)
+
+
+def test_prefill_128k_full_path_sampled_rows(msa_lib, oracle_mod):
+    """128k-token prefill, both stages at full size on the GPU, in the launch
+    configuration the benchmark times; 4096 seeded rows plus block-edge rows
+    compared with the oracle (ids, scores, outputs)."""
+    from parity import compare, run_gpu, sample_rows, to_host
+    from synthetic import make_workload
+    w = make_workload("prefill_128k", DEV)
+    m, st = run_gpu(w)
+    assert st == 0, f"device status {st}"
+    rows = sample_rows(w.Sq, 4096, seed=2)
+    rep = compare(oracle_mod, w, *to_host(m), rows=rows)
+    print("prefill_128k", rep)
 
 
 def test_repeat_calls_are_bit_identical(msa_lib):
