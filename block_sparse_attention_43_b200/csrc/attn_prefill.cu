@@ -42,7 +42,8 @@
 namespace msa {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;           // 4 control warps + 8 softmax/epilogue warps
+constexpr int kSoftWarps = 8;
 constexpr int kG = 8;                      // heads per group handled by this path
 constexpr int kTileRows = 128 / kG;        // query rows per 128-lane tile
 constexpr int kRange = 8192;               // query rows per bucket range
@@ -58,9 +59,14 @@ struct Smem {
     uint64_t kv_full[2], kv_empty[2], q_full[2], q_empty[2];
     uint64_t s_full[2], s_empty[2], o_full[2], o_empty[2];
     uint64_t p_full, p_empty;
+    uint64_t item_full[4], item_empty[4];  // work-item queue: producer -> MMA + softmax
+    long long item_q[4];
     uint32_t tmem_base;
     int abort_flag;
 };
+
+constexpr int kQueue = 4;
+constexpr int kQueueReaders = 1 + kSoftWarps;   // MMA thread + one arrival per softmax warp
 
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
     uint64_t d = static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
@@ -160,15 +166,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&S.kv_empty[i], 1);
             mbar_init(&S.q_full[i], 1);
             // Pass A reads each Q tile once more (its norms) after the MMA: the
-            // four softmax warps release it; in pass B the MMA commit does.
-            mbar_init(&S.q_empty[i], MODE == 0 ? 4 : 1);
+            // softmax warps release it; in pass B the MMA commit does.
+            mbar_init(&S.q_empty[i], MODE == 0 ? kSoftWarps : 1);
             mbar_init(&S.s_full[i], 1);
-            mbar_init(&S.s_empty[i], 4);
+            mbar_init(&S.s_empty[i], kSoftWarps);
             mbar_init(&S.o_full[i], 1);
-            mbar_init(&S.o_empty[i], 4);
+            mbar_init(&S.o_empty[i], kSoftWarps);
         }
-        mbar_init(&S.p_full, 4);
+        mbar_init(&S.p_full, kSoftWarps);
         mbar_init(&S.p_empty, 1);
+        for (int i = 0; i < kQueue; ++i) {
+            mbar_init(&S.item_full[i], 1);
+            mbar_init(&S.item_empty[i], kQueueReaders);
+        }
         S.abort_flag = 0;
         fence_mbar_init();
     }
@@ -182,6 +192,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = S.tmem_base;
     volatile int *abort_flag = &S.abort_flag;
 
+    // Work items are claimed in order from one global counter, so every CTA
+    // works on neighbouring items (the same row range): the accumulator and Q
+    // rows of that range stay in L2.  Warp 0 claims and publishes each item;
+    // the MMA thread and the softmax warps read it from the queue.
+    long long *counter = MODE == 0 ? P.item_next : P.item_next + 1;
+    // n-th item for a reader; returns -1 on abort, total when the work is done.
+    auto next_item = [&](int n, bool warp_reader) -> long long {
+        const int slot = n % kQueue;
+        bool ok = !*abort_flag && mbar_wait(&S.item_full[slot], (n / kQueue) & 1, P.status);
+        if (warp_reader) ok = __all_sync(0xffffffffu, ok);
+        if (!ok) return -1;
+        const long long it = S.item_q[slot];
+        if (warp_reader) __syncwarp();
+        if (!warp_reader || lane == 0) mbar_arrive(&S.item_empty[slot]);
+        return it;
+    };
+
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (whole warp:
         // lane 0 owns the barriers, lane r gathers tile row r)
@@ -192,7 +219,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         int ki = 0, qt = 0;
         bool ok = true;
-        for (long long it = blockIdx.x; it < total && ok; it += gridDim.x) {
+        for (int n = 0; ok; ++n) {
+            long long it = 0;
+            if (lane == 0) {
+                const int slot = n % kQueue;
+                if (n >= kQueue && (*abort_flag || !mbar_wait(&S.item_empty[slot],
+                                                              ((n / kQueue) - 1) & 1, P.status))) {
+                    it = -1;
+                } else {
+                    it = atomicAdd(reinterpret_cast<unsigned long long *>(counter), 1ull);
+                    if (it > total) it = total;
+                    S.item_q[slot] = it;
+                    mbar_arrive(&S.item_full[slot]);
+                }
+            }
+            it = __shfl_sync(0xffffffffu, it, 0);
+            if (it < 0) { ok = false; break; }
+            if (it >= total) break;
             const Item x = item_at<MODE>(P, it);
             if (!x.valid) continue;
             const int kvs = ki & 1;
@@ -259,7 +302,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (last_of_item) umma_commit(&S.kv_empty[kvs]);
             return true;
         };
-        for (long long it = blockIdx.x; it < total && ok; it += gridDim.x) {
+        for (int n = 0; ok; ++n) {
+            const long long it = next_item(n, false);
+            if (it < 0) { ok = false; break; }
+            if (it >= total) break;
             const Item x = item_at<MODE>(P, it);
             if (!x.valid) continue;
             const int kvs = ki & 1;
@@ -297,7 +343,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (pv_pending >= 0) mbar_wait(&S.o_full[pv_pending & 1], (pv_pending >> 1) & 1, nullptr);
     } else if (warp >= 4) {
         // ------------------------------------------------ softmax + epilogue
-        const int m = tid - 128;                       // TMEM lane
+        // Warps 4-7 and 8-11 share the TMEM lanes of warp % 4 and split each
+        // row's 128 columns: ch = 0 takes tokens (and output dims) 0-63,
+        // ch = 1 takes 64-127.  Each half-row sum goes to the accumulator on
+        // its own, so the two warps never wait for each other.
+        const int ch = (warp - 4) >> 2;
+        const int m = (warp & 3) * 32 + lane;          // TMEM lane = tile row x head
         const int ri = m / kG, h = m % kG;             // tile row, head in group
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         const float sl2 = P.softmax_scale * kLog2e;
@@ -316,28 +367,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             have = __all_sync(0xffffffffu, have);
             if (!have) return false;
             tc_fence_after();
-            float *acc = P.o_acc + (row * P.H_kv + g) * (kDim * kG) + h * 4;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float v[32];
-                tmem_ld32(lane_addr + 256 + os * 128 + c * 32, v);
-                tmem_ld_wait();
-                if (valid) {
-#pragma unroll
-                    for (int q4 = 0; q4 < 8; ++q4) {
-                        float *dst = acc + (c * 8 + q4) * (4 * kG);
-                        if (MODE == 0)
-                            *reinterpret_cast<float4 *>(dst) =
-                                make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
-                        else
-                            red_add_v4(dst, v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
-                    }
-                }
-            }
+            uint32_t a[32], b[32];
+            tmem_ld32r(lane_addr + 256 + os * 128 + ch * 64, a);
+            tmem_ld32r(lane_addr + 256 + os * 128 + ch * 64 + 32, b);
+            tmem_wait_ld(a);
+            tmem_tie(b);
             if (valid) {
-                float *lp = P.l_acc + row * P.H_q + g * kG + h;
-                if (MODE == 0) *lp = l;
-                else atomicAdd(lp, l);
+                float *acc = P.o_acc + (row * P.H_kv + g) * (kDim * kG) + h * 4 + ch * 16 * (4 * kG);
+#pragma unroll
+                for (int q4 = 0; q4 < 16; ++q4) {
+                    const uint32_t *r = q4 < 8 ? a + 4 * q4 : b + 4 * (q4 - 8);
+                    float *dst = acc + q4 * (4 * kG);
+                    if (MODE == 0)
+                        *reinterpret_cast<float4 *>(dst) =
+                            make_float4(__uint_as_float(r[0]), __uint_as_float(r[1]),
+                                        __uint_as_float(r[2]), __uint_as_float(r[3]));
+                    else
+                        red_add_v4(dst, __uint_as_float(r[0]), __uint_as_float(r[1]),
+                                   __uint_as_float(r[2]), __uint_as_float(r[3]));
+                }
+                atomicAdd(P.l_acc + row * P.H_q + g * kG + h, l);
             }
             tc_fence_before();
             __syncwarp();
@@ -345,7 +394,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             return true;
         };
 
-        for (long long it = blockIdx.x; it < total && ok; it += gridDim.x) {
+        for (int n = 0; ok; ++n) {
+            const long long it = next_item(n, true);
+            if (it < 0) { ok = false; break; }
+            if (it >= total) break;
             const Item x = item_at<MODE>(P, it);
             if (!x.valid) continue;
             for (int t0 = 0; t0 < x.n; t0 += kTileRows, ++qt) {
@@ -353,61 +405,62 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool valid = t0 + ri < x.n;
                 const long long row = valid ? tile_row(P, x, t0 + ri) : 0;
                 // Pass B's shift is known before S: fetch it while the MMA runs.
-                float shift_b = 0.f;
-                if (MODE == 1 && valid) shift_b = P.m_arr[row * P.H_q + x.g * kG + h];
+                float shift = 0.f;
+                if (MODE == 1 && valid) shift = P.m_arr[row * P.H_q + x.g * kG + h];
                 bool have = !*abort_flag && mbar_wait(&S.s_full[ss], (qt >> 1) & 1, P.status);
                 have = __all_sync(0xffffffffu, have);
                 if (!have) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t sa = lane_addr + ss * 128;
-                float shift, l = 0.f;
-                long long p = 0;
+                long long lim = 127;                   // last visible column of the row
                 if (MODE == 0) {
                     // own block: causal mask t <= p, exact max of the visible logits
-                    p = static_cast<long long>(x.L) - P.Sq + (row - static_cast<long long>(x.b) * P.Sq);
-                    const long long lim = p - static_cast<long long>(x.j) * 128;   // last visible column
+                    const long long p = static_cast<long long>(x.L) - P.Sq +
+                                        (row - static_cast<long long>(x.b) * P.Sq);
+                    lim = p - static_cast<long long>(x.j) * 128;
                     float mx = -INFINITY;
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        float v[32];
-                        tmem_ld32(sa + c * 32, v);
-                        tmem_ld_wait();
+                    for (int c = 0; c < 4; c += 2) {
+                        uint32_t a[32], b[32];
+                        tmem_ld32r(sa + c * 32, a);
+                        tmem_ld32r(sa + c * 32 + 32, b);
+                        tmem_wait_ld(a);
+                        tmem_tie(b);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (c * 32 + e <= lim) mx = fmaxf(mx, v[e] * sl2);
+                        for (int e = 0; e < 32; ++e) {
+                            if (c * 32 + e <= lim) mx = fmaxf(mx, __uint_as_float(a[e]) * sl2);
+                            if (c * 32 + 32 + e <= lim) mx = fmaxf(mx, __uint_as_float(b[e]) * sl2);
+                        }
                     }
                     shift = valid ? mx : 0.f;
-                } else {
-                    shift = shift_b;
+                }
+                uint32_t a[32], b[32];
+                tmem_ld32r(sa + ch * 64, a);
+                tmem_ld32r(sa + ch * 64 + 32, b);
+                tmem_wait_ld(a);
+                tmem_tie(b);
+                float l = 0.f;
+                uint32_t pk[32];                        // 64 probabilities as bf16 pairs
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int c0 = ch * 64 + 2 * e;
+                    const uint32_t *src = e < 16 ? a : b;
+                    const int k = (2 * e) & 31;
+                    float p0 = exp2f(__uint_as_float(src[k]) * sl2 - shift);
+                    float p1 = exp2f(__uint_as_float(src[k + 1]) * sl2 - shift);
+                    p0 = (valid && c0 <= lim) ? p0 : 0.f;
+                    p1 = (valid && c0 + 1 <= lim) ? p1 : 0.f;
+                    l += p0 + p1;
+                    pk[e] = pack_bf16x2(p0, p1);
                 }
                 // P buffer is free once the previous tile's PV has read it.
                 bool pfree = !*abort_flag && (qt == 0 || mbar_wait(&S.p_empty, (qt - 1) & 1, P.status));
                 pfree = __all_sync(0xffffffffu, pfree);
                 if (!pfree) { ok = false; break; }
-                const long long lim = MODE == 0 ? p - static_cast<long long>(x.j) * 128 : 127;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    float v[32];
-                    tmem_ld32(sa + c * 32, v);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float z = v[e] * sl2 - shift;
-                        v[e] = (c * 32 + e <= lim && valid) ? exp2f(z) : 0.f;
-                        l += v[e];
-                    }
-                    // 32 tokens = 4 chunks of 8 in half c / 2
-#pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8) {
-                        const int chunk = (c & 1) * 4 + q8;
-                        uint4 w;
-                        w.x = pack_bf16x2(v[8 * q8 + 0], v[8 * q8 + 1]);
-                        w.y = pack_bf16x2(v[8 * q8 + 2], v[8 * q8 + 3]);
-                        w.z = pack_bf16x2(v[8 * q8 + 4], v[8 * q8 + 5]);
-                        w.w = pack_bf16x2(v[8 * q8 + 6], v[8 * q8 + 7]);
-                        *reinterpret_cast<uint4 *>(S.p + (c >> 1) * 16384 + swz128(m, chunk)) = w;
-                    }
-                }
+                for (int c8 = 0; c8 < 8; ++c8)
+                    *reinterpret_cast<uint4 *>(S.p + ch * 16384 + swz128(m, c8)) =
+                        make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
@@ -419,30 +472,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bool qok = !*abort_flag && mbar_wait(&S.q_full[qt & 1], (qt >> 1) & 1, P.status);
                     qok = __all_sync(0xffffffffu, qok);
                     if (!qok) { ok = false; break; }
-                }
-                if (MODE == 0 && valid) {
-                    // Shift of this (row, head) and the safety test of the bound.
-                    const uint8_t *qs = S.q[qt & 1];
-                    float nq = 0.f;
+                    if (ch == 0 && valid) {
+                        // Shift of this (row, head) and the safety test of the bound.
+                        const uint8_t *qs = S.q[qt & 1];
+                        float nq = 0.f;
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        const uint4 w = *reinterpret_cast<const uint4 *>(
-                            qs + (c >> 3) * 16384 + swz128(m, c & 7));
-                        const uint32_t a4[4] = {w.x, w.y, w.z, w.w};
+                        for (int c = 0; c < 16; ++c) {
+                            const uint4 w = *reinterpret_cast<const uint4 *>(
+                                qs + (c >> 3) * 16384 + swz128(m, c & 7));
+                            const uint32_t a4[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            nq = fmaf(bf16lo(a4[e]), bf16lo(a4[e]), nq);
-                            nq = fmaf(bf16hi(a4[e]), bf16hi(a4[e]), nq);
+                            for (int e = 0; e < 4; ++e) {
+                                nq = fmaf(bf16lo(a4[e]), bf16lo(a4[e]), nq);
+                                nq = fmaf(bf16hi(a4[e]), bf16hi(a4[e]), nq);
+                            }
                         }
+                        const float bound = fabsf(sl2) * sqrtf(nq) * P.knorm[x.b * P.H_kv + x.g];
+                        const long long idx = row * P.H_q + x.g * kG + h;
+                        P.m_arr[idx] = shift;
+                        const uint8_t fl = !(bound - shift <= kSafeLog2);   // NaN-safe
+                        P.flags[idx] = fl;
+                        if (fl) atomicAdd(P.flag_count, 1);
                     }
-                    const float bound = fabsf(sl2) * sqrtf(nq) * P.knorm[x.b * P.H_kv + x.g];
-                    const long long idx = row * P.H_q + x.g * kG + h;
-                    P.m_arr[idx] = shift;
-                    const uint8_t fl = !(bound - shift <= kSafeLog2);   // NaN-safe
-                    P.flags[idx] = fl;
-                    if (fl) atomicAdd(P.flag_count, 1);
-                }
-                if (MODE == 0) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S.q_empty[qt & 1]);
                 }
@@ -689,6 +740,7 @@ size_t prefill_workspace_layout(int B, int Sq, int H_q, int H_kv, int K, int max
     L->knorm = o;        o += up(static_cast<size_t>(B) * H_kv * 4);
     L->cnt = o;          o += up(static_cast<size_t>(L->n_buckets) * 4);
     L->cur = o;          o += up(static_cast<size_t>(L->n_buckets) * 4);
+    L->l_acc = o;        o += up(static_cast<size_t>(rows) * H_q * 4);
     L->zero_end = o;                                  // [knorm, zero_end) is cleared per call
     L->off = o;          o += up(static_cast<size_t>(L->n_buckets + 1) * 4);
     L->item_off = o;     o += up(static_cast<size_t>(L->n_buckets + 1) * 8);
@@ -696,7 +748,6 @@ size_t prefill_workspace_layout(int B, int Sq, int H_q, int H_kv, int K, int max
     o += up((static_cast<size_t>(L->n_buckets) + static_cast<size_t>(rows) * H_kv * K / kItemRows + 1) * 4);
     L->rows = o;         o += up(static_cast<size_t>(rows) * H_kv * (K > 1 ? K - 1 : 1) * 4);
     L->o_acc = o;        o += up(static_cast<size_t>(rows) * H_q * kDim * 4);
-    L->l_acc = o;        o += up(static_cast<size_t>(rows) * H_q * 4);
     L->m_arr = o;        o += up(static_cast<size_t>(rows) * H_q * 4);
     L->flags = o;        o += up(static_cast<size_t>(rows) * H_q);
     L->total = o;
@@ -719,6 +770,7 @@ cudaError_t launch_prefill_attention(const PrefillArgs &a0, uint8_t *ws, const P
     a.flags = reinterpret_cast<uint8_t *>(ws + L.flags);
     a.flag_count = reinterpret_cast<int *>(ws + 4);
     a.item_total = reinterpret_cast<long long *>(ws + 8);
+    a.item_next = reinterpret_cast<long long *>(ws + 16);   // [pass A, pass B]
     a.nb_max = L.nb_max;
     a.n_ranges = L.n_ranges;
     a.n_buckets = L.n_buckets;

@@ -108,6 +108,7 @@ struct PrefillArgs {
     long long *item_off;
     int *item_bucket;       // bucket of every pass-B work item
     long long *item_total;
+    long long *item_next;   // claim counters of pass A and pass B (zeroed per call)
     float *o_acc, *l_acc, *m_arr;
     uint8_t *flags;
     int *flag_count;
