@@ -10,8 +10,9 @@
 //
 // Design (decode and short prefill):
 //   - warp 4 (one thread) TMA-loads each kept block's K and V tile of the
-//     group (3-D tensor maps, 128-byte swizzle, 4 x 16 KiB) into a 2-stage
-//     ring; the tile is shared by the G = H_q/H_kv heads of the group;
+//     group (3-D tensor maps, 128-byte swizzle, 4 x 16 KiB) into a 1- or
+//     2-stage ring (one stage when a CTA owns a single block, so three CTAs
+//     share an SM); the tile is shared by the G = H_q/H_kv heads of the group;
 //   - warps 0-3 each own 32 of the block's 128 tokens and run the swapped
 //     products on mma.sync m16n8k16 bf16: S^T = K Q^T (tokens x heads, heads
 //     fill N = 8) and O^T += V^T P^T, with P^T moved from the accumulator
@@ -27,13 +28,12 @@ namespace {
 
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kStages = 2;
 constexpr int kHalf = 16384;              // 128 tokens x 64 dims x bf16
 constexpr int kStageBytes = 4 * kHalf;    // K lo/hi + V lo/hi
 constexpr int kMaxK = 64;
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int NT>
+template <int NT, int kStages>
 struct Smem {
     uint8_t ring[kStages][kStageBytes];   // reused as the merge area at the end
     __nv_bfloat16 q[NT * 8][kDim];
@@ -56,13 +56,13 @@ __device__ __forceinline__ void consumers_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
 }
 
-template <int NT>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int NT, int kStages>
+__global__ void __launch_bounds__(kThreads, kStages == 1 ? 3 : 1)
     attn_rows_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const AttnRowsArgs P) {
     extern __shared__ uint8_t smem_raw[];
-    Smem<NT> &S = *reinterpret_cast<Smem<NT> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                ~uintptr_t(1023));
+    Smem<NT, kStages> &S = *reinterpret_cast<Smem<NT, kStages> *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = P.H_q / P.H_kv;
     const long long cta = blockIdx.x;
@@ -395,28 +395,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int NT>
+template <int NT, int STAGES>
 cudaError_t launch_nt(const AttnRowsArgs &a, cudaStream_t s) {
-    static_assert(sizeof(Merge<NT>) <= kStages * kStageBytes, "merge area fits in the ring");
-    static_assert(sizeof(Smem<NT>) + 1024 <= 227 * 1024, "shared memory budget");
+    static_assert(sizeof(Merge<NT>) <= STAGES * kStageBytes, "merge area fits in the ring");
+    static_assert(sizeof(Smem<NT, STAGES>) + 1024 <= 227 * 1024, "shared memory budget");
     CUtensorMap tk, tv;
     if (!encode_kv_tensor_map(&tk, a.k_cache, a.H_kv, a.capacity) ||
         !encode_kv_tensor_map(&tv, a.v_cache, a.H_kv, a.capacity))
         return cudaErrorInvalidValue;
-    const size_t smem = sizeof(Smem<NT>) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(attn_rows_kernel<NT>,
+    const size_t smem = sizeof(Smem<NT, STAGES>) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(attn_rows_kernel<NT, STAGES>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long long ctas = static_cast<long long>(a.B) * a.Sq * a.H_kv * a.nsplit;
     TraceScope trace(s, "sparse_attention_rows");
-    attn_rows_kernel<NT><<<static_cast<unsigned>(ctas), kThreads, smem, s>>>(tk, tv, a);
+    attn_rows_kernel<NT, STAGES><<<static_cast<unsigned>(ctas), kThreads, smem, s>>>(tk, tv, a);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 int attn_rows_nsplit(long long rows_x_groups, int top_k) {
-    // Aim at two CTAs per SM of a 148-SM part; at least one block per split.
+    // Few kept blocks in total (decode of a modest batch): one block per CTA,
+    // single-stage CTAs of ~70 KiB so three fit on an SM and every block's
+    // load is in flight at once.
+    if (rows_x_groups * top_k <= 1536) return top_k;
+    // Otherwise aim at two CTAs per SM of a 148-SM part.
     long long want = (2 * 148 + rows_x_groups - 1) / rows_x_groups;
     if (want < 1) want = 1;
     if (want > top_k) want = top_k;
@@ -426,8 +430,9 @@ int attn_rows_nsplit(long long rows_x_groups, int top_k) {
 
 cudaError_t launch_attn_rows(const AttnRowsArgs &a, cudaStream_t s) {
     const int G = a.H_q / a.H_kv;
-    if (G <= 8) return launch_nt<1>(a, s);
-    if (G <= 16) return launch_nt<2>(a, s);
+    const bool one = (a.K + a.nsplit - 1) / a.nsplit == 1;   // one block per CTA
+    if (G <= 8) return one ? launch_nt<1, 1>(a, s) : launch_nt<1, 2>(a, s);
+    if (G <= 16) return one ? launch_nt<2, 1>(a, s) : launch_nt<2, 2>(a, s);
     return cudaErrorInvalidValue;
 }
 

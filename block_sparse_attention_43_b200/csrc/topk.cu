@@ -9,10 +9,10 @@
 //
 // Selection runs on 64-bit keys (order-preserving score bits, complemented
 // id) so the order is total and the result is independent of the algorithm.
-// Each warp finds its m = k-1 best keys by repeated warp argmax: every lane
-// keeps the best key of its own candidates below the last winner, and only
-// the winning lane rescans.  Long rows are split over the 8 warps of a CTA
-// and the 8 partial lists are merged the same way by warp 0.
+// Each warp finds its m = k-1 best keys by repeated warp argmax over per-lane
+// register caches; long rows are split over the 8 warps of a CTA and the 8
+// partial lists are merged the same way by warp 0.  Prefill rows select
+// inside the tensor-core index kernel; this kernel serves decode.
 #include "msa_device.cuh"
 #include "msa_internal.h"
 
@@ -22,42 +22,64 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kMaxK = 64;
 
-// Best key < bound among scores[j] for j = lo + lane + 32 i, j < hi.
-__device__ __forceinline__ unsigned long long lane_best(const float *scores, int lo, int hi,
-                                                        int lane, unsigned long long bound) {
-    unsigned long long best = 0;
+// Keys are read once: every lane streams its candidates j = lo + lane + 32 i
+// (coalesced) and keeps its own best kCache keys in registers.  The warp then
+// takes its m best by repeated warp argmax over the lanes' heads; the winner
+// pops its head and, in the rare case its cache runs dry while it still has
+// candidates, rescans them below the last key it gave up.
+constexpr int kCache = 4;
+
+struct LaneTop {
+    unsigned long long k[kCache];
+    int popped;      // keys taken from this lane so far
+};
+
+template <typename Key>
+__device__ __forceinline__ void lane_fill(LaneTop &t, Key key_at, int lo, int hi, int lane,
+                                          unsigned long long bound) {
+#pragma unroll
+    for (int i = 0; i < kCache; ++i) t.k[i] = 0;
     for (int j = lo + lane; j < hi; j += 32) {
-        const unsigned long long k = topk_key(__ldg(scores + j), j);
-        if (k < bound && k > best) best = k;
+        unsigned long long x = key_at(j);
+        if (x >= bound || x <= t.k[kCache - 1]) continue;
+#pragma unroll
+        for (int i = 0; i < kCache; ++i) {
+            const unsigned long long hi_k = t.k[i] > x ? t.k[i] : x;
+            x = t.k[i] > x ? x : t.k[i];
+            t.k[i] = hi_k;
+        }
     }
-    return best;
 }
 
-// Best key < bound among list[i], i = lane + 32 q < n.
-__device__ __forceinline__ unsigned long long lane_best_list(const unsigned long long *list, int n,
-                                                             int lane, unsigned long long bound) {
-    unsigned long long best = 0;
-    for (int i = lane; i < n; i += 32) {
-        const unsigned long long k = list[i];
-        if (k < bound && k > best) best = k;
-    }
-    return best;
-}
-
-// The m best keys of this warp's candidates, descending, written to out[0..m)
-// (0 where the warp has fewer than m candidates).
-template <typename Best>
-__device__ __forceinline__ void warp_select(Best best_below, int m, int lane,
+// The m best keys of the warp's candidates [lo, hi), descending, into out[0..m)
+// (0 where there are fewer than m candidates).
+template <typename Key>
+__device__ __forceinline__ void warp_select(Key key_at, int lo, int hi, int m, int lane,
                                             unsigned long long *out) {
-    unsigned long long mine = best_below(~0ull);
+    LaneTop t;
+    lane_fill(t, key_at, lo, hi, lane, ~0ull);
+    const int mine_total = hi - lo > lane ? (hi - lo - lane + 31) / 32 : 0;
+    int have = mine_total < kCache ? mine_total : kCache;   // cached keys not yet popped
+    t.popped = 0;
     for (int q = 0; q < m; ++q) {
-        const unsigned long long top = warp_max_u64(mine);
+        const unsigned long long head = t.k[0];
+        const unsigned long long top = warp_max_u64(head);
         if (lane == 0) out[q] = top;
         if (top == 0) {
             for (int r = q + 1 + lane; r < m; r += 32) out[r] = 0;
             break;
         }
-        if (mine == top) mine = best_below(top);   // keys are unique: one lane
+        if (head == top) {                      // keys are unique: exactly one lane
+#pragma unroll
+            for (int i = 0; i < kCache - 1; ++i) t.k[i] = t.k[i + 1];
+            t.k[kCache - 1] = 0;
+            ++t.popped;
+            --have;
+            if (have == 0 && t.popped < mine_total) {
+                lane_fill(t, key_at, lo, hi, lane, top);
+                have = min(kCache, mine_total - t.popped);
+            }
+        }
         __syncwarp();
     }
     __syncwarp();
@@ -126,8 +148,8 @@ __global__ void __launch_bounds__(kWarps * 32) topk_warp_kernel(const TopkArgs P
         n = own + 1;
     } else {
         const int m = K - 1;
-        warp_select([&](unsigned long long bound) { return lane_best(scores, 0, own, lane, bound); },
-                    m, lane, keys[warp]);
+        warp_select([&](int j) { return topk_key(__ldg(scores + j), j); }, 0, own, m, lane,
+                    keys[warp]);
         for (int q = lane; q < m; q += 32) sel[warp][q] = topk_key_id(keys[warp][q]);
         if (lane == 0) sel[warp][m] = own;
         n = K;
@@ -168,13 +190,11 @@ __global__ void __launch_bounds__(kWarps * 32) topk_cta_kernel(const TopkArgs P)
     const int m = K - 1;
     const int chunk = (own + kWarps - 1) / kWarps;
     const int lo = min(own, warp * chunk), hi = min(own, lo + chunk);
-    warp_select([&](unsigned long long bound) { return lane_best(scores, lo, hi, lane, bound); }, m,
-                lane, part + warp * m);
+    warp_select([&](int j) { return topk_key(__ldg(scores + j), j); }, lo, hi, m, lane,
+                part + warp * m);
     __syncthreads();
     if (warp == 0) {
-        warp_select(
-            [&](unsigned long long bound) { return lane_best_list(part, kWarps * m, lane, bound); }, m,
-            lane, fin);
+        warp_select([&](int i) { return part[i]; }, 0, kWarps * m, m, lane, fin);
         for (int q = lane; q < m; q += 32) sel[q] = topk_key_id(fin[q]);
         if (lane == 0) sel[m] = own;
         __syncwarp();
