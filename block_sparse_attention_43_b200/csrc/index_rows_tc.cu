@@ -10,7 +10,7 @@
 //
 // Tiling: a work unit is (sequence, group, 128 query rows).  The unit's index
 // queries (32 KiB) sit in shared memory; its visible key blocks stream through
-// a 3-stage ring two blocks (64 KiB) at a time.  One thread issues
+// a 2-stage ring two blocks (64 KiB) at a time.  One thread issues
 // tcgen05.mma kind::f16 M=128, N=256 (or 128 for a lone last block), K=128 as
 // eight K=16 steps into one of two 256-column fp32 TMEM accumulators, and
 // commits to mbarriers.  Four epilogue warps (one TMEM lane = one query row
@@ -23,22 +23,27 @@
 // to a persistent grid in snake order of decreasing length.
 //
 // Roles: warp 0 = TMA producer, warp 1 = MMA issuer, warp 2 = TMEM owner,
-// warps 4-7 = epilogue (warp % 4 selects its 32 TMEM lanes).
+// warps 4-7 and 8-11 = two epilogue warpgroups on alternate accumulator
+// buffers (warp % 4 selects a warp's 32 TMEM lanes).
 #include "msa_device.cuh"
 #include "msa_internal.h"
 
 namespace msa {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kStages = 3;
+constexpr int kThreads = 384;               // 4 control warps + 2 epilogue warpgroups
+constexpr int kStages = 2;
 constexpr int kQBytes = 2 * 16384;          // 128 rows x 128 dims, two swizzled halves
 constexpr int kStageBytes = 2 * 32768;      // two key blocks: [256 rows x 128 B] per half
 constexpr uint32_t kTmemCols = 512;         // two 256-column accumulators
 
+template <int LIST>
 struct Smem {
     uint8_t q[kQBytes];
     uint8_t ring[kStages][kStageBytes];
+    unsigned long long xkeys[LIST][128];        // warpgroup 1's list, handed to warpgroup 0
+    float xown[128];
+    int xhas[128];
     uint64_t k_full[kStages], k_empty[kStages];
     uint64_t q_full, q_empty;
     uint64_t acc_full[2], acc_empty[2];
@@ -111,8 +116,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     index_rows_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK, const IndexRowsArgs P) {
     extern __shared__ uint8_t smem_raw[];
-    Smem &S = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                        ~uintptr_t(1023));
+    Smem<LIST> &S = *reinterpret_cast<Smem<LIST> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                    ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ntiles = (P.Sq + 127) / 128;
     const long long nunits = static_cast<long long>(ntiles) * P.B * P.H_kv;
@@ -126,7 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&S.q_empty, 1);
         for (int a = 0; a < 2; ++a) {
             mbar_init(&S.acc_full[a], 1);
-            mbar_init(&S.acc_empty[a], 4);
+            mbar_init(&S.acc_empty[a], 4);          // the four warps of the owning warpgroup
         }
         S.abort_flag = 0;
         fence_mbar_init();
@@ -227,13 +232,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= 4) {
         // ------------------------------------------------ epilogue
-        const int r = tid - 128;                     // TMEM lane = tile row
+        // Two warpgroups take alternate accumulator buffers (pairs of key
+        // blocks).  Each keeps its own running list per row; at the end of a
+        // unit warpgroup 1 hands its list to warpgroup 0, which merges and
+        // writes the row's selection.  A warpgroup that hits a timeout keeps
+        // stepping through the unit-end barriers so the other never waits on it.
+        const int wg = (warp - 4) >> 2;
+        const int r = (warp & 3) * 32 + lane;        // TMEM lane = tile row
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         const int keep = P.K - 1;                    // non-own blocks kept per row
         TopList<LIST> top;
         int ita = 0;
         bool ok = true;
-        for (int rr = 0; ok; ++rr) {
+        for (int rr = 0;; ++rr) {
             const long long u = unit_index(rr);
             if (u >= nunits) break;
             const Unit x = unit_at(P, u, ntiles);
@@ -241,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const long long out_off =
                 ((static_cast<long long>(x.b) * P.Sq + x.i0 + r) * P.H_kv + x.g) * P.K;
             if (!x.valid) {
-                if (row_ok)
+                if (row_ok && wg == 0)
                     for (int q = 0; q < P.K; ++q) {
                         P.ids[out_off + q] = -1;
                         P.out_scores[out_off + q] = -INFINITY;
@@ -251,41 +262,69 @@ __global__ void __launch_bounds__(kThreads, 1)
             const long long p = x.p_first + r;        // this row's query position
             const int own = static_cast<int>(p / kBlock);
             float s_own = -INFINITY;
+            bool has_own = false;
             top.reset(keep);
             for (int j = 0; j <= x.jmax; j += 2, ++ita) {
                 const int a = ita & 1;
-                bool have = !*abort_flag && mbar_wait(&S.acc_full[a], (ita >> 1) & 1, P.status);
-                have = __all_sync(0xffffffffu, have);
-                if (!have) { ok = false; break; }
-                tc_fence_after();
-                const int nb = min(2, x.jmax - j + 1);
-                for (int jj = 0; jj < nb; ++jj) {
-                    const int J = j + jj;
-                    const long long t0 = static_cast<long long>(J) * kBlock;
-                    const bool full = t0 + kBlock - 1 <= x.p_first;     // no masking for any row
-                    float m = -INFINITY;
+                if (a != wg) continue;
+                if (ok) {
+                    bool have = !*abort_flag && mbar_wait(&S.acc_full[a], (ita >> 1) & 1, P.status);
+                    have = __all_sync(0xffffffffu, have);
+                    if (!have) { ok = false; *abort_flag = 1; }
+                }
+                if (ok) {
+                    tc_fence_after();
+                    const int nb = min(2, x.jmax - j + 1);
+                    for (int jj = 0; jj < nb; ++jj) {
+                        const int J = j + jj;
+                        const long long t0 = static_cast<long long>(J) * kBlock;
+                        const bool full = t0 + kBlock - 1 <= x.p_first;   // no masking for any row
+                        float m = -INFINITY;
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        float v[32];
-                        tmem_ld32(lane_addr + a * 256 + jj * 128 + c * 32, v);
-                        tmem_ld_wait();
-                        if (full) {
+                        for (int c = 0; c < 4; c += 2) {
+                            uint32_t va[32], vb[32];
+                            tmem_ld32r(lane_addr + a * 256 + jj * 128 + c * 32, va);
+                            tmem_ld32r(lane_addr + a * 256 + jj * 128 + c * 32 + 32, vb);
+                            tmem_wait_ld(va);
+                            tmem_tie(vb);
+                            if (full) {
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) m = fmaxf(m, v[e]);
-                        } else {
+                                for (int e = 0; e < 32; ++e)
+                                    m = fmaxf(m, fmaxf(__uint_as_float(va[e]), __uint_as_float(vb[e])));
+                            } else {
 #pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                if (t0 + c * 32 + e <= p) m = fmaxf(m, v[e]);
+                                for (int e = 0; e < 32; ++e) {
+                                    if (t0 + c * 32 + e <= p) m = fmaxf(m, __uint_as_float(va[e]));
+                                    if (t0 + c * 32 + 32 + e <= p) m = fmaxf(m, __uint_as_float(vb[e]));
+                                }
+                            }
                         }
+                        if (J < own) top.offer(topk_key(m, J));
+                        else if (J == own) { s_own = m; has_own = true; }
                     }
-                    if (J < own) top.offer(topk_key(m, J));
-                    else if (J == own) s_own = m;
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.acc_empty[a]);
             }
-            if (!ok || !row_ok) continue;
+            // Warpgroup 1 hands over its list; warpgroup 0 merges and writes.
+            if (wg == 1) {
+#pragma unroll
+                for (int i = 0; i < LIST; ++i) S.xkeys[i][r] = top.L[i];
+                S.xown[r] = s_own;
+                S.xhas[r] = has_own;
+            }
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (wg == 0) {
+#pragma unroll
+                for (int i = 0; i < LIST; ++i) {
+                    const unsigned long long k2 = S.xkeys[i][r];
+                    if (k2 != 0ull && k2 != ~0ull) top.offer(k2);
+                }
+                if (S.xhas[r]) s_own = S.xown[r];
+            }
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (wg != 0 || !ok || !row_ok) continue;
             // Kept non-own blocks (all ids < own) ascending, then the own block.
             // They sit in slots [LIST - keep, LIST - keep + n_other), best first.
             const int n_other = min(own, keep);
@@ -324,16 +363,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_index_rows_tc(const IndexRowsArgs &a, cudaStream_t s) {
-    static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "shared memory budget");
+    static_assert(sizeof(Smem<64>) + 1024 <= 227 * 1024, "shared memory budget");
     CUtensorMap tq, tk;
     if (!encode_kv_tensor_map(&tq, a.q_idx, a.H_kv, static_cast<long long>(a.B) * a.Sq) ||
         !encode_kv_tensor_map(&tk, a.k_idx, a.H_kv, a.capacity))
         return cudaErrorInvalidValue;
-    const size_t smem = sizeof(Smem) + 1024;
     const long long ntiles = (a.Sq + 127) / 128;
     const long long units = ntiles * a.B * a.H_kv;
     const long long grid = units < device_sm_count() ? units : device_sm_count();
-    auto go = [&](auto kern) -> cudaError_t {
+    auto go = [&](auto kern, size_t smem) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
@@ -341,9 +379,9 @@ cudaError_t launch_index_rows_tc(const IndexRowsArgs &a, cudaStream_t s) {
         kern<<<static_cast<unsigned>(grid), kThreads, smem, s>>>(tq, tk, a);
         return cudaGetLastError();
     };
-    if (a.K <= 16) return go(index_rows_tc_kernel<16>);
-    if (a.K <= 32) return go(index_rows_tc_kernel<32>);
-    if (a.K <= 64) return go(index_rows_tc_kernel<64>);
+    if (a.K <= 16) return go(index_rows_tc_kernel<16>, sizeof(Smem<16>) + 1024);
+    if (a.K <= 32) return go(index_rows_tc_kernel<32>, sizeof(Smem<32>) + 1024);
+    if (a.K <= 64) return go(index_rows_tc_kernel<64>, sizeof(Smem<64>) + 1024);
     return cudaErrorInvalidValue;
 }
 
