@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--prefill-steps", type=int, default=5)
     ap.add_argument("--prefill-len", type=int, default=None,
                     help="override the prefill length (profiling captures of a smaller case)")
+    ap.add_argument("--decode-len", type=int, default=None,
+                    help="override the decode context length (profiling captures of a smaller case)")
     return ap.parse_args()
 
 
@@ -326,7 +328,15 @@ def main():
     dist, rank, local, world = dist_setup(args)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    w = make_workload(args.workload, dev)
+    if args.decode_len is None:
+        w = make_workload(args.workload, dev)
+    else:
+        from synthetic import WORKLOADS, make_inputs
+        c = WORKLOADS[args.workload]
+        w = make_inputs(B=c["B"], Sq=1, lens=[args.decode_len] * c["B"], H_q=c["H_q"],
+                        H_kv=c["H_kv"], top_k=c["top_k"], seed=c["seed"], device=dev,
+                        name=f"{args.workload}@{args.decode_len}", needles=c.get("needles", 0),
+                        amp=c.get("amp", 4.0))
     if world > 1:
         # independent batch per rank: perturb q so ranks differ
         w.q_idx.mul_(1.0 + 0.001 * rank)

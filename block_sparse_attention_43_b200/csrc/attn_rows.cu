@@ -89,26 +89,38 @@ __global__ void __launch_bounds__(kThreads, kStages == 1 ? 3 : 1)
     const int bps = (P.K + P.nsplit - 1) / P.nsplit;
 
     if (tid == 0) {
-        // Kept ids of this (row, group), -1 skipped, then this split's share.
-        const int32_t *ids = P.ids + pair * P.K;
-        int n = 0, bad = 0;
-        int list[kMaxK];
-        for (int q = 0; q < P.K; ++q) {
-            const int j = ids[q];
-            if (j < 0) { bad |= (j != -1); continue; }
-            if (j > own) { bad = 1; continue; }
-            list[n++] = j;
-        }
-        if (bad) set_status(P.status, kStatusBadLens);
-        const int lo = min(n, split * bps), hi = min(n, lo + bps);
-        for (int q = lo; q < hi; ++q) S.blocks[q - lo] = list[q];
-        S.nblk = hi - lo;
-        S.abort_flag = 0;
+        // Kept ids of this (row, group), -1 skipped, then this split's share;
+        // the first blocks' TMA loads go out before anything else is set up.
         for (int st = 0; st < kStages; ++st) {
             mbar_init(&S.full[st], 1);
             mbar_init(&S.empty[st], kConsumerWarps);
         }
         fence_mbar_init();
+        S.abort_flag = 0;
+        const int32_t *ids = P.ids + pair * P.K;
+        const int lo = split * bps, hi = lo + bps;
+        int n = 0, bad = 0, nblk = 0;
+        for (int q = 0; q < P.K; ++q) {
+            const int j = __ldg(ids + q);
+            if (j < 0) { bad |= (j != -1); continue; }
+            if (j > own) { bad = 1; continue; }
+            if (n >= lo && n < hi) {
+                S.blocks[nblk] = j;
+                if (nblk < kStages) {
+                    const int tok = static_cast<int>(off + (long long)j * kBlock);
+                    uint8_t *dst = S.ring[nblk];
+                    mbar_arrive_expect_tx(&S.full[nblk], kStageBytes);
+                    tma_load_3d(dst, &tmK, 0, g, tok, &S.full[nblk]);
+                    tma_load_3d(dst + kHalf, &tmK, 64, g, tok, &S.full[nblk]);
+                    tma_load_3d(dst + 2 * kHalf, &tmV, 0, g, tok, &S.full[nblk]);
+                    tma_load_3d(dst + 3 * kHalf, &tmV, 64, g, tok, &S.full[nblk]);
+                }
+                ++nblk;
+            }
+            ++n;
+        }
+        if (bad) set_status(P.status, kStatusBadLens);
+        S.nblk = nblk;
     }
     // Q rows of the group's heads (zero rows pad G up to 8 * NT).
     {
@@ -126,11 +138,9 @@ __global__ void __launch_bounds__(kThreads, kStages == 1 ? 3 : 1)
 
     if (warp == kConsumerWarps) {
         // ------------------------------------------------ producer
-        if (lane == 0 && nblk > 0) {
-            prefetch_tensormap(&tmK);
-            prefetch_tensormap(&tmV);
+        if (lane == 0 && nblk > kStages) {
             bool ok = true;
-            int it = 0;
+            int it = kStages;                      // the first stages were issued above
             for (; it < nblk; ++it) {
                 const int st = it % kStages;
                 if (it >= kStages &&
@@ -326,7 +336,8 @@ __global__ void __launch_bounds__(kThreads, kStages == 1 ? 3 : 1)
 
     // Thread -> (head, 8 dims); heads beyond G are padding and skipped.
     const int nthr = kConsumerWarps * 32;
-    const int rec = G * (kDim + 2);                 // floats per split partial
+    const int rec = attn_partial_floats(G);         // floats per split partial
+    const int ooff = attn_partial_o_offset(G);
     float *part = P.partials + (pair * P.nsplit) * rec;
     for (int e = tid; e < G * (kDim / 8); e += nthr) {
         const int h = e / (kDim / 8), d0 = (e % (kDim / 8)) * 8;
@@ -355,15 +366,15 @@ __global__ void __launch_bounds__(kThreads, kStages == 1 ? 3 : 1)
             float *pr = part + split * rec;
             if (d0 == 0) { pr[h] = mx; pr[G + h] = aborted ? NAN : l; }
 #pragma unroll
-            for (int x = 0; x < 8; ++x) pr[2 * G + h * kDim + d0 + x] = o[x];
+            for (int x = 0; x < 8; ++x) pr[ooff + h * kDim + d0 + x] = o[x];
         }
     }
     if (P.nsplit == 1) return;
 
     // ------------------------------------------------ last CTA merges splits
-    __threadfence();
-    consumers_sync();
+    consumers_sync();                     // every partial of this CTA is written
     if (tid == 0) {
+        __threadfence();                  // ... and visible before the ticket
         const int t = atomicAdd(P.tickets + pair, 1);
         S.last = (t == P.nsplit - 1);
         if (S.last) P.tickets[pair] = 0;
@@ -371,19 +382,42 @@ __global__ void __launch_bounds__(kThreads, kStages == 1 ? 3 : 1)
     consumers_sync();
     if (!S.last) return;
     __threadfence();
+    // Splits are read eight at a time with every load issued before its use.
     for (int e = tid; e < G * (kDim / 8); e += nthr) {
         const int h = e / (kDim / 8), d0 = (e % (kDim / 8)) * 8;
         float mx = -INFINITY;
-        for (int sp = 0; sp < P.nsplit; ++sp) mx = fmaxf(mx, __ldcg(part + sp * rec + h));
+        for (int s0 = 0; s0 < P.nsplit; s0 += 8) {
+            float mv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                mv[u] = s0 + u < P.nsplit ? __ldcg(part + (s0 + u) * rec + h) : -INFINITY;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) mx = fmaxf(mx, mv[u]);
+        }
         const float mref = mx == -INFINITY ? 0.f : mx;
         float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         float l = 0.f;
-        for (int sp = 0; sp < P.nsplit; ++sp) {
-            const float *pr = part + sp * rec;
-            const float wt = exp2f(__ldcg(pr + h) - mref);
-            l += wt * __ldcg(pr + G + h);
+        for (int s0 = 0; s0 < P.nsplit; s0 += 8) {
+            float mv[8], lv[8];
+            float4 ov[8][2];
 #pragma unroll
-            for (int x = 0; x < 8; ++x) o[x] += wt * __ldcg(pr + 2 * G + h * kDim + d0 + x);
+            for (int u = 0; u < 8; ++u) {
+                const bool in = s0 + u < P.nsplit;
+                const float *pr = part + (in ? s0 + u : 0) * rec;
+                mv[u] = in ? __ldcg(pr + h) : -INFINITY;
+                lv[u] = __ldcg(pr + G + h);
+                ov[u][0] = __ldcg(reinterpret_cast<const float4 *>(pr + ooff + h * kDim + d0));
+                ov[u][1] = __ldcg(reinterpret_cast<const float4 *>(pr + ooff + h * kDim + d0 + 4));
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float wt = exp2f(mv[u] - mref);          // 0 for splits past the end
+                l += wt * lv[u];
+                o[0] += wt * ov[u][0].x; o[1] += wt * ov[u][0].y;
+                o[2] += wt * ov[u][0].z; o[3] += wt * ov[u][0].w;
+                o[4] += wt * ov[u][1].x; o[5] += wt * ov[u][1].y;
+                o[6] += wt * ov[u][1].z; o[7] += wt * ov[u][1].w;
+            }
         }
         const float inv = 1.f / l;
         uint4 v;

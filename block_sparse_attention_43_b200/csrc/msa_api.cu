@@ -143,7 +143,8 @@ AttnLayout attn_layout(const msa_shape_t *s) {
     L.tickets_off = kWsHeaderBytes;
     L.tickets_bytes = L.nsplit > 1 ? round_up(static_cast<size_t>(pairs) * sizeof(int)) : 0;
     L.partials_off = L.tickets_off + L.tickets_bytes;
-    const size_t part = L.nsplit > 1 ? static_cast<size_t>(pairs) * L.nsplit * G * (kDim + 2) * 4 : 0;
+    const size_t part =
+        L.nsplit > 1 ? static_cast<size_t>(pairs) * L.nsplit * attn_partial_floats(G) * 4 : 0;
     L.total = L.partials_off + round_up(part);
     return L;
 }

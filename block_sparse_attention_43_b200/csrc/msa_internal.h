@@ -88,6 +88,10 @@ struct AttnRowsArgs {
 cudaError_t launch_attn_rows(const AttnRowsArgs &a, cudaStream_t s);
 // Splits used by launch_attn_rows for this shape (workspace sizing too).
 int attn_rows_nsplit(long long rows_x_groups, int top_k);
+// Floats of one split partial for G heads: m[G], l[G], padding to 16 bytes,
+// then o[G][128] (so the o rows can be read as float4).
+__host__ __device__ inline int attn_partial_floats(int G) { return ((2 * G + 3) & ~3) + G * 128; }
+__host__ __device__ inline int attn_partial_o_offset(int G) { return (2 * G + 3) & ~3; }
 
 // Prefill sparse attention organised around the KV blocks (attn_prefill.cu).
 struct PrefillArgs {

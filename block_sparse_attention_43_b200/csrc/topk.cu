@@ -39,14 +39,24 @@ __device__ __forceinline__ void lane_fill(LaneTop &t, Key key_at, int lo, int hi
                                           unsigned long long bound) {
 #pragma unroll
     for (int i = 0; i < kCache; ++i) t.k[i] = 0;
-    for (int j = lo + lane; j < hi; j += 32) {
-        unsigned long long x = key_at(j);
-        if (x >= bound || x <= t.k[kCache - 1]) continue;
+    // Eight independent loads in flight per round, then eight inserts.
+    for (int base = lo + lane; base < hi; base += 32 * 8) {
+        unsigned long long xs[8];
 #pragma unroll
-        for (int i = 0; i < kCache; ++i) {
-            const unsigned long long hi_k = t.k[i] > x ? t.k[i] : x;
-            x = t.k[i] > x ? x : t.k[i];
-            t.k[i] = hi_k;
+        for (int u = 0; u < 8; ++u) {
+            const int j = base + 32 * u;
+            xs[u] = j < hi ? key_at(j) : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            unsigned long long x = xs[u];
+            if (x >= bound || x <= t.k[kCache - 1]) continue;
+#pragma unroll
+            for (int i = 0; i < kCache; ++i) {
+                const unsigned long long hi_k = t.k[i] > x ? t.k[i] : x;
+                x = t.k[i] > x ? x : t.k[i];
+                t.k[i] = hi_k;
+            }
         }
     }
 }
