@@ -122,14 +122,21 @@ __device__ __forceinline__ Item item_at(const PrefillArgs &P, long long it) {
         x.i_lo = static_cast<int>(plo - p0);
         x.valid = x.n > 0;
     } else {
-        const long long bucket = P.item_bucket[it];
-        const int chunk = static_cast<int>(it - P.item_off[bucket]);
+        // range of the item (binary search over the ranges' item offsets), then
+        // its bucket (block j) and chunk inside the range
+        long long lo = 0, hi = P.n_ranges_total;
+        while (hi - lo > 1) {
+            const long long mid = (lo + hi) >> 1;
+            if (P.range_item_off[mid] <= it) lo = mid; else hi = mid;
+        }
+        const long long r = lo;
+        const int local = static_cast<int>(it - P.range_item_off[r]);
+        x.j = P.item_bucket[r * P.items_per_range + local];
+        const long long bucket = r * P.nb_max + x.j;
+        const int chunk = local - P.item_off[bucket];
         const int cnt = P.bucket_cnt[bucket];
-        x.j = static_cast<int>(bucket % P.nb_max);
-        long long t = bucket / P.nb_max;
-        t /= P.n_ranges;
-        x.g = static_cast<int>(t % P.H_kv);
-        x.b = static_cast<int>(t / P.H_kv);
+        x.g = static_cast<int>((r / P.n_ranges) % P.H_kv);
+        x.b = static_cast<int>(r / (static_cast<long long>(P.n_ranges) * P.H_kv));
         x.n = min(kItemRows, cnt - chunk * kItemRows);
         x.rows = P.bucket_rows + P.bucket_off[bucket] + static_cast<long long>(chunk) * kItemRows;
         x.valid = x.n > 0 && seq_ok(P, x.b, x.L, x.off);
@@ -556,72 +563,110 @@ __global__ void knorm_kernel(const PrefillArgs P) {
     }
 }
 
-// Visits every (row, group, slot) whose block is kept and is not the row's own.
-template <int PHASE>
-__global__ void bucket_kernel(const PrefillArgs P) {
-    const long long total = static_cast<long long>(P.B) * P.Sq * P.H_kv * P.K;
-    for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
-         e += static_cast<long long>(gridDim.x) * blockDim.x) {
-        const long long pair = e / P.K;
-        const long long row = pair / P.H_kv;
-        const int g = static_cast<int>(pair % P.H_kv);
-        const int b = static_cast<int>(row / P.Sq), i = static_cast<int>(row % P.Sq);
-        int L;
-        long long off;
-        if (!seq_ok(P, b, L, off)) continue;
-        const int j = P.ids[e];
+// Buckets of one (sequence, group, row range), built by one CTA: rows that
+// kept block j (j != own) are counted, given offsets in the range's own
+// region of bucket_rows, split into work items of <= kItemRows rows, and
+// scattered.  No grid-wide scan: each range owns fixed slices of the arrays.
+constexpr int kBuildThreads = 512;
+
+__global__ void __launch_bounds__(kBuildThreads) bucket_build_kernel(const PrefillArgs P) {
+    __shared__ int warp_c[kBuildThreads / 32], warp_i[kBuildThreads / 32];
+    __shared__ int carry_c, carry_i;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const long long r = blockIdx.x;
+    const int rng = static_cast<int>(r % P.n_ranges);
+    const int g = static_cast<int>((r / P.n_ranges) % P.H_kv);
+    const int b = static_cast<int>(r / (static_cast<long long>(P.n_ranges) * P.H_kv));
+    int L;
+    long long off;
+    if (!seq_ok(P, b, L, off)) {
+        if (tid == 0) P.range_count[r] = 0;
+        return;
+    }
+    const int i0 = rng * kRange, i1 = min(P.Sq, i0 + kRange);
+    const long long n_e = static_cast<long long>(i1 - i0) * P.K;
+    int *cnt = P.bucket_cnt + r * P.nb_max;
+    int *cur = P.bucket_cur + r * P.nb_max;
+    const int32_t *ids = P.ids;
+    auto entry = [&](long long e, long long &row) -> int {
+        const int i = i0 + static_cast<int>(e / P.K);
+        const int slot = static_cast<int>(e % P.K);
+        row = static_cast<long long>(b) * P.Sq + i;
+        const int j = ids[(row * P.H_kv + g) * P.K + slot];
         const long long p = static_cast<long long>(L) - P.Sq + i;
-        if (j < 0 || j >= p / 128) continue;            // padding, own block, or out of range
-        const long long bucket =
-            ((static_cast<long long>(b) * P.H_kv + g) * P.n_ranges + i / kRange) * P.nb_max + j;
-        if (PHASE == 0) {
-            atomicAdd(P.bucket_cnt + bucket, 1);
-        } else {
-            const int pos = atomicAdd(P.bucket_cur + bucket, 1);
-            P.bucket_rows[P.bucket_off[bucket] + pos] = static_cast<int>(row);
+        return (j >= 0 && j < p / 128) ? j : -1;   // padding, own block, or out of range
+    };
+    for (long long e = tid; e < n_e; e += kBuildThreads) {
+        long long row;
+        const int j = entry(e, row);
+        if (j >= 0) atomicAdd(cnt + j, 1);
+    }
+    if (tid == 0) { carry_c = 0; carry_i = 0; }
+    __syncthreads();
+    // Exclusive scans of row counts and item counts over j, 512 at a time.
+    const long long region = r * static_cast<long long>(P.rows_per_range) * (P.K > 1 ? P.K - 1 : 1);
+    for (int base = 0; base < P.nb_max; base += kBuildThreads) {
+        const int j = base + tid;
+        const int c = j < P.nb_max ? cnt[j] : 0;
+        const int ni = (c + kItemRows - 1) / kItemRows;
+        int ic = c, ii = ni;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int tc = __shfl_up_sync(0xffffffffu, ic, o), ti = __shfl_up_sync(0xffffffffu, ii, o);
+            if (lane >= o) { ic += tc; ii += ti; }
         }
+        if (lane == 31) { warp_c[wid] = ic; warp_i[wid] = ii; }
+        __syncthreads();
+        int pc = carry_c, pi = carry_i;
+        for (int w = 0; w < wid; ++w) { pc += warp_c[w]; pi += warp_i[w]; }
+        const int ex_c = pc + ic - c, ex_i = pi + ii - ni;
+        if (j < P.nb_max) {
+            const long long bk = r * P.nb_max + j;
+            P.bucket_off[bk] = static_cast<int>(region + ex_c);
+            P.item_off[bk] = ex_i;
+            for (int q = 0; q < ni; ++q) P.item_bucket[r * P.items_per_range + ex_i + q] = j;
+        }
+        __syncthreads();
+        if (tid == kBuildThreads - 1) { carry_c = ex_c + c; carry_i = ex_i + ni; }
+        __syncthreads();
+    }
+    if (tid == 0) P.range_count[r] = carry_i;
+    __syncthreads();
+    for (long long e = tid; e < n_e; e += kBuildThreads) {
+        long long row;
+        const int j = entry(e, row);
+        if (j < 0) continue;
+        const int pos = atomicAdd(cur + j, 1);
+        P.bucket_rows[P.bucket_off[r * P.nb_max + j] + pos] = static_cast<int>(row);
     }
 }
 
-// Exclusive scans of the bucket counts (row offsets) and of their item counts.
-__global__ void __launch_bounds__(1024) bucket_scan_kernel(const PrefillArgs P) {
-    __shared__ long long part_rows[1024], part_items[1024];
-    const long long n = P.n_buckets;
+// Exclusive scan of the ranges' item counts -> global item numbering.
+__global__ void __launch_bounds__(1024) range_scan_kernel(const PrefillArgs P) {
+    __shared__ long long part[1024];
     const int tid = threadIdx.x;
+    const long long n = P.n_ranges_total;
     const long long per = (n + 1023) / 1024;
     const long long lo = min(n, tid * per), hi = min(n, lo + per);
-    long long sr = 0, si = 0;
-    for (long long k = lo; k < hi; ++k) {
-        const int c = P.bucket_cnt[k];
-        sr += c;
-        si += (c + kItemRows - 1) / kItemRows;
-    }
-    part_rows[tid] = sr;
-    part_items[tid] = si;
+    long long sum = 0;
+    for (long long k = lo; k < hi; ++k) sum += P.range_count[k];
+    part[tid] = sum;
     __syncthreads();
     if (tid == 0) {
-        long long ar = 0, ai = 0;
+        long long a = 0;
         for (int t = 0; t < 1024; ++t) {
-            const long long r = part_rows[t], q = part_items[t];
-            part_rows[t] = ar;
-            part_items[t] = ai;
-            ar += r;
-            ai += q;
+            const long long v = part[t];
+            part[t] = a;
+            a += v;
         }
-        P.bucket_off[n] = static_cast<int>(ar);
-        P.item_off[n] = ai;
-        *P.item_total = ai;
+        P.range_item_off[n] = a;
+        *P.item_total = a;
     }
     __syncthreads();
-    long long ar = part_rows[tid], ai = part_items[tid];
+    long long a = part[tid];
     for (long long k = lo; k < hi; ++k) {
-        const int c = P.bucket_cnt[k];
-        const int ni = (c + kItemRows - 1) / kItemRows;
-        P.bucket_off[k] = static_cast<int>(ar);
-        P.item_off[k] = ai;
-        for (int q = 0; q < ni; ++q) P.item_bucket[ai + q] = static_cast<int>(k);
-        ar += c;
-        ai += ni;
+        P.range_item_off[k] = a;
+        a += P.range_count[k];
     }
 }
 
@@ -735,18 +780,23 @@ size_t prefill_workspace_layout(int B, int Sq, int H_q, int H_kv, int K, int max
     const long long rows = static_cast<long long>(B) * Sq;
     L->nb_max = (max_kv_len + 127) / 128;
     L->n_ranges = (Sq + kRange - 1) / kRange;
-    L->n_buckets = static_cast<long long>(B) * H_kv * L->n_ranges * L->nb_max;
+    L->n_ranges_total = static_cast<long long>(B) * H_kv * L->n_ranges;
+    L->rows_per_range = Sq < kRange ? Sq : kRange;
+    L->n_buckets = L->n_ranges_total * L->nb_max;
+    const size_t per_range_rows = static_cast<size_t>(L->rows_per_range) * (K > 1 ? K - 1 : 1);
+    L->items_per_range = static_cast<int>(L->nb_max + per_range_rows / kItemRows + 1);
     size_t o = kWsHeaderBytes;
     L->knorm = o;        o += up(static_cast<size_t>(B) * H_kv * 4);
     L->cnt = o;          o += up(static_cast<size_t>(L->n_buckets) * 4);
     L->cur = o;          o += up(static_cast<size_t>(L->n_buckets) * 4);
     L->l_acc = o;        o += up(static_cast<size_t>(rows) * H_q * 4);
     L->zero_end = o;                                  // [knorm, zero_end) is cleared per call
-    L->off = o;          o += up(static_cast<size_t>(L->n_buckets + 1) * 4);
-    L->item_off = o;     o += up(static_cast<size_t>(L->n_buckets + 1) * 8);
-    L->item_bucket = o;
-    o += up((static_cast<size_t>(L->n_buckets) + static_cast<size_t>(rows) * H_kv * K / kItemRows + 1) * 4);
-    L->rows = o;         o += up(static_cast<size_t>(rows) * H_kv * (K > 1 ? K - 1 : 1) * 4);
+    L->off = o;          o += up(static_cast<size_t>(L->n_buckets) * 4);
+    L->item_off = o;     o += up(static_cast<size_t>(L->n_buckets) * 4);
+    L->item_bucket = o;  o += up(static_cast<size_t>(L->n_ranges_total) * L->items_per_range * 4);
+    L->range_count = o;  o += up(static_cast<size_t>(L->n_ranges_total) * 8);
+    L->range_item_off = o; o += up(static_cast<size_t>(L->n_ranges_total + 1) * 8);
+    L->rows = o;         o += up(static_cast<size_t>(L->n_ranges_total) * per_range_rows * 4);
     L->o_acc = o;        o += up(static_cast<size_t>(rows) * H_q * kDim * 4);
     L->m_arr = o;        o += up(static_cast<size_t>(rows) * H_q * 4);
     L->flags = o;        o += up(static_cast<size_t>(rows) * H_q);
@@ -761,8 +811,10 @@ cudaError_t launch_prefill_attention(const PrefillArgs &a0, uint8_t *ws, const P
     a.bucket_cnt = reinterpret_cast<int *>(ws + L.cnt);
     a.bucket_cur = reinterpret_cast<int *>(ws + L.cur);
     a.bucket_off = reinterpret_cast<int *>(ws + L.off);
-    a.item_off = reinterpret_cast<long long *>(ws + L.item_off);
+    a.item_off = reinterpret_cast<int *>(ws + L.item_off);
     a.item_bucket = reinterpret_cast<int *>(ws + L.item_bucket);
+    a.range_count = reinterpret_cast<long long *>(ws + L.range_count);
+    a.range_item_off = reinterpret_cast<long long *>(ws + L.range_item_off);
     a.bucket_rows = reinterpret_cast<int *>(ws + L.rows);
     a.o_acc = reinterpret_cast<float *>(ws + L.o_acc);
     a.l_acc = reinterpret_cast<float *>(ws + L.l_acc);
@@ -773,7 +825,9 @@ cudaError_t launch_prefill_attention(const PrefillArgs &a0, uint8_t *ws, const P
     a.item_next = reinterpret_cast<long long *>(ws + 16);   // [pass A, pass B]
     a.nb_max = L.nb_max;
     a.n_ranges = L.n_ranges;
-    a.n_buckets = L.n_buckets;
+    a.n_ranges_total = L.n_ranges_total;
+    a.rows_per_range = L.rows_per_range;
+    a.items_per_range = L.items_per_range;
 
     CUtensorMap tq, tk, tv;
     if (!encode_q_gather_map(&tq, a.q, a.H_q, static_cast<long long>(a.B) * a.Sq) ||
@@ -789,9 +843,8 @@ cudaError_t launch_prefill_attention(const PrefillArgs &a0, uint8_t *ws, const P
     }
     {
         TraceScope t(s, "prefill_bucket");
-        bucket_kernel<0><<<sms * 8, 256, 0, s>>>(a);
-        bucket_scan_kernel<<<1, 1024, 0, s>>>(a);
-        bucket_kernel<1><<<sms * 8, 256, 0, s>>>(a);
+        bucket_build_kernel<<<static_cast<unsigned>(L.n_ranges_total), kBuildThreads, 0, s>>>(a);
+        range_scan_kernel<<<1, 1024, 0, s>>>(a);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_pass<0>(tq, tk, tv, a, s, "prefill_attn_own_block")) != cudaSuccess) return e;

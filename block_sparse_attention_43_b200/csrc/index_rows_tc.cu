@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (full) {
 #pragma unroll
                                 for (int e = 0; e < 32; ++e)
-                                    m = fmaxf(m, fmaxf(__uint_as_float(va[e]), __uint_as_float(vb[e])));
+                                    m = fmax3(m, __uint_as_float(va[e]), __uint_as_float(vb[e]));
                             } else {
 #pragma unroll
                                 for (int e = 0; e < 32; ++e) {

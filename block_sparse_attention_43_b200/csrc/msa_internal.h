@@ -108,22 +108,23 @@ struct PrefillArgs {
     float softmax_scale;
     // workspace views (filled by launch_prefill_attention)
     float *knorm;
-    int *bucket_cnt, *bucket_cur, *bucket_off, *bucket_rows;
-    long long *item_off;
-    int *item_bucket;       // bucket of every pass-B work item
+    int *bucket_cnt, *bucket_cur, *bucket_off, *bucket_rows;  // per (range, block j)
+    int *item_off;          // first item of each bucket, counted inside its range
+    int *item_bucket;       // [range][item] -> block j
+    long long *range_count, *range_item_off;
     long long *item_total;
     long long *item_next;   // claim counters of pass A and pass B (zeroed per call)
     float *o_acc, *l_acc, *m_arr;
     uint8_t *flags;
     int *flag_count;
-    int nb_max, n_ranges;
-    long long n_buckets;
+    int nb_max, n_ranges, rows_per_range, items_per_range;
+    long long n_ranges_total;
 };
 struct PrefillLayout {
-    size_t knorm, cnt, cur, zero_end, off, item_off, item_bucket, rows, o_acc, l_acc, m_arr, flags,
-        total;
-    int nb_max, n_ranges;
-    long long n_buckets;
+    size_t knorm, cnt, cur, l_acc, zero_end, off, item_off, item_bucket, range_count,
+        range_item_off, rows, o_acc, m_arr, flags, total;
+    int nb_max, n_ranges, rows_per_range, items_per_range;
+    long long n_ranges_total, n_buckets;
 };
 bool prefill_attention_supported(int H_q, int H_kv);
 size_t prefill_workspace_layout(int B, int Sq, int H_q, int H_kv, int K, int max_kv_len,
