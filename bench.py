@@ -253,6 +253,22 @@ def dist_setup(args):
     return None, 0, 0, 1
 
 
+def max_over_ranks(dist, x, device):
+    """The slowest rank's value (every rank calls this, in the same order)."""
+    if dist is None:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(dist, world, units_per_rank, seconds_local, device):
+    """Whole-job throughput: every rank's units over the slowest rank's time.
+    Returns (units per second, slowest seconds)."""
+    slow = max_over_ranks(dist, seconds_local, device)
+    return units_per_rank * world / slow, slow
+
+
 def cores_used():
     try:
         return len(os.sched_getaffinity(0))
@@ -387,12 +403,9 @@ def main():
     for n, t in trace:
         shares[n] = shares.get(n, 0.0) + t
 
-    if dist is not None:
-        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
-    ms_step = ms_total / args.steps
-    value = step_bytes * world / (ms_step / 1e3) / 1e9
+    rate, slow_s = whole_job_rate(dist, world, step_bytes * args.steps, ms_total / 1e3, dev)
+    ms_step = slow_s * 1e3 / args.steps
+    value = rate / 1e9
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -522,12 +535,8 @@ def run_e2e(w, eng, stream, args, step_bytes, world, dist):
     t0 = time.perf_counter()
     for _ in range(n):
         one()
-    dt = (time.perf_counter() - t0) / n
-    if dist is not None:
-        t = torch.tensor([dt], dtype=torch.float64, device=w.q.device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        dt = float(t.item())
-    return {"value": step_bytes * world / dt / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+    rate, dt = whole_job_rate(dist, world, step_bytes, (time.perf_counter() - t0) / n, w.q.device)
+    return {"value": rate / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": dt * 1e3, "steps": n}
 
 
