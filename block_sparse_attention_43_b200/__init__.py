@@ -24,6 +24,7 @@ STATUS_NAMES = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
 # Every entry point include/msa.h declares.
 EXPORTS = ("msa_index_topk_workspace_size", "msa_index_topk",
            "msa_sparse_attention_workspace_size", "msa_sparse_attention",
+           "msa_index_topk_paged", "msa_sparse_attention_paged", "msa_kv_append",
            "msa_index_topk_static", "msa_read_device_status", "msa_trace_enable",
            "msa_trace_read",
            "msa_status_string")
@@ -57,6 +58,13 @@ def _load():
     lib.msa_index_topk.restype = ctypes.c_int
     lib.msa_sparse_attention.argtypes = [S, P, P, P, P, P, P, ctypes.c_float, P, P, Z, P]
     lib.msa_sparse_attention.restype = ctypes.c_int
+    I32 = ctypes.c_int32
+    lib.msa_index_topk_paged.argtypes = [S, P, P, P, P, I32, P, P, P, Z, P]
+    lib.msa_index_topk_paged.restype = ctypes.c_int
+    lib.msa_sparse_attention_paged.argtypes = [S, P, P, P, P, P, P, I32, ctypes.c_float, P, P, Z, P]
+    lib.msa_sparse_attention_paged.restype = ctypes.c_int
+    lib.msa_kv_append.argtypes = [S, I32, P, P, P, P, P, P, I32, P, P, P, P, P]
+    lib.msa_kv_append.restype = ctypes.c_int
     lib.msa_index_topk_static.argtypes = [S, P, P, P, P, P, P, P]
     lib.msa_index_topk_static.restype = ctypes.c_int
     lib.msa_read_device_status.argtypes = [P, P]
@@ -125,6 +133,38 @@ def msa_sparse_attention(shape, q, k_cache, v_cache, block_ids, lens, kv_offsets
                                     float(softmax_scale), _ptr(out), _ptr(workspace),
                                     workspace.numel(), _stream(stream)),
            "msa_sparse_attention")
+
+
+def msa_index_topk_paged(shape, q_idx, k_idx_pool, lens, page_table, block_ids, block_scores,
+                         workspace, stream=None) -> None:
+    """Index branch on paged caches; page_table is int32 [B, pages_per_seq]."""
+    _check(lib.msa_index_topk_paged(ctypes.byref(shape), _ptr(q_idx), _ptr(k_idx_pool), _ptr(lens),
+                                    _ptr(page_table), int(page_table.shape[-1]), _ptr(block_ids),
+                                    _ptr(block_scores), _ptr(workspace), workspace.numel(),
+                                    _stream(stream)),
+           "msa_index_topk_paged")
+
+
+def msa_sparse_attention_paged(shape, q, k_pool, v_pool, block_ids, lens, page_table,
+                               softmax_scale, out, workspace, stream=None) -> None:
+    """Sparse branch on paged caches; page_table is int32 [B, pages_per_seq]."""
+    _check(lib.msa_sparse_attention_paged(ctypes.byref(shape), _ptr(q), _ptr(k_pool), _ptr(v_pool),
+                                          _ptr(block_ids), _ptr(lens), _ptr(page_table),
+                                          int(page_table.shape[-1]), float(softmax_scale),
+                                          _ptr(out), _ptr(workspace), workspace.numel(),
+                                          _stream(stream)),
+           "msa_sparse_attention_paged")
+
+
+def msa_kv_append(shape, new_k_idx, new_k, new_v, lens, k_idx_cache, k_cache, v_cache, *,
+                  kv_offsets=None, page_table=None, device_status=None, stream=None) -> None:
+    """Writes [B, n_new, H_kv, 128] new tokens after each sequence's length."""
+    pps = int(page_table.shape[-1]) if page_table is not None else 0
+    _check(lib.msa_kv_append(ctypes.byref(shape), int(new_k.shape[1]), _ptr(new_k_idx), _ptr(new_k),
+                             _ptr(new_v), _ptr(lens), _ptr(kv_offsets), _ptr(page_table), pps,
+                             _ptr(k_idx_cache), _ptr(k_cache), _ptr(v_cache), _ptr(device_status),
+                             _stream(stream)),
+           "msa_kv_append")
 
 
 def msa_index_topk_static(shape, q_idx, k_idx, lens, kv_offsets, block_ids, block_scores,

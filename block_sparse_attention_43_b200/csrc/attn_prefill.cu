@@ -83,10 +83,9 @@ __device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, 
                  : "memory");
 }
 
-__device__ __forceinline__ bool seq_ok(const PrefillArgs &P, int b, int &L, long long &off) {
+__device__ __forceinline__ bool seq_ok(const PrefillArgs &P, int b, int &L) {
     L = P.lens[b];
-    off = P.kv_offsets[b];
-    return L >= P.Sq && L >= 1 && L <= P.max_kv_len && off >= 0 && off + L <= P.capacity;
+    return L >= P.Sq && L >= 1 && L <= P.max_kv_len && kv_seq_ok(P.kv, b, L);
 }
 
 // A work item: one key block j of one (sequence, group) and the rows that
@@ -96,7 +95,6 @@ struct Item {
     int b, g, j, n;         // n = number of rows
     int i_lo;               // pass A: first query row
     const int *rows;        // pass B: flattened rows (b*Sq + i)
-    long long off;
     int L;
     bool valid;
 };
@@ -113,7 +111,7 @@ __device__ __forceinline__ Item item_at(const PrefillArgs &P, long long it) {
         const int rem = static_cast<int>(it % (static_cast<long long>(P.H_kv) * nj));
         x.g = rem / nj;
         const int jj = rem % nj;
-        if (!seq_ok(P, x.b, x.L, x.off)) { x.n = 0; return x; }
+        if (!seq_ok(P, x.b, x.L)) { x.n = 0; return x; }
         const long long p0 = static_cast<long long>(x.L) - P.Sq;   // position of row 0
         x.j = static_cast<int>(p0 / 128) + jj;
         const long long plo = max(p0, static_cast<long long>(x.j) * 128);
@@ -139,7 +137,7 @@ __device__ __forceinline__ Item item_at(const PrefillArgs &P, long long it) {
         x.b = static_cast<int>(r / (static_cast<long long>(P.n_ranges) * P.H_kv));
         x.n = min(kItemRows, cnt - chunk * kItemRows);
         x.rows = P.bucket_rows + P.bucket_off[bucket] + static_cast<long long>(chunk) * kItemRows;
-        x.valid = x.n > 0 && seq_ok(P, x.b, x.L, x.off);
+        x.valid = x.n > 0 && seq_ok(P, x.b, x.L);
     }
     return x;
 }
@@ -251,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     (*abort_flag || !mbar_wait(&S.kv_empty[kvs], ((ki >> 1) - 1) & 1, P.status))) {
                     ok = false;
                 } else {
-                    const int tok = static_cast<int>(x.off + static_cast<long long>(x.j) * 128);
+                    const int tok = static_cast<int>(kv_block_row(P.kv, x.b, x.j, P.status));
                     mbar_arrive_expect_tx(&S.kv_full[kvs], 65536);
                     tma_load_3d(S.kv[kvs], &tmK, 0, x.g, tok, &S.kv_full[kvs]);
                     tma_load_3d(S.kv[kvs] + 16384, &tmK, 64, x.g, tok, &S.kv_full[kvs]);
@@ -401,12 +399,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             return true;
         };
 
+        int ki = 0;                                    // items seen (K/V ring position)
         for (int n = 0; ok; ++n) {
             const long long it = next_item(n, true);
             if (it < 0) { ok = false; break; }
             if (it >= total) break;
             const Item x = item_at<MODE>(P, it);
             if (!x.valid) continue;
+            const int kvs = ki & 1, kv_par = (ki >> 1) & 1;
+            ++ki;
+            // Pass A only: in a sequence's last, partial block the value rows
+            // past its length may hold anything (padding of a paged pool);
+            // they get weight 0, but 0 * NaN is NaN, so zero them before the
+            // first PV of the item reads them (every softmax warp arrives on
+            // p_full only after its share is written).
+            const int nvalid_kv = MODE == 0 ? min(128, x.L - x.j * 128) : 128;
+            bool zero_v = MODE == 0 && nvalid_kv < 128;
             for (int t0 = 0; t0 < x.n; t0 += kTileRows, ++qt) {
                 const int ss = qt & 1;
                 const bool valid = t0 + ri < x.n;
@@ -468,6 +476,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c8 = 0; c8 < 8; ++c8)
                     *reinterpret_cast<uint4 *>(S.p + ch * 16384 + swz128(m, c8)) =
                         make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
+                if (zero_v) {
+                    bool kok = !*abort_flag && mbar_wait(&S.kv_full[kvs], kv_par, P.status);
+                    kok = __all_sync(0xffffffffu, kok);
+                    if (!kok) { ok = false; break; }
+                    // rows nvalid_kv..127 of V lo and V hi, 16 bytes per thread-step
+                    const int tsw = (warp - 4) * 32 + lane;           // 0..255
+                    for (int e = tsw; e < (128 - nvalid_kv) * 16; e += kSoftWarps * 32) {
+                        const int rrow = nvalid_kv + e / 16, c16 = e % 16;
+                        *reinterpret_cast<uint4 *>(S.kv[kvs] + 32768 + (c16 >> 3) * 16384 +
+                                                   rrow * 128 + (c16 & 7) * 16) = make_uint4(0, 0, 0, 0);
+                    }
+                    zero_v = false;
+                }
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
@@ -537,12 +558,12 @@ __global__ void knorm_kernel(const PrefillArgs P) {
         const int g = static_cast<int>((w / nb) % P.H_kv);
         const int b = static_cast<int>(w / (static_cast<long long>(nb) * P.H_kv));
         int L;
-        long long off;
-        if (!seq_ok(P, b, L, off) || j * 128 >= L) continue;
+        if (!seq_ok(P, b, L) || j * 128 >= L) continue;
         const __nv_bfloat16 *k = static_cast<const __nv_bfloat16 *>(P.k_cache);
+        const long long row0 = kv_block_row(P.kv, b, j, P.status);
         float best = 0.f;
-        for (int t = j * 128 + lane; t < min(L, j * 128 + 128); t += 32) {
-            const uint4 *row = reinterpret_cast<const uint4 *>(k + ((off + t) * P.H_kv + g) * kDim);
+        for (int t = lane; t < min(L - j * 128, 128); t += 32) {
+            const uint4 *row = reinterpret_cast<const uint4 *>(k + ((row0 + t) * P.H_kv + g) * kDim);
             float s = 0.f;
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
@@ -578,8 +599,7 @@ __global__ void __launch_bounds__(kBuildThreads) bucket_build_kernel(const Prefi
     const int g = static_cast<int>((r / P.n_ranges) % P.H_kv);
     const int b = static_cast<int>(r / (static_cast<long long>(P.n_ranges) * P.H_kv));
     int L;
-    long long off;
-    if (!seq_ok(P, b, L, off)) {
+    if (!seq_ok(P, b, L)) {
         if (tid == 0) P.range_count[r] = 0;
         return;
     }
@@ -686,8 +706,7 @@ __global__ void fixup_kernel(const PrefillArgs P) {
         const int g = static_cast<int>(pair % P.H_kv);
         const int b = static_cast<int>(row / P.Sq), i = static_cast<int>(row % P.Sq);
         int L;
-        long long off;
-        if (!seq_ok(P, b, L, off)) continue;
+        if (!seq_ok(P, b, L)) continue;
         const long long p = static_cast<long long>(L) - P.Sq + i;
         for (int h = 0; h < kG; ++h) {
             const long long idx = row * P.H_q + g * kG + h;
@@ -697,8 +716,9 @@ __global__ void fixup_kernel(const PrefillArgs P) {
             for (int s = 0; s < P.K; ++s) {
                 const int j = P.ids[pair * P.K + s];
                 if (j < 0 || j >= p / 128) continue;
-                for (int t = j * 128 + lane; t < j * 128 + 128; t += 32) {
-                    const __nv_bfloat16 *kt = kb + ((off + t) * P.H_kv + g) * kDim;
+                const long long row0 = kv_block_row(P.kv, b, j, P.status);
+                for (int t = lane; t < 128; t += 32) {
+                    const __nv_bfloat16 *kt = kb + ((row0 + t) * P.H_kv + g) * kDim;
                     float d = 0.f;
                     for (int c = 0; c < kDim; ++c) d = fmaf(__bfloat162float(qh[c]), __bfloat162float(kt[c]), d);
                     mx = fmaxf(mx, d * sl2);
@@ -736,9 +756,8 @@ __global__ void finalize_kernel(const PrefillArgs P) {
         const int g = static_cast<int>(pair % P.H_kv);
         const int b = static_cast<int>(row / P.Sq);
         int L;
-        long long off;
         __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(P.out) + (row * P.H_q + g * kG + h) * kDim + qd * 32;
-        if (!seq_ok(P, b, L, off)) {
+        if (!seq_ok(P, b, L)) {
             for (int d = 0; d < 32; ++d) out[d] = __float2bfloat16(NAN);
             continue;
         }
@@ -831,8 +850,8 @@ cudaError_t launch_prefill_attention(const PrefillArgs &a0, uint8_t *ws, const P
 
     CUtensorMap tq, tk, tv;
     if (!encode_q_gather_map(&tq, a.q, a.H_q, static_cast<long long>(a.B) * a.Sq) ||
-        !encode_kv_tensor_map(&tk, a.k_cache, a.H_kv, a.capacity) ||
-        !encode_kv_tensor_map(&tv, a.v_cache, a.H_kv, a.capacity))
+        !encode_kv_tensor_map(&tk, a.k_cache, a.H_kv, a.kv.capacity) ||
+        !encode_kv_tensor_map(&tv, a.v_cache, a.H_kv, a.kv.capacity))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaMemsetAsync(ws + L.knorm, 0, L.zero_end - L.knorm, s);
     if (e != cudaSuccess) return e;

@@ -73,8 +73,7 @@ __global__ void __launch_bounds__(kThreads, kStages == 1 ? 3 : 1)
     const int b = static_cast<int>(row / P.Sq);
     const int i = static_cast<int>(row % P.Sq);
     const int L = P.lens[b];
-    const long long off = P.kv_offsets[b];
-    const bool valid = L >= P.Sq && L >= 1 && L <= P.max_kv_len && off >= 0 && off + L <= P.capacity;
+    const bool valid = L >= P.Sq && L >= 1 && L <= P.max_kv_len && kv_seq_ok(P.kv, b, L);
     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(P.out) + (row * P.H_q + (long long)g * G) * kDim;
 
     if (!valid) {
@@ -107,7 +106,7 @@ __global__ void __launch_bounds__(kThreads, kStages == 1 ? 3 : 1)
             if (n >= lo && n < hi) {
                 S.blocks[nblk] = j;
                 if (nblk < kStages) {
-                    const int tok = static_cast<int>(off + (long long)j * kBlock);
+                    const int tok = static_cast<int>(kv_block_row(P.kv, b, j, P.status));
                     uint8_t *dst = S.ring[nblk];
                     mbar_arrive_expect_tx(&S.full[nblk], kStageBytes);
                     tma_load_3d(dst, &tmK, 0, g, tok, &S.full[nblk]);
@@ -150,7 +149,7 @@ __global__ void __launch_bounds__(kThreads, kStages == 1 ? 3 : 1)
                     ok = false;
                     break;
                 }
-                const int tok = static_cast<int>(off + (long long)S.blocks[it] * kBlock);
+                const int tok = static_cast<int>(kv_block_row(P.kv, b, S.blocks[it], P.status));
                 uint8_t *dst = S.ring[st];
                 mbar_arrive_expect_tx(&S.full[st], kStageBytes);
                 tma_load_3d(dst, &tmK, 0, g, tok, &S.full[st]);
@@ -434,8 +433,8 @@ cudaError_t launch_nt(const AttnRowsArgs &a, cudaStream_t s) {
     static_assert(sizeof(Merge<NT>) <= STAGES * kStageBytes, "merge area fits in the ring");
     static_assert(sizeof(Smem<NT, STAGES>) + 1024 <= 227 * 1024, "shared memory budget");
     CUtensorMap tk, tv;
-    if (!encode_kv_tensor_map(&tk, a.k_cache, a.H_kv, a.capacity) ||
-        !encode_kv_tensor_map(&tv, a.v_cache, a.H_kv, a.capacity))
+    if (!encode_kv_tensor_map(&tk, a.k_cache, a.H_kv, a.kv.capacity) ||
+        !encode_kv_tensor_map(&tv, a.v_cache, a.H_kv, a.kv.capacity))
         return cudaErrorInvalidValue;
     const size_t smem = sizeof(Smem<NT, STAGES>) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attn_rows_kernel<NT, STAGES>,

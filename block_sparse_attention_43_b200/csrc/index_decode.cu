@@ -39,8 +39,8 @@ __device__ __forceinline__ void consumers_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory");
 }
 
-__device__ __forceinline__ bool seq_valid(int L, long long off, int max_kv_len, long long cap) {
-    return L >= 1 && L <= max_kv_len && off >= 0 && off + L <= cap;
+__device__ __forceinline__ bool seq_valid(const IndexDecodeArgs &P, int b, int L) {
+    return L >= 1 && L <= P.max_kv_len && kv_seq_ok(P.kv, b, L);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) index_decode_kernel(const IndexDecodeArgs P) {
@@ -65,8 +65,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_decode_kernel(const IndexDe
         int sum = 0;
         for (int b = lo; b < hi; ++b) {
             const int L = P.lens[b];
-            const long long off = P.kv_offsets[b];
-            if (seq_valid(L, off, P.max_kv_len, P.capacity)) sum += (L + kBlock - 1) / kBlock;
+            if (seq_valid(P, b, L)) sum += (L + kBlock - 1) / kBlock;
             else if (blockIdx.x == 0) set_status(P.status, kStatusBadLens);
         }
         int incl = sum;
@@ -79,8 +78,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_decode_kernel(const IndexDe
         for (int b = lo; b < hi; ++b) {
             S.prefix[b] = run;
             const int L = P.lens[b];
-            if (seq_valid(L, P.kv_offsets[b], P.max_kv_len, P.capacity))
-                run += (L + kBlock - 1) / kBlock;
+            if (seq_valid(P, b, L)) run += (L + kBlock - 1) / kBlock;
         }
         if (lane == 31) S.prefix[P.B] = incl;
     }
@@ -109,7 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_decode_kernel(const IndexDe
                 int b, j;
                 unit_of(u, b, j);
                 const int L = P.lens[b];
-                const long long t_first = P.kv_offsets[b] + (long long)j * kBlock;
+                const long long t_first = kv_block_row(P.kv, b, j, P.status);
                 const int ntok = min(kBlock, L - j * kBlock);
                 for (int t0 = 0; t0 < ntok; t0 += tps, ++it) {
                     const int nt = min(tps, ntok - t0);

@@ -53,7 +53,7 @@ struct Smem {
 
 struct Unit {
     int b, g, i0, nrows, L;
-    long long off, p_first;
+    long long p_first;
     int jmax;        // last visible key block of the tile
     bool valid;
 };
@@ -69,9 +69,7 @@ __device__ __forceinline__ Unit unit_at(const IndexRowsArgs &P, long long u, int
     x.i0 = t * 128;
     x.nrows = min(128, P.Sq - x.i0);
     x.L = P.lens[x.b];
-    x.off = P.kv_offsets[x.b];
-    x.valid = x.L >= P.Sq && x.L >= 1 && x.L <= P.max_kv_len && x.off >= 0 &&
-              x.off + x.L <= P.capacity;
+    x.valid = x.L >= P.Sq && x.L >= 1 && x.L <= P.max_kv_len && kv_seq_ok(P.kv, x.b, x.L);
     x.p_first = static_cast<long long>(x.L) - P.Sq + x.i0;
     x.jmax = x.valid ? static_cast<int>((x.p_first + x.nrows - 1) / kBlock) : -1;
     return x;
@@ -179,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int nb = min(2, x.jmax - j + 1);
                 mbar_arrive_expect_tx(&S.k_full[s], nb * 32768);
                 for (int jj = 0; jj < nb; ++jj) {
-                    const int tok = static_cast<int>(x.off + (long long)(j + jj) * kBlock);
+                    const int tok = static_cast<int>(kv_block_row(P.kv, x.b, j + jj, P.status));
                     tma_load_3d(S.ring[s] + jj * 16384, &tmK, 0, x.g, tok, &S.k_full[s]);
                     tma_load_3d(S.ring[s] + 32768 + jj * 16384, &tmK, 64, x.g, tok, &S.k_full[s]);
                 }
@@ -366,7 +364,7 @@ cudaError_t launch_index_rows_tc(const IndexRowsArgs &a, cudaStream_t s) {
     static_assert(sizeof(Smem<64>) + 1024 <= 227 * 1024, "shared memory budget");
     CUtensorMap tq, tk;
     if (!encode_kv_tensor_map(&tq, a.q_idx, a.H_kv, static_cast<long long>(a.B) * a.Sq) ||
-        !encode_kv_tensor_map(&tk, a.k_idx, a.H_kv, a.capacity))
+        !encode_kv_tensor_map(&tk, a.k_idx, a.H_kv, a.kv.capacity))
         return cudaErrorInvalidValue;
     const long long ntiles = (a.Sq + 127) / 128;
     const long long units = ntiles * a.B * a.H_kv;

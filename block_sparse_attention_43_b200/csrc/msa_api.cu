@@ -169,16 +169,26 @@ size_t msa_sparse_attention_workspace_size(const msa_shape_t *shape) {
     return attn_layout(shape).total;
 }
 
-msa_status_t msa_index_topk(const msa_shape_t *shape, const void *q_idx, const void *k_idx,
-                            const int32_t *lens, const int64_t *kv_offsets, int32_t *block_ids,
-                            float *block_scores, void *workspace, size_t workspace_bytes,
-                            msa_stream_t stream) {
-    msa_status_t st = check_shape(shape);
-    if (st != MSA_OK) return st;
-    if (!q_idx || !k_idx || !lens || !kv_offsets || !block_ids || !block_scores)
-        return MSA_ERR_INVALID_ARG;
+}  // extern "C"
+
+namespace {
+
+// Paged caches: the pool holds whole 128-row pages and every sequence's
+// blocks fit its page-table row.
+msa_status_t check_paged(const msa_shape_t *s, const int32_t *page_table, int32_t pages_per_seq) {
+    if (!page_table || pages_per_seq < 1) return MSA_ERR_INVALID_ARG;
+    if (s->kv_capacity % kBlock) return MSA_ERR_INVALID_ARG;
+    if (static_cast<long long>(pages_per_seq) * kBlock < s->max_kv_len) return MSA_ERR_INVALID_ARG;
+    return MSA_OK;
+}
+
+msa_status_t index_topk_impl(const msa_shape_t *shape, const void *q_idx, const void *k_idx,
+                             const int32_t *lens, const KvMap &kv, int32_t *block_ids,
+                             float *block_scores, void *workspace, size_t workspace_bytes,
+                             msa_stream_t stream) {
+    if (!q_idx || !k_idx || !lens || !block_ids || !block_scores) return MSA_ERR_INVALID_ARG;
     if (!aligned16(q_idx) || !aligned16(k_idx)) return MSA_ERR_MISALIGNED;
-    st = check_ws(workspace, workspace_bytes, index_ws_bytes(shape));
+    msa_status_t st = check_ws(workspace, workspace_bytes, index_ws_bytes(shape));
     if (st != MSA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -187,30 +197,107 @@ msa_status_t msa_index_topk(const msa_shape_t *shape, const void *q_idx, const v
     const int nb_max = nb_max_of(shape);
 
     if (cudaMemsetAsync(ws, 0, kWsHeaderBytes, s) != cudaSuccess) return MSA_ERR_CUDA;
-    cudaError_t e;
-    if (shape->q_len == 1) {
-        IndexDecodeArgs a;
-        a.q_idx = q_idx; a.k_idx = k_idx; a.lens = lens; a.kv_offsets = kv_offsets;
-        a.scores = scores; a.status = status;
-        a.B = shape->batch; a.H_kv = shape->num_kv_heads; a.nb_max = nb_max;
-        a.max_kv_len = shape->max_kv_len; a.capacity = shape->kv_capacity;
-        e = launch_index_decode(a, s);
-    } else {
+    if (shape->q_len > 1) {
         IndexRowsArgs a;
-        a.q_idx = q_idx; a.k_idx = k_idx; a.lens = lens; a.kv_offsets = kv_offsets;
+        a.q_idx = q_idx; a.k_idx = k_idx; a.lens = lens; a.kv = kv;
         a.ids = block_ids; a.out_scores = block_scores; a.status = status;
         a.B = shape->batch; a.Sq = shape->q_len; a.H_kv = shape->num_kv_heads; a.K = shape->top_k;
-        a.max_kv_len = shape->max_kv_len; a.capacity = shape->kv_capacity;
+        a.max_kv_len = shape->max_kv_len;
         return launch_index_rows_tc(a, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
     }
-    if (e != cudaSuccess) return MSA_ERR_CUDA;
+    IndexDecodeArgs a;
+    a.q_idx = q_idx; a.k_idx = k_idx; a.lens = lens; a.kv = kv;
+    a.scores = scores; a.status = status;
+    a.B = shape->batch; a.H_kv = shape->num_kv_heads; a.nb_max = nb_max;
+    a.max_kv_len = shape->max_kv_len;
+    if (launch_index_decode(a, s) != cudaSuccess) return MSA_ERR_CUDA;
     TopkArgs t;
-    t.scores = scores; t.lens = lens; t.kv_offsets = kv_offsets; t.ids = block_ids;
+    t.scores = scores; t.lens = lens; t.kv = kv; t.ids = block_ids;
     t.out_scores = block_scores; t.status = status;
     t.B = shape->batch; t.Sq = shape->q_len; t.H_kv = shape->num_kv_heads; t.nb_max = nb_max;
-    t.K = shape->top_k; t.max_kv_len = shape->max_kv_len; t.capacity = shape->kv_capacity;
+    t.K = shape->top_k; t.max_kv_len = shape->max_kv_len;
     if (launch_topk(t, s) != cudaSuccess) return MSA_ERR_CUDA;
     return MSA_OK;
+}
+
+msa_status_t sparse_attention_impl(const msa_shape_t *shape, const void *q, const void *k_cache,
+                                   const void *v_cache, const int32_t *block_ids,
+                                   const int32_t *lens, const KvMap &kv, float softmax_scale,
+                                   void *out, void *workspace, size_t workspace_bytes,
+                                   msa_stream_t stream) {
+    if (!q || !k_cache || !v_cache || !block_ids || !lens || !out) return MSA_ERR_INVALID_ARG;
+    if (!(softmax_scale == softmax_scale) || softmax_scale == INFINITY || softmax_scale == -INFINITY)
+        return MSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return MSA_ERR_MISALIGNED;
+    const AttnLayout L = attn_layout(shape);
+    msa_status_t st = check_ws(workspace, workspace_bytes, L.total);
+    if (st != MSA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    if (cudaMemsetAsync(ws, 0, kWsHeaderBytes + L.tickets_bytes, s) != cudaSuccess)
+        return MSA_ERR_CUDA;
+    if (use_prefill_path(shape)) {
+        PrefillArgs p;
+        p.q = q; p.k_cache = k_cache; p.v_cache = v_cache; p.ids = block_ids; p.lens = lens;
+        p.kv = kv; p.out = out; p.status = reinterpret_cast<int *>(ws);
+        p.B = shape->batch; p.Sq = shape->q_len; p.H_q = shape->num_q_heads;
+        p.H_kv = shape->num_kv_heads; p.K = shape->top_k; p.max_kv_len = shape->max_kv_len;
+        p.softmax_scale = softmax_scale;
+        return launch_prefill_attention(p, ws, L.pre, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+    }
+    AttnRowsArgs a;
+    a.q = q; a.k_cache = k_cache; a.v_cache = v_cache; a.ids = block_ids; a.lens = lens;
+    a.kv = kv; a.out = out;
+    a.partials = reinterpret_cast<float *>(ws + L.partials_off);
+    a.tickets = reinterpret_cast<int *>(ws + L.tickets_off);
+    a.status = reinterpret_cast<int *>(ws);
+    a.B = shape->batch; a.Sq = shape->q_len; a.H_q = shape->num_q_heads;
+    a.H_kv = shape->num_kv_heads; a.K = shape->top_k; a.nsplit = L.nsplit;
+    a.max_kv_len = shape->max_kv_len;
+    a.softmax_scale = softmax_scale;
+    if (launch_attn_rows(a, s) != cudaSuccess) return MSA_ERR_CUDA;
+    return MSA_OK;
+}
+
+KvMap packed_map(const msa_shape_t *s, const int64_t *kv_offsets) {
+    KvMap m;
+    m.offsets = kv_offsets; m.pages = nullptr; m.pages_per_seq = 0; m.capacity = s->kv_capacity;
+    return m;
+}
+
+KvMap paged_map(const msa_shape_t *s, const int32_t *pages, int32_t pps) {
+    KvMap m;
+    m.offsets = nullptr; m.pages = pages; m.pages_per_seq = pps; m.capacity = s->kv_capacity;
+    return m;
+}
+
+}  // namespace
+
+extern "C" {
+
+msa_status_t msa_index_topk(const msa_shape_t *shape, const void *q_idx, const void *k_idx,
+                            const int32_t *lens, const int64_t *kv_offsets, int32_t *block_ids,
+                            float *block_scores, void *workspace, size_t workspace_bytes,
+                            msa_stream_t stream) {
+    msa_status_t st = check_shape(shape);
+    if (st != MSA_OK) return st;
+    if (!kv_offsets) return MSA_ERR_INVALID_ARG;
+    return index_topk_impl(shape, q_idx, k_idx, lens, packed_map(shape, kv_offsets), block_ids,
+                           block_scores, workspace, workspace_bytes, stream);
+}
+
+msa_status_t msa_index_topk_paged(const msa_shape_t *shape, const void *q_idx,
+                                  const void *k_idx_pool, const int32_t *lens,
+                                  const int32_t *page_table, int32_t pages_per_seq,
+                                  int32_t *block_ids, float *block_scores, void *workspace,
+                                  size_t workspace_bytes, msa_stream_t stream) {
+    msa_status_t st = check_shape(shape);
+    if (st != MSA_OK) return st;
+    if ((st = check_paged(shape, page_table, pages_per_seq)) != MSA_OK) return st;
+    return index_topk_impl(shape, q_idx, k_idx_pool, lens,
+                           paged_map(shape, page_table, pages_per_seq), block_ids, block_scores,
+                           workspace, workspace_bytes, stream);
 }
 
 msa_status_t msa_sparse_attention(const msa_shape_t *shape, const void *q, const void *k_cache,
@@ -220,40 +307,50 @@ msa_status_t msa_sparse_attention(const msa_shape_t *shape, const void *q, const
                                   size_t workspace_bytes, msa_stream_t stream) {
     msa_status_t st = check_shape(shape);
     if (st != MSA_OK) return st;
-    if (!q || !k_cache || !v_cache || !block_ids || !lens || !kv_offsets || !out)
-        return MSA_ERR_INVALID_ARG;
-    if (!(softmax_scale == softmax_scale) || softmax_scale == INFINITY || softmax_scale == -INFINITY)
-        return MSA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
-        return MSA_ERR_MISALIGNED;
-    const AttnLayout L = attn_layout(shape);
-    st = check_ws(workspace, workspace_bytes, L.total);
+    if (!kv_offsets) return MSA_ERR_INVALID_ARG;
+    return sparse_attention_impl(shape, q, k_cache, v_cache, block_ids, lens,
+                                 packed_map(shape, kv_offsets), softmax_scale, out, workspace,
+                                 workspace_bytes, stream);
+}
+
+msa_status_t msa_sparse_attention_paged(const msa_shape_t *shape, const void *q,
+                                        const void *k_pool, const void *v_pool,
+                                        const int32_t *block_ids, const int32_t *lens,
+                                        const int32_t *page_table, int32_t pages_per_seq,
+                                        float softmax_scale, void *out, void *workspace,
+                                        size_t workspace_bytes, msa_stream_t stream) {
+    msa_status_t st = check_shape(shape);
     if (st != MSA_OK) return st;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    if (cudaMemsetAsync(ws, 0, kWsHeaderBytes + L.tickets_bytes, s) != cudaSuccess)
-        return MSA_ERR_CUDA;
-    if (use_prefill_path(shape)) {
-        PrefillArgs p;
-        p.q = q; p.k_cache = k_cache; p.v_cache = v_cache; p.ids = block_ids; p.lens = lens;
-        p.kv_offsets = kv_offsets; p.out = out; p.status = reinterpret_cast<int *>(ws);
-        p.B = shape->batch; p.Sq = shape->q_len; p.H_q = shape->num_q_heads;
-        p.H_kv = shape->num_kv_heads; p.K = shape->top_k; p.max_kv_len = shape->max_kv_len;
-        p.capacity = shape->kv_capacity; p.softmax_scale = softmax_scale;
-        return launch_prefill_attention(p, ws, L.pre, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
-    }
-    AttnRowsArgs a;
-    a.q = q; a.k_cache = k_cache; a.v_cache = v_cache; a.ids = block_ids; a.lens = lens;
-    a.kv_offsets = kv_offsets; a.out = out;
-    a.partials = reinterpret_cast<float *>(ws + L.partials_off);
-    a.tickets = reinterpret_cast<int *>(ws + L.tickets_off);
-    a.status = reinterpret_cast<int *>(ws);
-    a.B = shape->batch; a.Sq = shape->q_len; a.H_q = shape->num_q_heads;
-    a.H_kv = shape->num_kv_heads; a.K = shape->top_k; a.nsplit = L.nsplit;
-    a.max_kv_len = shape->max_kv_len; a.capacity = shape->kv_capacity;
-    a.softmax_scale = softmax_scale;
-    if (launch_attn_rows(a, s) != cudaSuccess) return MSA_ERR_CUDA;
-    return MSA_OK;
+    if ((st = check_paged(shape, page_table, pages_per_seq)) != MSA_OK) return st;
+    return sparse_attention_impl(shape, q, k_pool, v_pool, block_ids, lens,
+                                 paged_map(shape, page_table, pages_per_seq), softmax_scale, out,
+                                 workspace, workspace_bytes, stream);
+}
+
+msa_status_t msa_kv_append(const msa_shape_t *shape, int32_t n_new, const void *new_k_idx,
+                           const void *new_k, const void *new_v, const int32_t *lens,
+                           const int64_t *kv_offsets, const int32_t *page_table,
+                           int32_t pages_per_seq, void *k_idx_cache, void *k_cache,
+                           void *v_cache, int32_t *device_status, msa_stream_t stream) {
+    msa_status_t st = check_shape(shape);
+    if (st != MSA_OK) return st;
+    if (n_new < 1 || !lens || !new_k_idx || !new_k || !new_v || !k_idx_cache || !k_cache ||
+        !v_cache || (!kv_offsets) == (!page_table))
+        return MSA_ERR_INVALID_ARG;
+    if (page_table && (st = check_paged(shape, page_table, pages_per_seq)) != MSA_OK) return st;
+    if (!aligned16(new_k_idx) || !aligned16(new_k) || !aligned16(new_v) ||
+        !aligned16(k_idx_cache) || !aligned16(k_cache) || !aligned16(v_cache))
+        return MSA_ERR_MISALIGNED;
+    KvAppendArgs a;
+    a.src[0] = new_k_idx; a.src[1] = new_k; a.src[2] = new_v;
+    a.dst[0] = k_idx_cache; a.dst[1] = k_cache; a.dst[2] = v_cache;
+    a.lens = lens;
+    a.kv = page_table ? paged_map(shape, page_table, pages_per_seq) : packed_map(shape, kv_offsets);
+    a.status = device_status;
+    a.B = shape->batch; a.n_new = n_new; a.H_kv = shape->num_kv_heads;
+    a.max_kv_len = shape->max_kv_len;
+    return launch_kv_append(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? MSA_OK
+                                                                                     : MSA_ERR_CUDA;
 }
 
 msa_status_t msa_read_device_status(const void *workspace, msa_stream_t stream) {

@@ -8,6 +8,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "msa_internal.h"
+
 namespace msa {
 
 constexpr int kBlock = 128;     // tokens per KV block
@@ -25,6 +27,28 @@ constexpr size_t kWsHeaderBytes = 256;
 
 __device__ __forceinline__ void set_status(int *status, int bit) {
     if (status) atomicOr(status, bit);
+}
+
+// Can sequence b hold L tokens under this layout?
+__device__ __forceinline__ bool kv_seq_ok(const KvMap &m, int b, long long L) {
+    if (m.pages) return L <= static_cast<long long>(m.pages_per_seq) * kBlock;
+    const long long off = m.offsets[b];
+    return off >= 0 && off + L <= m.capacity;
+}
+
+// First cache row of block j of sequence b.  A page number outside the pool
+// records kStatusBadLens and maps to row 0 (always addressable), so no access
+// leaves the caches; that sequence's outputs are then meaningless.
+__device__ __forceinline__ long long kv_block_row(const KvMap &m, int b, int j, int *status) {
+    if (m.pages) {
+        const long long pg = m.pages[static_cast<long long>(b) * m.pages_per_seq + j];
+        if (pg < 0 || (pg + 1) * kBlock > m.capacity) {
+            set_status(status, kStatusBadLens);
+            return 0;
+        }
+        return pg * kBlock;
+    }
+    return m.offsets[b] + static_cast<long long>(j) * kBlock;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

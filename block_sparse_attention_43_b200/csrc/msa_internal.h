@@ -9,6 +9,16 @@
 
 namespace msa {
 
+// Where the tokens of a sequence live in the [capacity, H_kv, 128] caches:
+// packed (sequence b starts at row offsets[b]) or paged (block j of sequence
+// b is the 128-row page pages[b * pages_per_seq + j]).
+struct KvMap {
+    const int64_t *offsets;   // packed layout, or nullptr
+    const int32_t *pages;     // paged layout, or nullptr
+    int pages_per_seq;
+    long long capacity;       // rows in the caches
+};
+
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
 
@@ -31,11 +41,10 @@ struct IndexDecodeArgs {
     const void *q_idx;
     const void *k_idx;
     const int32_t *lens;
-    const int64_t *kv_offsets;
+    KvMap kv;
     float *scores;          // [B][H_kv][nb_max]
     int *status;
     int B, H_kv, nb_max, max_kv_len;
-    long long capacity;
 };
 cudaError_t launch_index_decode(const IndexDecodeArgs &a, cudaStream_t s);
 
@@ -46,12 +55,11 @@ struct IndexRowsArgs {
     const void *q_idx;      // [B][Sq][H_kv][128]
     const void *k_idx;
     const int32_t *lens;
-    const int64_t *kv_offsets;
+    KvMap kv;
     int32_t *ids;
     float *out_scores;
     int *status;
     int B, Sq, H_kv, K, max_kv_len;
-    long long capacity;
 };
 // tcgen05 tensor-core kernel (index_rows_tc.cu).
 cudaError_t launch_index_rows_tc(const IndexRowsArgs &a, cudaStream_t s);
@@ -60,12 +68,11 @@ cudaError_t launch_index_rows_tc(const IndexRowsArgs &a, cudaStream_t s);
 struct TopkArgs {
     const float *scores;    // [B*Sq][H_kv][nb_max]
     const int32_t *lens;
-    const int64_t *kv_offsets;
+    KvMap kv;
     int32_t *ids;           // [B*Sq][H_kv][K]
     float *out_scores;      // [B*Sq][H_kv][K]
     int *status;
     int B, Sq, H_kv, nb_max, K, max_kv_len;
-    long long capacity;
 };
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t s);
 
@@ -76,13 +83,12 @@ struct AttnRowsArgs {
     const void *v_cache;
     const int32_t *ids;     // [B*Sq][H_kv][K]
     const int32_t *lens;
-    const int64_t *kv_offsets;
+    KvMap kv;
     void *out;              // [B][Sq][H_q][128]
-    float *partials;        // [B*Sq][H_kv][nsplit][G*(128+2)]
+    float *partials;        // [B*Sq][H_kv][nsplit][attn_partial_floats(G)]
     int *tickets;           // [B*Sq][H_kv]
     int *status;
     int B, Sq, H_q, H_kv, K, nsplit, max_kv_len;
-    long long capacity;
     float softmax_scale;
 };
 cudaError_t launch_attn_rows(const AttnRowsArgs &a, cudaStream_t s);
@@ -100,11 +106,10 @@ struct PrefillArgs {
     const void *v_cache;
     const int32_t *ids;     // [B*Sq][H_kv][K]
     const int32_t *lens;
-    const int64_t *kv_offsets;
+    KvMap kv;
     void *out;
     int *status;
     int B, Sq, H_q, H_kv, K, max_kv_len;
-    long long capacity;
     float softmax_scale;
     // workspace views (filled by launch_prefill_attention)
     float *knorm;
@@ -133,6 +138,18 @@ cudaError_t launch_prefill_attention(const PrefillArgs &a, uint8_t *ws, const Pr
                                      cudaStream_t s);
 // 3-D map over q [rows, H_q, 128] with an 8-head x 64-dim box (one row).
 bool encode_q_gather_map(CUtensorMap *map, const void *q, int H_q, long long rows);
+
+// Appends n_new tokens per sequence after its current length (kv_append.cu):
+// src[i] [B][n_new][H_kv][128] -> dst[i] at rows of tokens lens[b] .. + n_new - 1.
+struct KvAppendArgs {
+    const void *src[3];
+    void *dst[3];
+    const int32_t *lens;
+    KvMap kv;
+    int *status;
+    int B, n_new, H_kv, max_kv_len;
+};
+cudaError_t launch_kv_append(const KvAppendArgs &a, cudaStream_t s);
 
 // Encodes a [capacity, H_kv, 128] bf16 cache as a 3-D TMA tensor map whose
 // box is (64 dims, 1 group, 128 tokens) with 128-byte swizzling.

@@ -95,9 +95,8 @@ __device__ __forceinline__ void warp_select(Key key_at, int lo, int hi, int m, i
     __syncwarp();
 }
 
-__device__ __forceinline__ bool seq_valid(int L, long long off, int Sq, int max_kv_len,
-                                          long long cap) {
-    return L >= Sq && L >= 1 && L <= max_kv_len && off >= 0 && off + L <= cap;
+__device__ __forceinline__ bool seq_valid(const TopkArgs &P, int b, int L) {
+    return L >= P.Sq && L >= 1 && L <= P.max_kv_len && kv_seq_ok(P.kv, b, L);
 }
 
 // Writes the ascending selection: ids sel[0..n) (unsorted), padded to K.
@@ -125,9 +124,8 @@ __device__ __forceinline__ RowInfo row_info(const TopkArgs &P, long long row) {
     const int b = static_cast<int>(row / P.Sq);
     const int i = static_cast<int>(row % P.Sq);
     const int L = P.lens[b];
-    const long long off = P.kv_offsets[b];
     RowInfo r;
-    r.valid = seq_valid(L, off, P.Sq, P.max_kv_len, P.capacity);
+    r.valid = seq_valid(P, b, L);
     r.own = r.valid ? (L - P.Sq + i) / kBlock : 0;
     return r;
 }

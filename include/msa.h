@@ -133,6 +133,44 @@ MSA_API msa_status_t msa_sparse_attention(const msa_shape_t *shape, const void *
                                   float softmax_scale, void *out,
                                   void *workspace, size_t workspace_bytes, msa_stream_t stream);
 
+/* Paged caches (a block-table layout for serving): the index keys, keys and
+ * values of all sequences live in pools of 128-token pages, [kv_capacity,
+ * H_kv, dim] with page p = rows p*128 .. p*128+127, and block j of sequence b
+ * (tokens 128j .. 128j+127) is page page_table[b * pages_per_seq + j].  The
+ * MSA block and the page are the same 128 tokens, so a kept block is one
+ * page.  Requirements: kv_capacity a multiple of 128, pages_per_seq * 128 >=
+ * max_kv_len, page_table device int32 [B, pages_per_seq].  A page number
+ * outside the pool sets MSA_ERR_BAD_LENS in the device status word; the
+ * outputs of that sequence are then unspecified, and nothing outside the
+ * pools is read.  Everything else is as for the packed calls above; the
+ * results are the same as on a packed copy of the same tokens. */
+MSA_API msa_status_t msa_index_topk_paged(const msa_shape_t *shape, const void *q_idx,
+                                          const void *k_idx_pool, const int32_t *lens,
+                                          const int32_t *page_table, int32_t pages_per_seq,
+                                          int32_t *block_ids, float *block_scores,
+                                          void *workspace, size_t workspace_bytes,
+                                          msa_stream_t stream);
+MSA_API msa_status_t msa_sparse_attention_paged(const msa_shape_t *shape, const void *q,
+                                                const void *k_pool, const void *v_pool,
+                                                const int32_t *block_ids, const int32_t *lens,
+                                                const int32_t *page_table, int32_t pages_per_seq,
+                                                float softmax_scale, void *out, void *workspace,
+                                                size_t workspace_bytes, msa_stream_t stream);
+
+/* Appends n_new tokens to every sequence: new_k_idx, new_k, new_v are device
+ * bf16 [B, n_new, H_kv, 128]; token i of sequence b is written at position
+ * lens[b] + i of the packed (kv_offsets) or paged (page_table, pages_per_seq)
+ * caches -- pass exactly one of kv_offsets / page_table.  lens is not
+ * changed; the caller advances it.  A token that would land at or past
+ * max_kv_len or outside the layout is not written and ORs MSA_ERR_BAD_LENS's
+ * bit (1) into *device_status when device_status is not null.  This is the
+ * step before a decode call (the new token attends to itself). */
+MSA_API msa_status_t msa_kv_append(const msa_shape_t *shape, int32_t n_new, const void *new_k_idx,
+                                   const void *new_k, const void *new_v, const int32_t *lens,
+                                   const int64_t *kv_offsets, const int32_t *page_table,
+                                   int32_t pages_per_seq, void *k_idx_cache, void *k_cache,
+                                   void *v_cache, int32_t *device_status, msa_stream_t stream);
+
 /* msa_index_topk without a workspace argument, for callers that cannot
  * allocate device memory or hand over a workspace (plugin hosts that pass a
  * kernel only its inputs and outputs, processes whose device memory belongs

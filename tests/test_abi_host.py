@@ -85,3 +85,26 @@ def test_status_strings(m):
     for code in range(8):
         assert m.msa_status_string(code).startswith(m.STATUS_NAMES[code])
     assert m.msa_status_string(99) == "MSA_ERR_UNKNOWN"
+
+
+def test_paged_and_append_arguments_are_checked(m):
+    P = ctypes.c_void_p
+    s = _shape(m, kv_capacity=4 << 20)
+    args = [P(0x10000), P(0x20000), P(0x30000)]
+    tail = [P(0x60000), P(0x70000), P(0x100000), 1 << 40, None]
+    # pages_per_seq * 128 < max_kv_len
+    assert m.lib.msa_index_topk_paged(ctypes.byref(s), *args, P(0x40000), 8, *tail) == 1
+    # pool not a whole number of pages
+    bad = _shape(m, kv_capacity=(4 << 20) + 5)
+    assert m.lib.msa_index_topk_paged(ctypes.byref(bad), *args, P(0x40000), 8192, *tail) == 1
+    # null page table
+    assert m.lib.msa_index_topk_paged(ctypes.byref(s), *args, None, 8192, *tail) == 1
+    # kv_append needs exactly one of kv_offsets / page_table
+    ptrs = [P(0x10000)] * 4
+    caches = [P(0x20000)] * 3
+    assert m.lib.msa_kv_append(ctypes.byref(s), 1, *ptrs[:3], P(0x30000), None, None, 0, *caches,
+                               None, None) == 1
+    assert m.lib.msa_kv_append(ctypes.byref(s), 1, *ptrs[:3], P(0x30000), P(0x40000),
+                               P(0x50000), 8192, *caches, None, None) == 1
+    assert m.lib.msa_kv_append(ctypes.byref(s), 0, *ptrs[:3], P(0x30000), P(0x40000), None, 0,
+                               *caches, None, None) == 1
