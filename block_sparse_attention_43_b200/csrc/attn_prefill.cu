@@ -24,49 +24,121 @@
 //   pass A     own block of every row (causal), query-outer: writes the
 //              partial output, sum and shift
 //   fixup      flagged (row, head) only: exact shift, rescale pass A's partials
-//   pass B     the other kept blocks, block-outer: partials reduced into the
-//              accumulator with red.global.add.v4.f32
+//   pass B     the other kept blocks, block-outer: partials added into the
+//              accumulator with bulk fp32 reductions (cp.reduce.async.bulk)
 //   finalize   out = accumulator / sum, bf16
 //
 // Passes A and B share one kernel: per 16-row tile, 16 rows x 8 heads = 128
 // TMEM lanes; the tile's Q rows are gathered by TMA (one 8-head x 64-dim box
 // per row and half), S = Q K^T and O = P V run as tcgen05.mma kind::f16
-// (M=128, N=128, K=128; P is written to shared memory in the K-major
-// 128-byte-swizzled layout, V is read MN-major).  Roles: warp 0 TMA, warp 1
-// MMA issue, warp 2 TMEM owner, warps 4-7 softmax and epilogue.  The
-// accumulator interleaves the 8 heads of a row at 16-byte granularity so
-// that every warp-wide reduction covers whole 128-byte lines.
+// (M=128, N=128, K=128).  S and O live in TMEM; the softmax writes P back to
+// TMEM as bf16 pairs and the PV product reads it from there (V from shared
+// memory, MN-major).  Roles: warp 0 TMA, warp 1 MMA issue, warp 2 TMEM owner,
+// warps 4-11 softmax, warps 12-15 epilogue.  The epilogue stages each partial
+// output in shared memory and hands it to the bulk-copy engine as one fp32
+// add-reduction per row: the reductions, which bound pass B, then never sit
+// in the SM's load/store queue in front of the softmax's memory operations.
+// The accumulator interleaves the 8 heads of a row at 16-byte granularity,
+// so a row's partial output is one contiguous 4 KiB run.
 #include "msa_device.cuh"
 #include "msa_internal.h"
 
 namespace msa {
 namespace {
 
-constexpr int kThreads = 384;           // 4 control warps + 8 softmax/epilogue warps
+constexpr int kThreads = 512;           // 4 control, 8 softmax and 4 epilogue warps
 constexpr int kSoftWarps = 8;
+constexpr int kEpiWarps = 4;
+constexpr int kEpiWarp0 = 4 + kSoftWarps;    // first epilogue warp
 constexpr int kG = 8;                      // heads per group handled by this path
 constexpr int kTileRows = 128 / kG;        // query rows per 128-lane tile
 constexpr int kRange = 8192;               // query rows per bucket range
 constexpr int kItemRows = 256;             // max rows per pass-B work item
-constexpr uint32_t kTmemCols = 512;        // S[2] + O[2], 128 columns each
+constexpr uint32_t kTmemCols = 512;        // S, P and O[2]
+// TMEM columns: S (128 fp32), P (64 columns of bf16 pairs), O[2] (2 x 128 fp32).
+constexpr uint32_t kColS = 0, kColP = 128, kColO = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kSafeLog2 = 64.f;          // max (bound - shift) accepted, base 2
+
+__device__ __forceinline__ bool seq_ok(const PrefillArgs &P, int b, int &L) {
+    L = P.lens[b];
+    return L >= P.Sq && L >= 1 && L <= P.max_kv_len && kv_seq_ok(P.kv, b, L);
+}
+
+// A work item: one key block j of one (sequence, group) and the rows that
+// use it.  Pass A: the rows whose own block is j (consecutive query rows
+// from i_lo).  Pass B: a slice of the bucket of rows that kept j as a
+// non-own block, entries rows_off .. rows_off + n - 1 of bucket_rows (and
+// of bucket_shift).
+struct Item {
+    int b, g, j, n;         // n = number of rows; n <= 0: nothing to do
+    int i_lo;               // pass A: first query row
+    int rows_off;           // pass B: first bucket entry
+    int L;
+    int pad;
+};
+
+template <int MODE>
+__device__ __forceinline__ Item item_at(const PrefillArgs &P, long long it) {
+    Item x;
+    x.i_lo = 0;
+    x.rows_off = 0;
+    x.pad = 0;
+    if (MODE == 0) {
+        const int nj = (P.Sq + 127) / 128 + 1;
+        x.b = static_cast<int>(it / (static_cast<long long>(P.H_kv) * nj));
+        const int rem = static_cast<int>(it % (static_cast<long long>(P.H_kv) * nj));
+        x.g = rem / nj;
+        const int jj = rem % nj;
+        x.j = 0;
+        if (!seq_ok(P, x.b, x.L)) { x.n = 0; return x; }
+        const long long p0 = static_cast<long long>(x.L) - P.Sq;   // position of row 0
+        x.j = static_cast<int>(p0 / 128) + jj;
+        const long long plo = max(p0, static_cast<long long>(x.j) * 128);
+        const long long phi = min(static_cast<long long>(x.L), static_cast<long long>(x.j) * 128 + 128);
+        x.n = phi > plo ? static_cast<int>(phi - plo) : 0;
+        x.i_lo = static_cast<int>(plo - p0);
+    } else {
+        // one 32-byte descriptor, written by item_table_kernel
+        const int4 *d = reinterpret_cast<const int4 *>(P.item_desc) + 2 * it;
+        const int4 a = d[0], c = d[1];
+        x.b = a.x; x.g = a.y; x.j = a.z; x.n = a.w;
+        x.rows_off = c.x; x.L = c.y;
+    }
+    return x;
+}
+
+// Flattened row (b*Sq + i) of row r of the item.
+template <int MODE>
+__device__ __forceinline__ long long tile_row(const PrefillArgs &P, const Item &x, int r) {
+    return MODE == 1 ? static_cast<long long>(P.bucket_rows[x.rows_off + r])
+                     : static_cast<long long>(x.b) * P.Sq + x.i_lo + r;
+}
+
+template <int MODE>
+__device__ __forceinline__ long long n_items(const PrefillArgs &P) {
+    if (MODE == 0) return static_cast<long long>(P.B) * P.H_kv * ((P.Sq + 127) / 128 + 1);
+    return *P.item_total;
+}
 
 struct Smem {
     uint8_t kv[2][65536];                  // K lo, K hi, V lo, V hi (16 KiB each)
     uint8_t q[2][32768];                   // gathered Q tile, two swizzled halves
-    uint8_t p[32768];                      // P tile (bf16), two swizzled halves
+    uint8_t ostage[kEpiWarps][8192];       // epilogue: 4 rows x 64 dims x 8 heads fp32 per warp
     uint64_t kv_full[2], kv_empty[2], q_full[2], q_empty[2];
-    uint64_t s_full[2], s_empty[2], o_full[2], o_empty[2];
+    uint64_t s_full, s_empty, o_full[2], o_empty[2];
     uint64_t p_full, p_empty;
-    uint64_t item_full[4], item_empty[4];  // work-item queue: producer -> MMA + softmax
-    long long item_q[4];
+    uint64_t item_full[4], item_empty[4];  // work-item queue: producer -> MMA, softmax, epilogue
+    Item item_q[4];                        // decoded items (n = -1: no more work)
     uint32_t tmem_base;
     int abort_flag;
 };
 
+// 227 KiB is the per-block shared-memory limit; 1 KiB more aligns the base.
+static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory over the per-block limit");
+
 constexpr int kQueue = 4;
-constexpr int kQueueReaders = 1 + kSoftWarps;   // MMA thread + one arrival per softmax warp
+constexpr int kQueueReaders = 1 + kSoftWarps + kEpiWarps;   // MMA thread + one per consumer warp
 
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
     uint64_t d = static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
@@ -77,81 +149,13 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint
     return d;
 }
 
-__device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
-                 "f"(d)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool seq_ok(const PrefillArgs &P, int b, int &L) {
-    L = P.lens[b];
-    return L >= P.Sq && L >= 1 && L <= P.max_kv_len && kv_seq_ok(P.kv, b, L);
-}
-
-// A work item: one key block j of one (sequence, group) and the rows that
-// use it.  Pass A: the rows whose own block is j (consecutive query rows).
-// Pass B: a slice of the bucket of rows that kept j as a non-own block.
-struct Item {
-    int b, g, j, n;         // n = number of rows
-    int i_lo;               // pass A: first query row
-    const int *rows;        // pass B: flattened rows (b*Sq + i)
-    int L;
-    bool valid;
-};
-
-template <int MODE>
-__device__ __forceinline__ Item item_at(const PrefillArgs &P, long long it) {
-    Item x;
-    x.valid = false;
-    x.rows = nullptr;
-    x.i_lo = 0;
-    if (MODE == 0) {
-        const int nj = (P.Sq + 127) / 128 + 1;
-        x.b = static_cast<int>(it / (static_cast<long long>(P.H_kv) * nj));
-        const int rem = static_cast<int>(it % (static_cast<long long>(P.H_kv) * nj));
-        x.g = rem / nj;
-        const int jj = rem % nj;
-        if (!seq_ok(P, x.b, x.L)) { x.n = 0; return x; }
-        const long long p0 = static_cast<long long>(x.L) - P.Sq;   // position of row 0
-        x.j = static_cast<int>(p0 / 128) + jj;
-        const long long plo = max(p0, static_cast<long long>(x.j) * 128);
-        const long long phi = min(static_cast<long long>(x.L), static_cast<long long>(x.j) * 128 + 128);
-        x.n = phi > plo ? static_cast<int>(phi - plo) : 0;
-        x.i_lo = static_cast<int>(plo - p0);
-        x.valid = x.n > 0;
-    } else {
-        // range of the item (binary search over the ranges' item offsets), then
-        // its bucket (block j) and chunk inside the range
-        long long lo = 0, hi = P.n_ranges_total;
-        while (hi - lo > 1) {
-            const long long mid = (lo + hi) >> 1;
-            if (P.range_item_off[mid] <= it) lo = mid; else hi = mid;
-        }
-        const long long r = lo;
-        const int local = static_cast<int>(it - P.range_item_off[r]);
-        x.j = P.item_bucket[r * P.items_per_range + local];
-        const long long bucket = r * P.nb_max + x.j;
-        const int chunk = local - P.item_off[bucket];
-        const int cnt = P.bucket_cnt[bucket];
-        x.g = static_cast<int>((r / P.n_ranges) % P.H_kv);
-        x.b = static_cast<int>(r / (static_cast<long long>(P.n_ranges) * P.H_kv));
-        x.n = min(kItemRows, cnt - chunk * kItemRows);
-        x.rows = P.bucket_rows + P.bucket_off[bucket] + static_cast<long long>(chunk) * kItemRows;
-        x.valid = x.n > 0 && seq_ok(P, x.b, x.L);
-    }
-    return x;
-}
-
-template <int MODE>
-__device__ __forceinline__ long long n_items(const PrefillArgs &P) {
-    if (MODE == 0) return static_cast<long long>(P.B) * P.H_kv * ((P.Sq + 127) / 128 + 1);
-    return *P.item_total;
-}
-
-// Flattened row (b*Sq + i) of row r of tile t of the item.
-__device__ __forceinline__ long long tile_row(const PrefillArgs &P, const Item &x, int r) {
-    return x.rows ? static_cast<long long>(x.rows[r])
-                  : static_cast<long long>(x.b) * P.Sq + x.i_lo + r;
+// 2^x on the special-function unit (relative error ~2^-22, results below
+// 2^-126 flushed to 0).  Probabilities are rounded to bf16 right after, and
+// the shift keeps every kept term above 2^-64 of the row's largest one.
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 template <int MODE>
@@ -173,11 +177,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Pass A reads each Q tile once more (its norms) after the MMA: the
             // softmax warps release it; in pass B the MMA commit does.
             mbar_init(&S.q_empty[i], MODE == 0 ? kSoftWarps : 1);
-            mbar_init(&S.s_full[i], 1);
-            mbar_init(&S.s_empty[i], kSoftWarps);
             mbar_init(&S.o_full[i], 1);
-            mbar_init(&S.o_empty[i], kSoftWarps);
+            mbar_init(&S.o_empty[i], kEpiWarps);
         }
+        mbar_init(&S.s_full, 1);
+        mbar_init(&S.s_empty, kSoftWarps);
         mbar_init(&S.p_full, kSoftWarps);
         mbar_init(&S.p_empty, 1);
         for (int i = 0; i < kQueue; ++i) {
@@ -199,19 +203,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // Work items are claimed in order from one global counter, so every CTA
     // works on neighbouring items (the same row range): the accumulator and Q
-    // rows of that range stay in L2.  Warp 0 claims and publishes each item;
-    // the MMA thread and the softmax warps read it from the queue.
+    // rows of that range stay in L2.  Warp 0 claims, decodes and publishes
+    // each item; the MMA thread, softmax and epilogue warps read it from the
+    // queue.
     long long *counter = MODE == 0 ? P.item_next : P.item_next + 1;
-    // n-th item for a reader; returns -1 on abort, total when the work is done.
-    auto next_item = [&](int n, bool warp_reader) -> long long {
+    // n-th item for a reader, decoded by the producer; false on abort.
+    // x.n < 0 marks the end of the work.
+    auto next_item = [&](int n, bool warp_reader, Item &x) -> bool {
         const int slot = n % kQueue;
         bool ok = !*abort_flag && mbar_wait(&S.item_full[slot], (n / kQueue) & 1, P.status);
         if (warp_reader) ok = __all_sync(0xffffffffu, ok);
-        if (!ok) return -1;
-        const long long it = S.item_q[slot];
+        if (!ok) return false;
+        x = S.item_q[slot];
         if (warp_reader) __syncwarp();
         if (!warp_reader || lane == 0) mbar_arrive(&S.item_empty[slot]);
-        return it;
+        return true;
     };
 
     if (warp == 0) {
@@ -232,17 +238,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                               ((n / kQueue) - 1) & 1, P.status))) {
                     it = -1;
                 } else {
+                    // Decode once here; the other roles read the result.
                     it = atomicAdd(reinterpret_cast<unsigned long long *>(counter), 1ull);
-                    if (it > total) it = total;
-                    S.item_q[slot] = it;
+                    Item d;
+                    if (it >= total) {
+                        it = total;
+                        d.n = -1;
+                    } else {
+                        d = item_at<MODE>(P, it);
+                    }
+                    S.item_q[slot] = d;
                     mbar_arrive(&S.item_full[slot]);
                 }
             }
             it = __shfl_sync(0xffffffffu, it, 0);
             if (it < 0) { ok = false; break; }
             if (it >= total) break;
-            const Item x = item_at<MODE>(P, it);
-            if (!x.valid) continue;
+            __syncwarp();
+            const Item x = S.item_q[n % kQueue];
+            if (x.n <= 0) continue;
             const int kvs = ki & 1;
             if (lane == 0) {
                 if (ki >= 2 &&
@@ -264,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int qs = qt & 1;
                 const int nr = min(kTileRows, x.n - t0);
                 // Row index of this lane's gather, loaded before the wait.
-                const int row = lane < nr ? static_cast<int>(tile_row(P, x, t0 + lane)) : 0;
+                const int row = lane < nr ? static_cast<int>(tile_row<MODE>(P, x, t0 + lane)) : 0;
                 if (lane == 0) {
                     if (qt >= 2 &&
                         (*abort_flag || !mbar_wait(&S.q_empty[qs], ((qt >> 1) - 1) & 1, P.status)))
@@ -288,19 +302,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         int ki = 0, qt = 0;
         int pv_pending = -1, pv_kvs = 0, pv_last = 0;   // tile waiting for its PV
         bool ok = true;
+        // O = P V: P (bf16) from TMEM, V from shared memory.
         auto issue_pv = [&](int t, int kvs, int last_of_item) -> bool {
             const int os = t & 1;
             if (*abort_flag || !mbar_wait(&S.p_full, t & 1, P.status)) return false;
             if (t >= 2 && (*abort_flag || !mbar_wait(&S.o_empty[os], ((t >> 1) - 1) & 1, P.status)))
                 return false;
             tc_fence_after();
-            const uint32_t pa = smem_u32(S.p);
             const uint32_t va = smem_u32(S.kv[kvs] + 32768);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t ad = umma_desc(pa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
                 const uint64_t bd = umma_desc(va + kk * 2048, 16384, 1024);
-                umma_bf16_ss(tmem + 256 + os * 128, ad, bd, idesc_pv, kk > 0 ? 1u : 0u);
+                umma_bf16_ts(tmem + kColO + os * 128, tmem + kColP + kk * 8, bd, idesc_pv,
+                             kk > 0 ? 1u : 0u);
             }
             umma_commit(&S.o_full[os]);
             umma_commit(&S.p_empty);
@@ -308,19 +322,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             return true;
         };
         for (int n = 0; ok; ++n) {
-            const long long it = next_item(n, false);
-            if (it < 0) { ok = false; break; }
-            if (it >= total) break;
-            const Item x = item_at<MODE>(P, it);
-            if (!x.valid) continue;
+            Item x;
+            if (!next_item(n, false, x)) { ok = false; break; }
+            if (x.n < 0) break;
+            if (x.n == 0) continue;
             const int kvs = ki & 1;
             if (*abort_flag || !mbar_wait(&S.kv_full[kvs], (ki >> 1) & 1, P.status)) { ok = false; break; }
             ++ki;
             const uint32_t ka = smem_u32(S.kv[kvs]);
             for (int t0 = 0; t0 < x.n; t0 += kTileRows, ++qt) {
-                const int qs = qt & 1, ss = qt & 1;
+                const int qs = qt & 1;
                 if (*abort_flag || !mbar_wait(&S.q_full[qs], (qt >> 1) & 1, P.status)) { ok = false; break; }
-                if (qt >= 2 && (*abort_flag || !mbar_wait(&S.s_empty[ss], ((qt >> 1) - 1) & 1, P.status))) {
+                // One S buffer: the previous tile's S must have been read.
+                if (qt >= 1 && (*abort_flag || !mbar_wait(&S.s_empty, (qt - 1) & 1, P.status))) {
                     ok = false;
                     break;
                 }
@@ -330,9 +344,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint64_t ad = umma_desc(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
                     const uint64_t bd = umma_desc(ka + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                    umma_bf16_ss(tmem + ss * 128, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                    umma_bf16_ss(tmem + kColS, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&S.s_full[ss]);
+                umma_commit(&S.s_full);
                 if (MODE == 1) umma_commit(&S.q_empty[qs]);
                 // PV of the previous tile runs behind this tile's QK.
                 if (pv_pending >= 0 && !issue_pv(pv_pending, pv_kvs, pv_last)) { ok = false; break; }
@@ -344,14 +358,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && pv_pending >= 0 && !issue_pv(pv_pending, pv_kvs, pv_last)) ok = false;
         if (!ok) *abort_flag = 1;
         // Every MMA issued must finish before TMEM is released.
-        if (qt > 0) mbar_wait(&S.s_full[(qt - 1) & 1], ((qt - 1) >> 1) & 1, nullptr);
+        if (qt > 0) mbar_wait(&S.s_full, (qt - 1) & 1, nullptr);
         if (pv_pending >= 0) mbar_wait(&S.o_full[pv_pending & 1], (pv_pending >> 1) & 1, nullptr);
-    } else if (warp >= 4) {
-        // ------------------------------------------------ softmax + epilogue
+    } else if (warp >= 4 && warp < kEpiWarp0) {
+        // ------------------------------------------------ softmax
         // Warps 4-7 and 8-11 share the TMEM lanes of warp % 4 and split each
-        // row's 128 columns: ch = 0 takes tokens (and output dims) 0-63,
-        // ch = 1 takes 64-127.  Each half-row sum goes to the accumulator on
-        // its own, so the two warps never wait for each other.
+        // row's 128 columns: ch = 0 takes tokens 0-63, ch = 1 takes 64-127.
+        // Each half-row sum goes to the row's running sum on its own, so the
+        // two warps never wait for each other.  P goes back to TMEM as bf16
+        // pairs (columns kColP + 32 ch ...), where the PV product reads it.
         const int ch = (warp - 4) >> 2;
         const int m = (warp & 3) * 32 + lane;          // TMEM lane = tile row x head
         const int ri = m / kG, h = m % kG;             // tile row, head in group
@@ -359,53 +374,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float sl2 = P.softmax_scale * kLog2e;
         int qt = 0;
         bool ok = true;
-        // state of the tile whose output is still in TMEM
-        int prev = -1;
-        long long prev_row = 0;
-        int prev_g = 0;
-        bool prev_valid = false;
-        float prev_l = 0.f;
-
-        auto epilogue = [&](int t, long long row, int g, bool valid, float l) -> bool {
-            const int os = t & 1;
-            bool have = !*abort_flag && mbar_wait(&S.o_full[os], (t >> 1) & 1, P.status);
-            have = __all_sync(0xffffffffu, have);
-            if (!have) return false;
-            tc_fence_after();
-            uint32_t a[32], b[32];
-            tmem_ld32r(lane_addr + 256 + os * 128 + ch * 64, a);
-            tmem_ld32r(lane_addr + 256 + os * 128 + ch * 64 + 32, b);
-            tmem_wait_ld(a);
-            tmem_tie(b);
-            if (valid) {
-                float *acc = P.o_acc + (row * P.H_kv + g) * (kDim * kG) + h * 4 + ch * 16 * (4 * kG);
-#pragma unroll
-                for (int q4 = 0; q4 < 16; ++q4) {
-                    const uint32_t *r = q4 < 8 ? a + 4 * q4 : b + 4 * (q4 - 8);
-                    float *dst = acc + q4 * (4 * kG);
-                    if (MODE == 0)
-                        *reinterpret_cast<float4 *>(dst) =
-                            make_float4(__uint_as_float(r[0]), __uint_as_float(r[1]),
-                                        __uint_as_float(r[2]), __uint_as_float(r[3]));
-                    else
-                        red_add_v4(dst, __uint_as_float(r[0]), __uint_as_float(r[1]),
-                                   __uint_as_float(r[2]), __uint_as_float(r[3]));
-                }
-                atomicAdd(P.l_acc + row * P.H_q + g * kG + h, l);
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.o_empty[os]);
+        int ki = 0;                                    // items seen (K/V ring position)
+        // Each tile's row and (pass B) shift are loaded one tile ahead, so their
+        // latency hides behind the previous tile's work; at an item's last tile
+        // the next item is read from the queue early for that.
+        int n = 0;
+        auto fetch = [&](Item &it) -> bool {       // next non-empty item or the end
+            do {
+                if (!next_item(n++, true, it)) return false;
+            } while (it.n == 0);
             return true;
         };
-
-        int ki = 0;                                    // items seen (K/V ring position)
-        for (int n = 0; ok; ++n) {
-            const long long it = next_item(n, true);
-            if (it < 0) { ok = false; break; }
-            if (it >= total) break;
-            const Item x = item_at<MODE>(P, it);
-            if (!x.valid) continue;
+        auto load_tile = [&](const Item &it, int t0, long long &row, float &shift) {
+            row = 0;
+            shift = 0.f;
+            if (t0 + ri < it.n) {
+                row = tile_row<MODE>(P, it, t0 + ri);
+                if (MODE == 1)
+                    shift = P.bucket_shift[static_cast<long long>(it.rows_off + t0 + ri) * kG + h];
+            }
+        };
+        Item x;
+        long long row_nx = 0;
+        float shift_nx = 0.f;
+        if (!fetch(x)) ok = false;
+        else if (x.n > 0) load_tile(x, 0, row_nx, shift_nx);
+        while (ok && x.n > 0) {
+            Item xn;
+            xn.n = -1;
             const int kvs = ki & 1, kv_par = (ki >> 1) & 1;
             ++ki;
             // Pass A only: in a sequence's last, partial block the value rows
@@ -416,17 +412,44 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nvalid_kv = MODE == 0 ? min(128, x.L - x.j * 128) : 128;
             bool zero_v = MODE == 0 && nvalid_kv < 128;
             for (int t0 = 0; t0 < x.n; t0 += kTileRows, ++qt) {
-                const int ss = qt & 1;
                 const bool valid = t0 + ri < x.n;
-                const long long row = valid ? tile_row(P, x, t0 + ri) : 0;
-                // Pass B's shift is known before S: fetch it while the MMA runs.
-                float shift = 0.f;
-                if (MODE == 1 && valid) shift = P.m_arr[row * P.H_q + x.g * kG + h];
-                bool have = !*abort_flag && mbar_wait(&S.s_full[ss], (qt >> 1) & 1, P.status);
+                const long long row = row_nx;
+                float shift = shift_nx;
+                if (t0 + kTileRows < x.n) {
+                    load_tile(x, t0 + kTileRows, row_nx, shift_nx);
+                } else {
+                    if (!fetch(xn)) { ok = false; break; }
+                    if (xn.n > 0) load_tile(xn, 0, row_nx, shift_nx);
+                }
+                bool have = !*abort_flag && mbar_wait(&S.s_full, qt & 1, P.status);
                 have = __all_sync(0xffffffffu, have);
                 if (!have) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t sa = lane_addr + ss * 128;
+                float nq = 0.f;                        // pass A: |q|^2 of this (row, head)
+                if (MODE == 0) {
+                    // The Q tile goes back to the producer as soon as its norms
+                    // are read, so the next tiles' loads overlap this softmax.
+                    bool qok = !*abort_flag && mbar_wait(&S.q_full[qt & 1], (qt >> 1) & 1, P.status);
+                    qok = __all_sync(0xffffffffu, qok);
+                    if (!qok) { ok = false; break; }
+                    if (ch == 0 && valid) {
+                        const uint8_t *qs = S.q[qt & 1];
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) {
+                            const uint4 w = *reinterpret_cast<const uint4 *>(
+                                qs + (c >> 3) * 16384 + swz128(m, c & 7));
+                            const uint32_t a4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                nq = fmaf(bf16lo(a4[e]), bf16lo(a4[e]), nq);
+                                nq = fmaf(bf16hi(a4[e]), bf16hi(a4[e]), nq);
+                            }
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.q_empty[qt & 1]);
+                }
+                const uint32_t sa = lane_addr + kColS;
                 long long lim = 127;                   // last visible column of the row
                 if (MODE == 0) {
                     // own block: causal mask t <= p, exact max of the visible logits
@@ -454,6 +477,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32r(sa + ch * 64 + 32, b);
                 tmem_wait_ld(a);
                 tmem_tie(b);
+                // S is in registers: the next tile's QK may overwrite it.
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.s_empty);
                 float l = 0.f;
                 uint32_t pk[32];                        // 64 probabilities as bf16 pairs
 #pragma unroll
@@ -461,21 +488,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int c0 = ch * 64 + 2 * e;
                     const uint32_t *src = e < 16 ? a : b;
                     const int k = (2 * e) & 31;
-                    float p0 = exp2f(__uint_as_float(src[k]) * sl2 - shift);
-                    float p1 = exp2f(__uint_as_float(src[k + 1]) * sl2 - shift);
+                    float p0 = fast_exp2(__uint_as_float(src[k]) * sl2 - shift);
+                    float p1 = fast_exp2(__uint_as_float(src[k + 1]) * sl2 - shift);
                     p0 = (valid && c0 <= lim) ? p0 : 0.f;
                     p1 = (valid && c0 + 1 <= lim) ? p1 : 0.f;
                     l += p0 + p1;
                     pk[e] = pack_bf16x2(p0, p1);
                 }
-                // P buffer is free once the previous tile's PV has read it.
+                // P's columns are free once the previous tile's PV has read them.
                 bool pfree = !*abort_flag && (qt == 0 || mbar_wait(&S.p_empty, (qt - 1) & 1, P.status));
                 pfree = __all_sync(0xffffffffu, pfree);
                 if (!pfree) { ok = false; break; }
-#pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8)
-                    *reinterpret_cast<uint4 *>(S.p + ch * 16384 + swz128(m, c8)) =
-                        make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
+                tc_fence_after();
+                tmem_st32(lane_addr + kColP + ch * 32, pk);
                 if (zero_v) {
                     bool kok = !*abort_flag && mbar_wait(&S.kv_full[kvs], kv_par, P.status);
                     kok = __all_sync(0xffffffffu, kok);
@@ -487,34 +512,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         *reinterpret_cast<uint4 *>(S.kv[kvs] + 32768 + (c16 >> 3) * 16384 +
                                                    rrow * 128 + (c16 & 7) * 16) = make_uint4(0, 0, 0, 0);
                     }
+                    fence_proxy_async_smem();
                     zero_v = false;
                 }
-                fence_proxy_async_smem();
+                tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&S.s_empty[ss]);
-                    mbar_arrive(&S.p_full);
-                }
+                if (lane == 0) mbar_arrive(&S.p_full);
+                if (valid) atomicAdd(P.l_acc + row * P.H_q + x.g * kG + h, l);
                 if (MODE == 0) {
-                    bool qok = !*abort_flag && mbar_wait(&S.q_full[qt & 1], (qt >> 1) & 1, P.status);
-                    qok = __all_sync(0xffffffffu, qok);
-                    if (!qok) { ok = false; break; }
                     if (ch == 0 && valid) {
                         // Shift of this (row, head) and the safety test of the bound.
-                        const uint8_t *qs = S.q[qt & 1];
-                        float nq = 0.f;
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            const uint4 w = *reinterpret_cast<const uint4 *>(
-                                qs + (c >> 3) * 16384 + swz128(m, c & 7));
-                            const uint32_t a4[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                nq = fmaf(bf16lo(a4[e]), bf16lo(a4[e]), nq);
-                                nq = fmaf(bf16hi(a4[e]), bf16hi(a4[e]), nq);
-                            }
-                        }
                         const float bound = fabsf(sl2) * sqrtf(nq) * P.knorm[x.b * P.H_kv + x.g];
                         const long long idx = row * P.H_q + x.g * kG + h;
                         P.m_arr[idx] = shift;
@@ -522,19 +530,109 @@ __global__ void __launch_bounds__(kThreads, 1)
                         P.flags[idx] = fl;
                         if (fl) atomicAdd(P.flag_count, 1);
                     }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&S.q_empty[qt & 1]);
                 }
-                // Output of the previous tile (its PV ran while this tile's QK did).
-                if (prev >= 0 && !epilogue(prev, prev_row, prev_g, prev_valid, prev_l)) { ok = false; break; }
-                prev = qt;
-                prev_row = row;
-                prev_g = x.g;
-                prev_valid = valid;
-                prev_l = l;
             }
+            x = xn;
         }
-        if (ok && prev >= 0 && !epilogue(prev, prev_row, prev_g, prev_valid, prev_l)) ok = false;
+        if (!ok) *abort_flag = 1;
+    } else if (warp >= kEpiWarp0) {
+        // ------------------------------------------------ epilogue
+        // Warp w owns the TMEM lanes of w % 4 (tile rows 4(w%4) .. +3, all 8
+        // heads), one (tile row, head) per thread.  Each half of the output
+        // dims goes through the warp's 8 KiB staging slot, laid out as the
+        // accumulator is (a row's 8 heads interleaved at 16-byte granularity),
+        // and leaves as one 2 KiB bulk copy (pass A) or bulk fp32 add (pass B)
+        // per row, issued by the row's head-0 lane: the reductions run on the
+        // bulk-copy engine.
+        const int w = warp & 3;
+        const int m = w * 32 + lane;
+        const int ri = m / kG, h = m % kG;
+        const bool issuer = lane == 0;
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(w * 32) << 16);
+        uint8_t *stage = S.ostage[w] + (ri & 3) * 2048;
+        uint8_t *stage0 = S.ostage[w];
+        int qt = 0;
+        bool ok = true;
+        // Rows are loaded one tile ahead, as in the softmax warps.
+        int n = 0;
+        auto fetch = [&](Item &it) -> bool {
+            do {
+                if (!next_item(n++, true, it)) return false;
+            } while (it.n == 0);
+            return true;
+        };
+        auto load_row = [&](const Item &it, int t0) -> long long {
+            return t0 + ri < it.n ? tile_row<MODE>(P, it, t0 + ri) : -1;
+        };
+        Item x;
+        long long row_nx = -1;
+        if (!fetch(x)) ok = false;
+        else if (x.n > 0) row_nx = load_row(x, 0);
+        while (ok && x.n > 0) {
+            Item xn;
+            xn.n = -1;
+            for (int t0 = 0; t0 < x.n; t0 += kTileRows, ++qt) {
+                const int os = qt & 1;
+                const long long row = row_nx;
+                const bool valid = row >= 0;
+                if (t0 + kTileRows < x.n) {
+                    row_nx = load_row(x, t0 + kTileRows);
+                } else {
+                    if (!fetch(xn)) { ok = false; break; }
+                    if (xn.n > 0) row_nx = load_row(xn, 0);
+                }
+                float *dst4[4];
+#pragma unroll
+                for (int r4 = 0; r4 < 4; ++r4) {
+                    const long long rr = __shfl_sync(0xffffffffu, row, r4 * 8);
+                    dst4[r4] = rr >= 0 ? P.o_acc + (rr * P.H_kv + x.g) * (kDim * kG) : nullptr;
+                }
+                bool have = !*abort_flag && mbar_wait(&S.o_full[os], (qt >> 1) & 1, P.status);
+                have = __all_sync(0xffffffffu, have);
+                if (!have) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t a[32], b[32];
+                    tmem_ld32r(lane_addr + kColO + os * 128 + half * 64, a);
+                    tmem_ld32r(lane_addr + kColO + os * 128 + half * 64 + 32, b);
+                    tmem_wait_ld(a);
+                    tmem_tie(b);
+                    if (half == 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&S.o_empty[os]);
+                    }
+                    // The slot is free once the bulk engine has read the last groups.
+                    if (issuer) bulk_wait_read_all();
+                    __syncwarp();
+                    if (valid) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 16; ++q4) {
+                            const uint32_t *r = q4 < 8 ? a + 4 * q4 : b + 4 * (q4 - 8);
+                            *reinterpret_cast<uint4 *>(stage + q4 * 128 + h * 16) =
+                                make_uint4(r[0], r[1], r[2], r[3]);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (issuer) {
+#pragma unroll
+                        for (int r4 = 0; r4 < 4; ++r4) {
+                            if (!dst4[r4]) continue;
+                            float *g = dst4[r4] + half * (kDim * kG / 2);
+                            if (MODE == 0) bulk_s2g(g, stage0 + r4 * 2048, 2048);
+                            else bulk_s2g_add_f32(g, stage0 + r4 * 2048, 2048);
+                        }
+                        bulk_commit();
+                    }
+                }
+            }
+            x = xn;
+        }
+        // Staging must stay valid, and the adds land, before the CTA ends.
+        if (issuer) bulk_wait_all();
+        __syncwarp();
         if (!ok) *abort_flag = 1;
     }
 
@@ -690,6 +788,47 @@ __global__ void __launch_bounds__(1024) range_scan_kernel(const PrefillArgs P) {
     }
 }
 
+// Flat table of pass-B work items: the descriptor of global item
+// range_item_off[r] + li, for every range r and local item li, so that an item
+// is decoded with one 32-byte load.  One CTA per range.
+__global__ void item_table_kernel(const PrefillArgs P) {
+    const long long r = blockIdx.x;
+    const long long n = P.range_count[r];
+    if (n == 0) return;                        // also every range of a rejected sequence
+    const int g = static_cast<int>((r / P.n_ranges) % P.H_kv);
+    const int b = static_cast<int>(r / (static_cast<long long>(P.n_ranges) * P.H_kv));
+    const int L = P.lens[b];
+    const long long base = P.range_item_off[r];
+    for (long long li = threadIdx.x; li < n; li += blockDim.x) {
+        const int j = P.item_bucket[r * P.items_per_range + li];
+        const long long bk = r * P.nb_max + j;
+        const int chunk = static_cast<int>(li) - P.item_off[bk];
+        const int cnt = P.bucket_cnt[bk];
+        int4 *d = reinterpret_cast<int4 *>(P.item_desc) + 2 * (base + li);
+        d[0] = make_int4(b, g, j, min(kItemRows, cnt - chunk * kItemRows));
+        d[1] = make_int4(P.bucket_off[bk] + chunk * kItemRows, L, 0, 0);
+    }
+}
+
+// The shift of every (bucket entry, head), copied from the per-(row, head)
+// shifts once pass A and the fix-up have set them: pass B then reads a tile's
+// shifts as one contiguous 512-byte run.  Two threads per entry (4 heads each).
+__global__ void bucket_shift_kernel(const PrefillArgs P) {
+    const long long total = *P.item_total * (kItemRows * 2);
+    const int4 *desc = reinterpret_cast<const int4 *>(P.item_desc);
+    for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+         t += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long it = t / (kItemRows * 2);
+        const int rr = static_cast<int>((t >> 1) % kItemRows), half = static_cast<int>(t & 1);
+        const int4 a = desc[2 * it];            // b, g, j, n
+        if (rr >= a.w) continue;
+        const long long e = desc[2 * it + 1].x + rr;
+        const long long row = P.bucket_rows[e];
+        const float4 v = *reinterpret_cast<const float4 *>(P.m_arr + row * P.H_q + a.y * kG + half * 4);
+        *reinterpret_cast<float4 *>(P.bucket_shift + e * kG + half * 4) = v;
+    }
+}
+
 // Flagged (row, head): exact max logit over the row's other kept keys, then
 // the own-block partials are rescaled to the new shift.  Exits at once when
 // no row was flagged.  One warp per (row, group).
@@ -816,6 +955,8 @@ size_t prefill_workspace_layout(int B, int Sq, int H_q, int H_kv, int K, int max
     L->range_count = o;  o += up(static_cast<size_t>(L->n_ranges_total) * 8);
     L->range_item_off = o; o += up(static_cast<size_t>(L->n_ranges_total + 1) * 8);
     L->rows = o;         o += up(static_cast<size_t>(L->n_ranges_total) * per_range_rows * 4);
+    L->shift = o;        o += up(static_cast<size_t>(L->n_ranges_total) * per_range_rows * kG * 4);
+    L->item_desc = o;    o += up(static_cast<size_t>(L->n_ranges_total) * L->items_per_range * 32);
     L->o_acc = o;        o += up(static_cast<size_t>(rows) * H_q * kDim * 4);
     L->m_arr = o;        o += up(static_cast<size_t>(rows) * H_q * 4);
     L->flags = o;        o += up(static_cast<size_t>(rows) * H_q);
@@ -835,6 +976,8 @@ cudaError_t launch_prefill_attention(const PrefillArgs &a0, uint8_t *ws, const P
     a.range_count = reinterpret_cast<long long *>(ws + L.range_count);
     a.range_item_off = reinterpret_cast<long long *>(ws + L.range_item_off);
     a.bucket_rows = reinterpret_cast<int *>(ws + L.rows);
+    a.bucket_shift = reinterpret_cast<float *>(ws + L.shift);
+    a.item_desc = reinterpret_cast<int *>(ws + L.item_desc);
     a.o_acc = reinterpret_cast<float *>(ws + L.o_acc);
     a.l_acc = reinterpret_cast<float *>(ws + L.l_acc);
     a.m_arr = reinterpret_cast<float *>(ws + L.m_arr);
@@ -864,12 +1007,17 @@ cudaError_t launch_prefill_attention(const PrefillArgs &a0, uint8_t *ws, const P
         TraceScope t(s, "prefill_bucket");
         bucket_build_kernel<<<static_cast<unsigned>(L.n_ranges_total), kBuildThreads, 0, s>>>(a);
         range_scan_kernel<<<1, 1024, 0, s>>>(a);
+        item_table_kernel<<<static_cast<unsigned>(L.n_ranges_total), 256, 0, s>>>(a);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_pass<0>(tq, tk, tv, a, s, "prefill_attn_own_block")) != cudaSuccess) return e;
     {
         TraceScope t(s, "prefill_fixup");
         fixup_kernel<<<sms * 4, 256, 0, s>>>(a);
+    }
+    {
+        TraceScope t(s, "prefill_bucket_shift");
+        bucket_shift_kernel<<<sms * 8, 256, 0, s>>>(a);
     }
     if ((e = launch_pass<1>(tq, tk, tv, a, s, "prefill_attn_kv_outer")) != cudaSuccess) return e;
     {

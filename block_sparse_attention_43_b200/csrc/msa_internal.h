@@ -116,6 +116,8 @@ struct PrefillArgs {
     int *bucket_cnt, *bucket_cur, *bucket_off, *bucket_rows;  // per (range, block j)
     int *item_off;          // first item of each bucket, counted inside its range
     int *item_bucket;       // [range][item] -> block j
+    int *item_desc;         // [item] {b, g, j, n}, {first bucket entry, L, 0, 0}
+    float *bucket_shift;    // [bucket entry][8 heads] softmax shift of the entry's row
     long long *range_count, *range_item_off;
     long long *item_total;
     long long *item_next;   // claim counters of pass A and pass B (zeroed per call)
@@ -127,7 +129,7 @@ struct PrefillArgs {
 };
 struct PrefillLayout {
     size_t knorm, cnt, cur, l_acc, zero_end, off, item_off, item_bucket, range_count,
-        range_item_off, rows, o_acc, m_arr, flags, total;
+        range_item_off, rows, shift, item_desc, o_acc, m_arr, flags, total;
     int nb_max, n_ranges, rows_per_range, items_per_range;
     long long n_ranges_total, n_buckets;
 };
