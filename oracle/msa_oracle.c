@@ -23,8 +23,19 @@
  * own block always kept, ties to the lower block id, 1/sqrt(d) on the sparse
  * branch) are listed in the design notes and restated at each step below.
  *
- * Arithmetic: bf16 inputs are widened exactly to double; every sum, max and
- * exponential is in double.  Rows are independent, so they are spread over
+ * Index-branch variants (the guide's configuration sets
+ * sparse_num_index_heads = 4, which one index head per GQA group cannot
+ * match; the pages fix nothing more, so these are the plainest readings):
+ *   - Hi index heads partition the GQA groups into contiguous sets of
+ *     H_kv / Hi groups, and every group of a set uses its index head's
+ *     selection (Hi = H_kv is one index head per group);
+ *   - index keys are either one per (token, index head) or one per token,
+ *     shared by every index head;
+ *   - index keys are bf16, or FP8 E4M3 with one fp32 scale per key row: the
+ *     score is scale * (q_idx . k), the dot over the exactly decoded values.
+ *
+ * Arithmetic: bf16 and e4m3 inputs are widened exactly to double; every sum,
+ * max and exponential is in double.  Rows are independent, so they are spread over
  * POSIX threads; no row's arithmetic is split, reordered or fused.
  *
  * Build: gcc -O2 -std=c11 -fPIC -shared -pthread -ffp-contract=off
@@ -44,8 +55,28 @@ static double bf16_to_double(uint16_t h)
     return (double)f;
 }
 
+/* FP8 E4M3 (the OCP 8-bit floating-point format, "E4M3FN": no infinities,
+ * S.1111.111 is NaN) -> double, exact.  Exponent bias 7; exponent field 0 is
+ * the subnormal range 2^-6 * m/8. */
+static double e4m3_to_double(uint8_t x)
+{
+    const int sgn = x >> 7, e = (x >> 3) & 15, m = x & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m / 8.0, -6);
+    else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sgn ? -v : v;
+}
+
+double oracle_e4m3_to_double(int x) { return e4m3_to_double((uint8_t)x); }
+
 typedef struct {
     int B, Sq, H_q, H_kv, D, block, top_k;
+    int KH;               /* index-key heads: 1 (shared) or H_kv (= index heads) */
+    int key_fp8;          /* index keys are E4M3 bytes with per-row scales */
+    int n_idx;            /* sparse branch: index heads whose selections the groups use */
+    const uint8_t *k_idx8;
+    const float *k_scale; /* [T, KH] */
     int64_t kv_capacity;
     const uint16_t *q_idx, *k_idx, *q, *k, *v;
     const int32_t *lens, *block_ids_in;
@@ -115,18 +146,28 @@ static void index_row(job_t *J, int64_t rr, int g)
     int *sel = (int *)malloc(sizeof(int) * (K + 1));
     {
         const uint16_t *qi = J->q_idx + (r * J->H_kv + g) * (int64_t)Di;
-        /* Step 1+2: per-token index score (plain dot product of the group's
-         * index query with the token's index key, no scale), then the block
+        const int kh = J->KH == 1 ? 0 : g;   /* shared keys: one row per token */
+        /* Step 1+2: per-token index score (plain dot product of the index
+         * head's query with the token's index key, no scale; FP8 keys: the
+         * row's scale times the dot over the decoded values), then the block
          * max-pool over the visible tokens t <= p of each block. */
         for (int j = 0; j < nvis; ++j) {
             double best = -INFINITY;
             int64_t t_end = (int64_t)(j + 1) * blk;
             if (t_end > p + 1) t_end = p + 1;
             for (int64_t t = (int64_t)j * blk; t < t_end; ++t) {
-                const uint16_t *ki = J->k_idx + ((off + t) * J->H_kv + g) * (int64_t)Di;
+                const int64_t krow = (off + t) * J->KH + kh;
                 double s = 0.0;
-                for (int d = 0; d < Di; ++d)
-                    s += bf16_to_double(qi[d]) * bf16_to_double(ki[d]);
+                if (J->key_fp8) {
+                    const uint8_t *ki = J->k_idx8 + krow * (int64_t)Di;
+                    for (int d = 0; d < Di; ++d)
+                        s += bf16_to_double(qi[d]) * e4m3_to_double(ki[d]);
+                    s *= (double)J->k_scale[krow];
+                } else {
+                    const uint16_t *ki = J->k_idx + krow * (int64_t)Di;
+                    for (int d = 0; d < Di; ++d)
+                        s += bf16_to_double(qi[d]) * bf16_to_double(ki[d]);
+                }
                 if (s > best) best = s;
             }
             S[j] = best;
@@ -180,7 +221,9 @@ static void attn_row(job_t *J, int64_t rr, int h)
     double *z = (double *)malloc(sizeof(double) * max_keys);
     {
         const int g = h / G;                 /* contiguous head -> group map */
-        const int32_t *ids = J->block_ids_in + (r * J->H_kv + g) * (int64_t)K;
+        /* contiguous group -> index-head map: H_kv / n_idx groups per index head */
+        const int gi = g / (J->H_kv / J->n_idx);
+        const int32_t *ids = J->block_ids_in + (r * J->n_idx + gi) * (int64_t)K;
         int64_t nk = 0;
         for (int q = 0; q < K; ++q) {
             int j = ids[q];
@@ -261,17 +304,25 @@ static int run(job_t *J, int kind, int n_threads)
  * visible block score and the ranking boundary (score of the last kept and of
  * the first dropped non-own block).  rows == NULL means all B*Sq rows.
  * Returns 0, or non-zero on an invalid input. */
-int oracle_index_topk(int B, int Sq, int H_kv, int D_idx, int block, int top_k,
-                      const uint16_t *q_idx, const uint16_t *k_idx,
-                      const int32_t *lens, const int64_t *kv_offsets, int64_t kv_capacity,
-                      const int64_t *rows, int64_t n_rows,
-                      int32_t *block_ids, float *block_scores,
-                      double *all_scores, int nb_max, double *boundary, int n_threads)
+/* Index branch with n_idx index heads (q_idx [B, Sq, n_idx, D_idx]), key_heads
+ * index-key rows per token (1: shared; n_idx: one per index head), keys bf16
+ * (k_idx) or E4M3 bytes (k_idx8, with k_scale [T, key_heads]).  Outputs as
+ * oracle_index_topk, with n_idx in place of H_kv. */
+int oracle_index_topk_ex(int B, int Sq, int n_idx, int key_heads, int D_idx, int block, int top_k,
+                         const uint16_t *q_idx, const uint16_t *k_idx, const uint8_t *k_idx8,
+                         const float *k_scale,
+                         const int32_t *lens, const int64_t *kv_offsets, int64_t kv_capacity,
+                         const int64_t *rows, int64_t n_rows,
+                         int32_t *block_ids, float *block_scores,
+                         double *all_scores, int nb_max, double *boundary, int n_threads)
 {
-    if (B < 1 || Sq < 1 || H_kv < 1 || D_idx < 1 || block < 1 || top_k < 1) return -1;
+    if (B < 1 || Sq < 1 || n_idx < 1 || D_idx < 1 || block < 1 || top_k < 1) return -1;
+    if (key_heads != 1 && key_heads != n_idx) return -1;
+    if ((k_idx8 == NULL) == (k_idx == NULL) || (k_idx8 != NULL && k_scale == NULL)) return -1;
     job_t J;
     memset(&J, 0, sizeof J);
-    J.B = B; J.Sq = Sq; J.H_kv = H_kv; J.D = D_idx; J.block = block; J.top_k = top_k;
+    J.B = B; J.Sq = Sq; J.H_kv = n_idx; J.D = D_idx; J.block = block; J.top_k = top_k;
+    J.KH = key_heads; J.key_fp8 = k_idx8 != NULL; J.k_idx8 = k_idx8; J.k_scale = k_scale;
     J.q_idx = q_idx; J.k_idx = k_idx; J.lens = lens; J.kv_offsets = kv_offsets;
     J.kv_capacity = kv_capacity; J.rows = rows;
     J.n_rows = rows ? n_rows : (int64_t)B * Sq;
@@ -280,8 +331,44 @@ int oracle_index_topk(int B, int Sq, int H_kv, int D_idx, int block, int top_k,
     return run(&J, 0, n_threads);
 }
 
+/* One index head per GQA group with its own bf16 keys (k_idx [T, H_kv, D]). */
+int oracle_index_topk(int B, int Sq, int H_kv, int D_idx, int block, int top_k,
+                      const uint16_t *q_idx, const uint16_t *k_idx,
+                      const int32_t *lens, const int64_t *kv_offsets, int64_t kv_capacity,
+                      const int64_t *rows, int64_t n_rows,
+                      int32_t *block_ids, float *block_scores,
+                      double *all_scores, int nb_max, double *boundary, int n_threads)
+{
+    return oracle_index_topk_ex(B, Sq, H_kv, H_kv, D_idx, block, top_k, q_idx, k_idx, NULL, NULL,
+                                lens, kv_offsets, kv_capacity, rows, n_rows, block_ids,
+                                block_scores, all_scores, nb_max, boundary, n_threads);
+}
+
 /* Sparse branch: out[n_rows, H_q, D] in double, given the block ids of each
- * (row, group); optionally the sum of each row's normalised weights. */
+ * (row, index head) [B*Sq, n_idx, top_k], group g using index head
+ * g / (H_kv / n_idx); optionally the sum of each row's normalised weights. */
+int oracle_sparse_attention_ex(int B, int Sq, int H_q, int H_kv, int n_idx, int D, int block,
+                               int top_k, const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                               const int32_t *block_ids, const int32_t *lens,
+                               const int64_t *kv_offsets, int64_t kv_capacity, double scale,
+                               const int64_t *rows, int64_t n_rows,
+                               double *out, double *wsum, int n_threads)
+{
+    if (B < 1 || Sq < 1 || H_q < 1 || H_kv < 1 || H_q % H_kv || D < 1 || block < 1 || top_k < 1)
+        return -1;
+    if (n_idx < 1 || H_kv % n_idx) return -1;
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.B = B; J.Sq = Sq; J.H_q = H_q; J.H_kv = H_kv; J.D = D; J.block = block; J.top_k = top_k;
+    J.n_idx = n_idx;
+    J.q = q; J.k = k; J.v = v; J.block_ids_in = block_ids; J.lens = lens;
+    J.kv_offsets = kv_offsets; J.kv_capacity = kv_capacity; J.scale = scale;
+    J.rows = rows; J.n_rows = rows ? n_rows : (int64_t)B * Sq;
+    J.out = out; J.wsum = wsum;
+    return run(&J, 1, n_threads);
+}
+
+/* One index head per GQA group: block_ids [B*Sq, H_kv, top_k]. */
 int oracle_sparse_attention(int B, int Sq, int H_q, int H_kv, int D, int block, int top_k,
                             const uint16_t *q, const uint16_t *k, const uint16_t *v,
                             const int32_t *block_ids, const int32_t *lens,
@@ -289,14 +376,7 @@ int oracle_sparse_attention(int B, int Sq, int H_q, int H_kv, int D, int block, 
                             const int64_t *rows, int64_t n_rows,
                             double *out, double *wsum, int n_threads)
 {
-    if (B < 1 || Sq < 1 || H_q < 1 || H_kv < 1 || H_q % H_kv || D < 1 || block < 1 || top_k < 1)
-        return -1;
-    job_t J;
-    memset(&J, 0, sizeof J);
-    J.B = B; J.Sq = Sq; J.H_q = H_q; J.H_kv = H_kv; J.D = D; J.block = block; J.top_k = top_k;
-    J.q = q; J.k = k; J.v = v; J.block_ids_in = block_ids; J.lens = lens;
-    J.kv_offsets = kv_offsets; J.kv_capacity = kv_capacity; J.scale = scale;
-    J.rows = rows; J.n_rows = rows ? n_rows : (int64_t)B * Sq;
-    J.out = out; J.wsum = wsum;
-    return run(&J, 1, n_threads);
+    return oracle_sparse_attention_ex(B, Sq, H_q, H_kv, H_kv, D, block, top_k, q, k, v, block_ids,
+                                      lens, kv_offsets, kv_capacity, scale, rows, n_rows, out, wsum,
+                                      n_threads);
 }
