@@ -1,11 +1,13 @@
 """Benchmark of the MSA hot path on B200: one step = the whole decode path
 (index score + block max-pool, top-k, sparse attention with split-K merge)
-for one batch, through the C ABI; a decode run also times one 128k-token
-prefill (index GEMM + fused top-k, sparse attention) as a sub-object.
+for one batch, through the C ABI; a decode run also times the same decode
+step on the index-branch variants (fewer index heads, shared index keys,
+E4M3 index keys) and one 128k-token prefill (index GEMM + fused top-k,
+sparse attention) as sub-objects.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode_1m]
                     [--impl msa|reference] [--no-cpu-baseline] [--no-e2e]
-                    [--no-prefill] [--prefill-steps S] [--prefill-len N]
+                    [--no-prefill] [--no-variants] [--prefill-steps S] [--prefill-len N]
 
 Prints ONE JSON line (rank 0).  N > 1 runs under torchrun: every rank runs
 its own independent batch (weak scaling, no data-path collective).
@@ -47,6 +49,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the prefill_128k measurement attached to a decode run")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the index-branch variant measurement attached to a decode run")
     ap.add_argument("--prefill-steps", type=int, default=5)
     ap.add_argument("--prefill-len", type=int, default=None,
                     help="override the prefill length (profiling captures of a smaller case)")
@@ -158,6 +162,86 @@ def measure_prefill(name, dev, steps, warmup, seq_len=None):
     del eng, w
     torch.cuda.empty_cache()
     return res
+
+
+def _variant_keys(w, Hi, fmt, msa):
+    """Index queries / keys of an index-branch variant, built from w's tensors
+    (per-head keys are the first Hi groups' keys; shared keys the first
+    group's; E4M3 codes quantised per key row in chunks)."""
+    from synthetic import quantize_e4m3_rows
+    shared = fmt in (msa.INDEX_KEYS_BF16_SHARED, msa.INDEX_KEYS_FP8_SHARED)
+    q_idx = w.q_idx[:, :, :Hi].contiguous()
+    src = w.k_idx[:, :1 if shared else Hi]
+    if fmt in (msa.INDEX_KEYS_BF16, msa.INDEX_KEYS_BF16_SHARED):
+        return q_idx, src.contiguous(), None
+    T = src.shape[0]
+    codes = torch.empty(src.shape, dtype=torch.uint8, device=src.device)
+    scale = torch.empty(src.shape[:2], dtype=torch.float32, device=src.device)
+    step = 1 << 20
+    for t0 in range(0, T, step):
+        c, s = quantize_e4m3_rows(src[t0:t0 + step])
+        codes[t0:t0 + step] = c
+        scale[t0:t0 + step] = s
+    return q_idx, codes, scale
+
+
+def measure_index_variants(w, dev, steps, warmup):
+    """Decode step (index + top-k + sparse attention) on the index-branch
+    variants: the guide's 4 index heads for 8 groups (bf16 keys per head),
+    keys shared by the index heads (bf16, E4M3) and E4M3 keys per head.
+    Index bytes = keys (+ row scales) + index queries + block scores."""
+    import block_sparse_attention_43_b200 as msa
+    peak, _, _, kind = measured_peaks()
+    lens = np.asarray(w.lens_host, np.int64)
+    nb = int(((lens + 127) // 128).sum())
+    ntok = int(lens.sum())
+    cases = [("4_index_heads_bf16", 4, msa.INDEX_KEYS_BF16),
+             ("shared_keys_bf16", w.H_kv, msa.INDEX_KEYS_BF16_SHARED),
+             ("per_head_keys_fp8", w.H_kv, msa.INDEX_KEYS_FP8),
+             ("shared_keys_fp8", w.H_kv, msa.INDEX_KEYS_FP8_SHARED)]
+    out = {}
+    stream = torch.cuda.Stream(device=dev)
+    for name, Hi, fmt in cases:
+        q_idx, keys, scale = _variant_keys(w, Hi, fmt, msa)
+        eng = msa.MSA(batch=w.B, q_len=1, max_kv_len=max(w.lens_host), num_q_heads=w.H_q,
+                      num_kv_heads=w.H_kv, top_k=w.top_k, kv_capacity=w.kv_capacity, device=dev,
+                      num_index_heads=Hi, index_key_format=fmt)
+
+        def step():
+            eng.index_topk(q_idx, keys, w.lens, w.kv_offsets, stream, k_idx_scale=scale)
+            eng.sparse_attention(w.q, w.k, w.v, w.lens, w.kv_offsets, stream=stream)
+
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize()
+        st = eng.device_status(stream)
+        if st != 0:
+            raise RuntimeError(f"{name}: device status {msa.STATUS_NAMES.get(st, st)}")
+        msa.msa_trace_enable(True)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        trace = msa.msa_trace_read()
+        msa.msa_trace_enable(False)
+        per = {}
+        for n, t in trace:
+            per[n] = per.get(n, 0.0) + t / steps
+        idx_name = [n for n in per if n.startswith("index_score_maxpool_decode")][0]
+        kh = keys.shape[1]
+        key_bytes = ntok * kh * w.d_idx * keys.element_size() + (ntok * kh * 4 if scale is not None else 0)
+        idx_bytes = key_bytes + w.B * Hi * w.d_idx * 2 + nb * Hi * 4
+        gbs = idx_bytes / (per[idx_name] / 1e3) / 1e9
+        out[name] = {"index_heads": Hi, "key_rows_per_token": kh,
+                     "key_dtype": "e4m3" if scale is not None else "bf16",
+                     "ms_per_step": ev0.elapsed_time(ev1) / steps, "kernel_ms": per,
+                     "index_bytes": idx_bytes, "index_gbs": gbs, "index_frac_of_hbm": gbs / peak,
+                     "peak_kind": kind}
+        del eng, q_idx, keys, scale
+        torch.cuda.empty_cache()
+    return out
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -418,6 +502,10 @@ def main():
         cpu = {"value": gbs, "unit": "GB/s", "cores": used, "kind": "oracle", "sample": note,
                "seconds": dt}
 
+    variants = None
+    if not args.no_variants and world == 1:
+        variants = measure_index_variants(w, dev, 20, 3)
+
     prefill = None
     if not args.no_prefill and world == 1:
         del eng
@@ -457,6 +545,7 @@ def main():
             "e2e": e2e,
             "cpu_baseline": cpu,
             "prefill_128k": prefill,
+            "index_variants": variants,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
                 6: "MSA_ERR_BAD_LENS", 7: "MSA_ERR_MISALIGNED"}
 
 # Every entry point include/msa.h declares.
-EXPORTS = ("msa_index_topk_workspace_size", "msa_index_topk",
+EXPORTS = ("msa_index_topk_workspace_size", "msa_index_topk", "msa_index_topk_fp8",
            "msa_sparse_attention_workspace_size", "msa_sparse_attention",
            "msa_index_topk_paged", "msa_sparse_attention_paged", "msa_kv_append",
            "msa_index_topk_static", "msa_read_device_status", "msa_trace_enable",
@@ -35,7 +35,12 @@ class msa_shape_t(ctypes.Structure):
                 ("max_kv_len", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("index_dim", ctypes.c_int32), ("block_size", ctypes.c_int32),
-                ("top_k", ctypes.c_int32), ("kv_capacity", ctypes.c_int64)]
+                ("top_k", ctypes.c_int32), ("kv_capacity", ctypes.c_int64),
+                ("num_index_heads", ctypes.c_int32), ("index_key_format", ctypes.c_int32)]
+
+
+# msa_index_key_format_t
+INDEX_KEYS_BF16, INDEX_KEYS_BF16_SHARED, INDEX_KEYS_FP8, INDEX_KEYS_FP8_SHARED = 0, 1, 2, 3
 
 
 class MSAError(RuntimeError):
@@ -56,6 +61,8 @@ def _load():
     lib.msa_sparse_attention_workspace_size.restype = Z
     lib.msa_index_topk.argtypes = [S, P, P, P, P, P, P, P, Z, P]
     lib.msa_index_topk.restype = ctypes.c_int
+    lib.msa_index_topk_fp8.argtypes = [S, P, P, P, P, P, P, P, P, Z, P]
+    lib.msa_index_topk_fp8.restype = ctypes.c_int
     lib.msa_sparse_attention.argtypes = [S, P, P, P, P, P, P, ctypes.c_float, P, P, Z, P]
     lib.msa_sparse_attention.restype = ctypes.c_int
     I32 = ctypes.c_int32
@@ -83,9 +90,10 @@ lib = _load()
 
 
 def make_shape(*, batch, q_len, max_kv_len, num_q_heads, num_kv_heads, top_k, kv_capacity,
-               head_dim=128, index_dim=128, block_size=128) -> msa_shape_t:
+               head_dim=128, index_dim=128, block_size=128, num_index_heads=0,
+               index_key_format=INDEX_KEYS_BF16) -> msa_shape_t:
     return msa_shape_t(batch, q_len, max_kv_len, num_q_heads, num_kv_heads, head_dim, index_dim,
-                       block_size, top_k, kv_capacity)
+                       block_size, top_k, kv_capacity, num_index_heads, index_key_format)
 
 
 def _ptr(t):
@@ -123,6 +131,17 @@ def msa_index_topk(shape, q_idx, k_idx, lens, kv_offsets, block_ids, block_score
                               _ptr(kv_offsets), _ptr(block_ids), _ptr(block_scores),
                               _ptr(workspace), workspace.numel(), _stream(stream)),
            "msa_index_topk")
+
+
+def msa_index_topk_fp8(shape, q_idx, k_idx_fp8, k_idx_scale, lens, kv_offsets, block_ids,
+                       block_scores, workspace, stream=None) -> None:
+    """Index branch on FP8 E4M3 index keys (uint8 codes) with fp32 per-row
+    scales, decode only; see include/msa.h."""
+    _check(lib.msa_index_topk_fp8(ctypes.byref(shape), _ptr(q_idx), _ptr(k_idx_fp8),
+                                  _ptr(k_idx_scale), _ptr(lens), _ptr(kv_offsets), _ptr(block_ids),
+                                  _ptr(block_scores), _ptr(workspace), workspace.numel(),
+                                  _stream(stream)),
+           "msa_index_topk_fp8")
 
 
 def msa_sparse_attention(shape, q, k_cache, v_cache, block_ids, lens, kv_offsets, softmax_scale,
@@ -204,10 +223,11 @@ class MSA:
     Holds torch tensors only; every call goes straight to the C ABI."""
 
     def __init__(self, *, batch, q_len, max_kv_len, num_q_heads, num_kv_heads, top_k,
-                 kv_capacity, device="cuda"):
+                 kv_capacity, device="cuda", num_index_heads=0, index_key_format=INDEX_KEYS_BF16):
         self.shape = make_shape(batch=batch, q_len=q_len, max_kv_len=max_kv_len,
                                 num_q_heads=num_q_heads, num_kv_heads=num_kv_heads, top_k=top_k,
-                                kv_capacity=kv_capacity)
+                                kv_capacity=kv_capacity, num_index_heads=num_index_heads,
+                                index_key_format=index_key_format)
         n_idx = msa_index_topk_workspace_size(self.shape)
         n_att = msa_sparse_attention_workspace_size(self.shape)
         if n_idx == 0 or n_att == 0:
@@ -215,16 +235,21 @@ class MSA:
         self.device = torch.device(device)
         self.ws_index = alloc_workspace(n_idx, self.device)
         self.ws_attn = alloc_workspace(n_att, self.device)
-        sel = (batch, q_len, num_kv_heads, top_k)
+        sel = (batch, q_len, num_index_heads or num_kv_heads, top_k)
         self.block_ids = torch.empty(sel, dtype=torch.int32, device=self.device)
         self.block_scores = torch.empty(sel, dtype=torch.float32, device=self.device)
         self.out = torch.empty((batch, q_len, num_q_heads, 128), dtype=torch.bfloat16,
                                device=self.device)
         self.softmax_scale = 1.0 / math.sqrt(128)
 
-    def index_topk(self, q_idx, k_idx, lens, kv_offsets, stream=None):
-        msa_index_topk(self.shape, q_idx, k_idx, lens, kv_offsets, self.block_ids,
-                       self.block_scores, self.ws_index, stream)
+    def index_topk(self, q_idx, k_idx, lens, kv_offsets, stream=None, k_idx_scale=None):
+        """k_idx_scale given: FP8 index keys (msa_index_topk_fp8)."""
+        if k_idx_scale is not None:
+            msa_index_topk_fp8(self.shape, q_idx, k_idx, k_idx_scale, lens, kv_offsets,
+                               self.block_ids, self.block_scores, self.ws_index, stream)
+        else:
+            msa_index_topk(self.shape, q_idx, k_idx, lens, kv_offsets, self.block_ids,
+                           self.block_scores, self.ws_index, stream)
         return self.block_ids, self.block_scores
 
     def sparse_attention(self, q, k_cache, v_cache, lens, kv_offsets, block_ids=None, stream=None):

@@ -710,7 +710,7 @@ __global__ void __launch_bounds__(kBuildThreads) bucket_build_kernel(const Prefi
         const int i = i0 + static_cast<int>(e / P.K);
         const int slot = static_cast<int>(e % P.K);
         row = static_cast<long long>(b) * P.Sq + i;
-        const int j = ids[(row * P.H_kv + g) * P.K + slot];
+        const int j = ids[(row * P.n_idx + g / (P.H_kv / P.n_idx)) * P.K + slot];
         const long long p = static_cast<long long>(L) - P.Sq + i;
         return (j >= 0 && j < p / 128) ? j : -1;   // padding, own block, or out of range
     };
@@ -853,7 +853,7 @@ __global__ void fixup_kernel(const PrefillArgs P) {
             const __nv_bfloat16 *qh = qb + idx * kDim;
             float mx = -INFINITY;
             for (int s = 0; s < P.K; ++s) {
-                const int j = P.ids[pair * P.K + s];
+                const int j = P.ids[(row * P.n_idx + g / (P.H_kv / P.n_idx)) * P.K + s];
                 if (j < 0 || j >= p / 128) continue;
                 const long long row0 = kv_block_row(P.kv, b, j, P.status);
                 for (int t = lane; t < 128; t += 32) {

@@ -96,7 +96,8 @@ __global__ void __launch_bounds__(kThreads, kStages == 1 ? 3 : 1)
         }
         fence_mbar_init();
         S.abort_flag = 0;
-        const int32_t *ids = P.ids + pair * P.K;
+        // the group's index head: contiguous sets of H_kv / n_idx groups
+        const int32_t *ids = P.ids + (row * P.n_idx + g / (P.H_kv / P.n_idx)) * P.K;
         const int lo = split * bps, hi = lo + bps;
         int n = 0, bad = 0, nblk = 0;
         for (int q = 0; q < P.K; ++q) {

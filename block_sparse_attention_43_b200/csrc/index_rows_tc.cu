@@ -154,6 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const long long u = unit_index(r);
             if (u >= nunits) break;
             const Unit x = unit_at(P, u, ntiles);
+            const int kh = P.KH == 1 ? 0 : x.g;   // shared index keys: one row per token
             if (!x.valid) {
                 if (x.i0 == 0 && x.g == 0) set_status(P.status, kStatusBadLens);
                 continue;
@@ -178,8 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive_expect_tx(&S.k_full[s], nb * 32768);
                 for (int jj = 0; jj < nb; ++jj) {
                     const int tok = static_cast<int>(kv_block_row(P.kv, x.b, j + jj, P.status));
-                    tma_load_3d(S.ring[s] + jj * 16384, &tmK, 0, x.g, tok, &S.k_full[s]);
-                    tma_load_3d(S.ring[s] + 32768 + jj * 16384, &tmK, 64, x.g, tok, &S.k_full[s]);
+                    tma_load_3d(S.ring[s] + jj * 16384, &tmK, 0, kh, tok, &S.k_full[s]);
+                    tma_load_3d(S.ring[s] + 32768 + jj * 16384, &tmK, 64, kh, tok, &S.k_full[s]);
                 }
             }
         }
@@ -364,7 +365,7 @@ cudaError_t launch_index_rows_tc(const IndexRowsArgs &a, cudaStream_t s) {
     static_assert(sizeof(Smem<64>) + 1024 <= 227 * 1024, "shared memory budget");
     CUtensorMap tq, tk;
     if (!encode_kv_tensor_map(&tq, a.q_idx, a.H_kv, static_cast<long long>(a.B) * a.Sq) ||
-        !encode_kv_tensor_map(&tk, a.k_idx, a.H_kv, a.kv.capacity))
+        !encode_kv_tensor_map(&tk, a.k_idx, a.KH, a.kv.capacity))
         return cudaErrorInvalidValue;
     const long long ntiles = (a.Sq + 127) / 128;
     const long long units = ntiles * a.B * a.H_kv;

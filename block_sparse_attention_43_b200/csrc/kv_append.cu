@@ -7,7 +7,8 @@
 namespace msa {
 namespace {
 
-// One warp per (sequence, new token, tensor): H_kv x 256 contiguous bytes.
+// One warp per (sequence, new token, tensor): H x 256 contiguous bytes, H =
+// H_idx for the index keys, H_kv for the keys and values.
 __global__ void kv_append_kernel(const KvAppendArgs P) {
     const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
@@ -23,7 +24,7 @@ __global__ void kv_append_kernel(const KvAppendArgs P) {
         return;
     }
     const long long row = kv_block_row(P.kv, b, static_cast<int>(t / kBlock), P.status) + t % kBlock;
-    const int n16 = P.H_kv * kDim * 2 / 16;          // 16-byte chunks per token
+    const int n16 = (which == 0 ? P.H_idx : P.H_kv) * kDim * 2 / 16;   // 16-byte chunks per token
     const uint4 *src = static_cast<const uint4 *>(P.src[which]) + bt * n16;
     uint4 *dst = static_cast<uint4 *>(P.dst[which]) + row * n16;
     for (int c = lane; c < n16; c += 32) dst[c] = src[c];

@@ -84,6 +84,20 @@ bool pow2_le16(int x) { return x == 1 || x == 2 || x == 4 || x == 8 || x == 16; 
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// Index heads (0 in the shape: one per group), index-key rows per token, key dtype.
+int index_heads(const msa_shape_t *s) {
+    return s->num_index_heads > 0 ? s->num_index_heads : s->num_kv_heads;
+}
+int key_heads(const msa_shape_t *s) {
+    return (s->index_key_format == MSA_INDEX_KEYS_BF16_SHARED ||
+            s->index_key_format == MSA_INDEX_KEYS_FP8_SHARED)
+               ? 1
+               : index_heads(s);
+}
+bool key_fp8(const msa_shape_t *s) {
+    return s->index_key_format == MSA_INDEX_KEYS_FP8 || s->index_key_format == MSA_INDEX_KEYS_FP8_SHARED;
+}
+
 // Shape checks shared by both calls.
 msa_status_t check_shape(const msa_shape_t *s) {
     if (!s) return MSA_ERR_INVALID_ARG;
@@ -92,10 +106,14 @@ msa_status_t check_shape(const msa_shape_t *s) {
         s->index_dim < 1 || s->block_size < 1)
         return MSA_ERR_INVALID_ARG;
     if (s->num_q_heads % s->num_kv_heads) return MSA_ERR_INVALID_ARG;
+    if (s->num_index_heads < 0 || s->index_key_format < MSA_INDEX_KEYS_BF16 ||
+        s->index_key_format > MSA_INDEX_KEYS_FP8_SHARED)
+        return MSA_ERR_INVALID_ARG;
+    if (s->num_kv_heads % index_heads(s)) return MSA_ERR_INVALID_ARG;
     if (s->q_len > s->max_kv_len) return MSA_ERR_INVALID_ARG;
     if (s->head_dim != kDim || s->index_dim != kDim || s->block_size != kBlock)
         return MSA_ERR_UNSUPPORTED;
-    if (s->top_k > 64 || !pow2_le16(s->num_kv_heads) ||
+    if (s->top_k > 64 || !pow2_le16(s->num_kv_heads) || !pow2_le16(index_heads(s)) ||
         !pow2_le16(s->num_q_heads / s->num_kv_heads))
         return MSA_ERR_UNSUPPORTED;
     if (s->batch > 4096 || s->max_kv_len > (1 << 27) || s->kv_capacity >= (1LL << 31))
@@ -107,12 +125,12 @@ long long rows_of(const msa_shape_t *s) { return static_cast<long long>(s->batch
 
 int nb_max_of(const msa_shape_t *s) { return (s->max_kv_len + kBlock - 1) / kBlock; }
 
-// Decode keeps one fp32 score per (sequence, group, block) for the top-k
+// Decode keeps one fp32 score per (sequence, index head, block) for the top-k
 // pass; prefill selects inside the tensor-core kernel and needs only the header.
 size_t index_ws_bytes(const msa_shape_t *s) {
     if (s->q_len > 1) return kWsHeaderBytes;
     return kWsHeaderBytes +
-           round_up(static_cast<size_t>(rows_of(s)) * s->num_kv_heads * nb_max_of(s) * sizeof(float));
+           round_up(static_cast<size_t>(rows_of(s)) * index_heads(s) * nb_max_of(s) * sizeof(float));
 }
 
 // Prefill rows with groups of 8 heads run the block-outer tensor-core path;
@@ -183,11 +201,16 @@ msa_status_t check_paged(const msa_shape_t *s, const int32_t *page_table, int32_
 }
 
 msa_status_t index_topk_impl(const msa_shape_t *shape, const void *q_idx, const void *k_idx,
-                             const int32_t *lens, const KvMap &kv, int32_t *block_ids,
-                             float *block_scores, void *workspace, size_t workspace_bytes,
-                             msa_stream_t stream) {
+                             const float *k_scale, const int32_t *lens, const KvMap &kv,
+                             int32_t *block_ids, float *block_scores, void *workspace,
+                             size_t workspace_bytes, msa_stream_t stream) {
     if (!q_idx || !k_idx || !lens || !block_ids || !block_scores) return MSA_ERR_INVALID_ARG;
     if (!aligned16(q_idx) || !aligned16(k_idx)) return MSA_ERR_MISALIGNED;
+    const bool fp8 = key_fp8(shape);
+    if (fp8 && !k_scale) return MSA_ERR_INVALID_ARG;
+    if (fp8 && (reinterpret_cast<uintptr_t>(k_scale) & 3)) return MSA_ERR_MISALIGNED;
+    if (fp8 && shape->q_len > 1) return MSA_ERR_UNSUPPORTED;
+    const int hi = index_heads(shape), kh = key_heads(shape);
     msa_status_t st = check_ws(workspace, workspace_bytes, index_ws_bytes(shape));
     if (st != MSA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -201,20 +224,30 @@ msa_status_t index_topk_impl(const msa_shape_t *shape, const void *q_idx, const 
         IndexRowsArgs a;
         a.q_idx = q_idx; a.k_idx = k_idx; a.lens = lens; a.kv = kv;
         a.ids = block_ids; a.out_scores = block_scores; a.status = status;
-        a.B = shape->batch; a.Sq = shape->q_len; a.H_kv = shape->num_kv_heads; a.K = shape->top_k;
-        a.max_kv_len = shape->max_kv_len;
+        a.B = shape->batch; a.Sq = shape->q_len; a.H_kv = hi; a.K = shape->top_k;
+        a.max_kv_len = shape->max_kv_len; a.KH = kh;
         return launch_index_rows_tc(a, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
     }
-    IndexDecodeArgs a;
-    a.q_idx = q_idx; a.k_idx = k_idx; a.lens = lens; a.kv = kv;
-    a.scores = scores; a.status = status;
-    a.B = shape->batch; a.H_kv = shape->num_kv_heads; a.nb_max = nb_max;
-    a.max_kv_len = shape->max_kv_len;
-    if (launch_index_decode(a, s) != cudaSuccess) return MSA_ERR_CUDA;
+    if (!fp8 && kh == hi) {
+        // one bf16 key per index head
+        IndexDecodeArgs a;
+        a.q_idx = q_idx; a.k_idx = k_idx; a.lens = lens; a.kv = kv;
+        a.scores = scores; a.status = status;
+        a.B = shape->batch; a.H_kv = hi; a.nb_max = nb_max;
+        a.max_kv_len = shape->max_kv_len;
+        if (launch_index_decode(a, s) != cudaSuccess) return MSA_ERR_CUDA;
+    } else {
+        IndexDecodeVarArgs a;
+        a.q_idx = q_idx; a.k_idx = k_idx; a.k_scale = k_scale; a.lens = lens; a.kv = kv;
+        a.scores = scores; a.status = status;
+        a.B = shape->batch; a.H = hi; a.KH = kh; a.nb_max = nb_max;
+        a.max_kv_len = shape->max_kv_len; a.fp8 = fp8 ? 1 : 0;
+        if (launch_index_decode_variant(a, s) != cudaSuccess) return MSA_ERR_CUDA;
+    }
     TopkArgs t;
     t.scores = scores; t.lens = lens; t.kv = kv; t.ids = block_ids;
     t.out_scores = block_scores; t.status = status;
-    t.B = shape->batch; t.Sq = shape->q_len; t.H_kv = shape->num_kv_heads; t.nb_max = nb_max;
+    t.B = shape->batch; t.Sq = shape->q_len; t.H_kv = hi; t.nb_max = nb_max;
     t.K = shape->top_k; t.max_kv_len = shape->max_kv_len;
     if (launch_topk(t, s) != cudaSuccess) return MSA_ERR_CUDA;
     return MSA_OK;
@@ -243,6 +276,7 @@ msa_status_t sparse_attention_impl(const msa_shape_t *shape, const void *q, cons
         p.kv = kv; p.out = out; p.status = reinterpret_cast<int *>(ws);
         p.B = shape->batch; p.Sq = shape->q_len; p.H_q = shape->num_q_heads;
         p.H_kv = shape->num_kv_heads; p.K = shape->top_k; p.max_kv_len = shape->max_kv_len;
+        p.n_idx = index_heads(shape);
         p.softmax_scale = softmax_scale;
         return launch_prefill_attention(p, ws, L.pre, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
     }
@@ -255,6 +289,7 @@ msa_status_t sparse_attention_impl(const msa_shape_t *shape, const void *q, cons
     a.B = shape->batch; a.Sq = shape->q_len; a.H_q = shape->num_q_heads;
     a.H_kv = shape->num_kv_heads; a.K = shape->top_k; a.nsplit = L.nsplit;
     a.max_kv_len = shape->max_kv_len;
+    a.n_idx = index_heads(shape);
     a.softmax_scale = softmax_scale;
     if (launch_attn_rows(a, s) != cudaSuccess) return MSA_ERR_CUDA;
     return MSA_OK;
@@ -283,8 +318,22 @@ msa_status_t msa_index_topk(const msa_shape_t *shape, const void *q_idx, const v
     msa_status_t st = check_shape(shape);
     if (st != MSA_OK) return st;
     if (!kv_offsets) return MSA_ERR_INVALID_ARG;
-    return index_topk_impl(shape, q_idx, k_idx, lens, packed_map(shape, kv_offsets), block_ids,
-                           block_scores, workspace, workspace_bytes, stream);
+    if (key_fp8(shape)) return MSA_ERR_UNSUPPORTED;   // msa_index_topk_fp8
+    return index_topk_impl(shape, q_idx, k_idx, nullptr, lens, packed_map(shape, kv_offsets),
+                           block_ids, block_scores, workspace, workspace_bytes, stream);
+}
+
+msa_status_t msa_index_topk_fp8(const msa_shape_t *shape, const void *q_idx,
+                                const void *k_idx_fp8, const float *k_idx_scale,
+                                const int32_t *lens, const int64_t *kv_offsets,
+                                int32_t *block_ids, float *block_scores, void *workspace,
+                                size_t workspace_bytes, msa_stream_t stream) {
+    msa_status_t st = check_shape(shape);
+    if (st != MSA_OK) return st;
+    if (!kv_offsets || !key_fp8(shape)) return MSA_ERR_INVALID_ARG;
+    return index_topk_impl(shape, q_idx, k_idx_fp8, k_idx_scale, lens,
+                           packed_map(shape, kv_offsets), block_ids, block_scores, workspace,
+                           workspace_bytes, stream);
 }
 
 msa_status_t msa_index_topk_paged(const msa_shape_t *shape, const void *q_idx,
@@ -295,7 +344,8 @@ msa_status_t msa_index_topk_paged(const msa_shape_t *shape, const void *q_idx,
     msa_status_t st = check_shape(shape);
     if (st != MSA_OK) return st;
     if ((st = check_paged(shape, page_table, pages_per_seq)) != MSA_OK) return st;
-    return index_topk_impl(shape, q_idx, k_idx_pool, lens,
+    if (key_fp8(shape)) return MSA_ERR_UNSUPPORTED;
+    return index_topk_impl(shape, q_idx, k_idx_pool, nullptr, lens,
                            paged_map(shape, page_table, pages_per_seq), block_ids, block_scores,
                            workspace, workspace_bytes, stream);
 }
@@ -337,6 +387,7 @@ msa_status_t msa_kv_append(const msa_shape_t *shape, int32_t n_new, const void *
     if (n_new < 1 || !lens || !new_k_idx || !new_k || !new_v || !k_idx_cache || !k_cache ||
         !v_cache || (!kv_offsets) == (!page_table))
         return MSA_ERR_INVALID_ARG;
+    if (key_fp8(shape)) return MSA_ERR_UNSUPPORTED;
     if (page_table && (st = check_paged(shape, page_table, pages_per_seq)) != MSA_OK) return st;
     if (!aligned16(new_k_idx) || !aligned16(new_k) || !aligned16(new_v) ||
         !aligned16(k_idx_cache) || !aligned16(k_cache) || !aligned16(v_cache))
@@ -348,6 +399,7 @@ msa_status_t msa_kv_append(const msa_shape_t *shape, int32_t n_new, const void *
     a.kv = page_table ? paged_map(shape, page_table, pages_per_seq) : packed_map(shape, kv_offsets);
     a.status = device_status;
     a.B = shape->batch; a.n_new = n_new; a.H_kv = shape->num_kv_heads;
+    a.H_idx = key_heads(shape);
     a.max_kv_len = shape->max_kv_len;
     return launch_kv_append(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? MSA_OK
                                                                                      : MSA_ERR_CUDA;

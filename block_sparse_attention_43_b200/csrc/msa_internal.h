@@ -48,6 +48,22 @@ struct IndexDecodeArgs {
 };
 cudaError_t launch_index_decode(const IndexDecodeArgs &a, cudaStream_t s);
 
+// Decode index branch on the other index-key formats (index_decode_variants.cu):
+// keys shared by the H index heads ([T][1][128], bf16 or E4M3) or one E4M3 key
+// per index head ([T][H][128]); E4M3 rows carry an fp32 scale (k_scale [T][KH]).
+struct IndexDecodeVarArgs {
+    const void *q_idx;      // [B][H][128] bf16
+    const void *k_idx;      // [T][KH][128] bf16 or E4M3
+    const float *k_scale;   // [T][KH] (E4M3 only)
+    const int32_t *lens;
+    KvMap kv;
+    float *scores;          // [B][H][nb_max]
+    int *status;
+    int B, H, KH, nb_max, max_kv_len;
+    int fp8;
+};
+cudaError_t launch_index_decode_variant(const IndexDecodeVarArgs &a, cudaStream_t s);
+
 // Index branch for q_len >= 1 query rows per sequence (prefill), causal:
 // block max-pooled scores of every visible block and the top-k selection,
 // written straight to ids / out_scores [B*Sq][H_kv][K].
@@ -59,7 +75,8 @@ struct IndexRowsArgs {
     int32_t *ids;
     float *out_scores;
     int *status;
-    int B, Sq, H_kv, K, max_kv_len;
+    int B, Sq, H_kv, K, max_kv_len;   // H_kv here: index heads
+    int KH;                           // index-key rows per token: H_kv, or 1 (shared)
 };
 // tcgen05 tensor-core kernel (index_rows_tc.cu).
 cudaError_t launch_index_rows_tc(const IndexRowsArgs &a, cudaStream_t s);
@@ -89,6 +106,7 @@ struct AttnRowsArgs {
     int *tickets;           // [B*Sq][H_kv]
     int *status;
     int B, Sq, H_q, H_kv, K, nsplit, max_kv_len;
+    int n_idx;              // index heads: group g reads ids of g / (H_kv / n_idx)
     float softmax_scale;
 };
 cudaError_t launch_attn_rows(const AttnRowsArgs &a, cudaStream_t s);
@@ -110,6 +128,7 @@ struct PrefillArgs {
     void *out;
     int *status;
     int B, Sq, H_q, H_kv, K, max_kv_len;
+    int n_idx;              // index heads: group g reads ids of g / (H_kv / n_idx)
     float softmax_scale;
     // workspace views (filled by launch_prefill_attention)
     float *knorm;
@@ -150,6 +169,7 @@ struct KvAppendArgs {
     KvMap kv;
     int *status;
     int B, n_new, H_kv, max_kv_len;
+    int H_idx;              // index-key rows per token (src[0] / dst[0])
 };
 cudaError_t launch_kv_append(const KvAppendArgs &a, cudaStream_t s);
 

@@ -15,7 +15,7 @@
 namespace {
 
 // 256-byte header (device status word) + 4 MiB of block scores: enough for a
-// decode batch with batch * num_kv_heads * ceil(max_kv_len / 128) <= 1,048,576
+// decode batch with batch * index heads * ceil(max_kv_len / 128) <= 1,048,576
 // (e.g. 4 sequences x 8 groups at 1M tokens, or 64 x 8 at 256k).
 constexpr size_t kStaticScratchBytes = 256 + (size_t(4) << 20);
 

@@ -15,7 +15,8 @@
  * Block size 128, top-k 16 and index dimension 128 are the configuration the
  * mlqm.cn MiniMax-M3 guide prints ("sparse_block_size", "sparse_topk_blocks",
  * "sparse_index_dim").  The pages give no formula; this library fixes:
- *   - index score s[t] = dot(q_idx[b,i,g,:], k_idx[t,g,:]), no scale;
+ *   - index score s[t] = dot(q_idx[b,i,g,:], k_idx[t,g,:]), no scale, for
+ *     index head g (one per GQA group unless num_index_heads says fewer);
  *   - block score S[j] = max of s[t] over the tokens t of block j with
  *     t <= p, where p = lens[b] - q_len + i is the query's position;
  *   - the query's own block floor(p/128) is always kept; the other k-1 slots
@@ -24,12 +25,22 @@
  *   - sparse branch: softmax(softmax_scale * q.k) over the keys t <= p of the
  *     kept blocks, applied to v; head h belongs to group h / (H_q / H_kv).
  *
+ * Index-branch variants.  The guide's configuration also prints
+ * "sparse_num_index_heads: 4", which one index query per group cannot match;
+ * the pages say nothing more, so this library reads it as Hi index heads that
+ * partition the groups into contiguous sets: group g uses index head
+ * g / (H_kv / Hi) (Hi = H_kv is the default, one per group).  Index keys may
+ * be one row per (token, index head) or one row per token shared by every
+ * index head, in bf16 or in FP8 E4M3 with one fp32 scale per key row (score
+ * = scale * dot(q_idx, decoded key)); see index_key_format.
+ *
  * Layouts (all row-major, head dim innermost, bf16 = IEEE bfloat16 bits):
- *   q_idx  [B, q_len, H_kv, index_dim]     q   [B, q_len, H_q, head_dim]
- *   k_idx, k_cache, v_cache: packed [kv_capacity, H_kv, dim]; sequence b
- *          owns rows kv_offsets[b] .. kv_offsets[b] + lens[b] - 1 (a padded
- *          cache is the case kv_offsets[b] = b * stride).
- *   block_ids [B, q_len, H_kv, top_k] int32, ascending, -1 padded
+ *   q_idx  [B, q_len, Hi, index_dim]       q   [B, q_len, H_q, head_dim]
+ *   k_cache, v_cache: packed [kv_capacity, H_kv, dim]; k_idx: packed
+ *          [kv_capacity, KH, index_dim] with KH = Hi, or 1 for shared index
+ *          keys; sequence b owns rows kv_offsets[b] .. kv_offsets[b] +
+ *          lens[b] - 1 (a padded cache is the case kv_offsets[b] = b * stride).
+ *   block_ids [B, q_len, Hi, top_k] int32, ascending, -1 padded
  *   block_scores: same shape, float32, -inf padded
  *   out    [B, q_len, H_q, head_dim] bf16 (round to nearest even)
  *
@@ -80,39 +91,66 @@ typedef enum {
     MSA_ERR_MISALIGNED = 7      /* a tensor pointer is not 16-byte aligned */
 } msa_status_t;
 
+/* Layout of the index keys (msa_shape_t.index_key_format). */
+typedef enum {
+    MSA_INDEX_KEYS_BF16 = 0,        /* bf16 [kv_capacity, Hi, index_dim]: one key per index head */
+    MSA_INDEX_KEYS_BF16_SHARED = 1, /* bf16 [kv_capacity, 1, index_dim]: one key per token */
+    MSA_INDEX_KEYS_FP8 = 2,         /* E4M3 [kv_capacity, Hi, index_dim] + fp32 scale [kv_capacity, Hi] */
+    MSA_INDEX_KEYS_FP8_SHARED = 3   /* E4M3 [kv_capacity, 1, index_dim] + fp32 scale [kv_capacity, 1] */
+} msa_index_key_format_t;
+
 /* Problem shape.  Supported by this build: head_dim == index_dim == 128,
  * block_size == 128, 1 <= top_k <= 64, num_kv_heads in {1, 2, 4, 8, 16},
- * num_q_heads / num_kv_heads in {1, 2, 4, 8, 16}, batch <= 4096,
- * max_kv_len <= 2^27, kv_capacity < 2^31. */
+ * num_q_heads / num_kv_heads in {1, 2, 4, 8, 16}, index heads in {1, 2, 4,
+ * 8, 16} dividing num_kv_heads, batch <= 4096, max_kv_len <= 2^27,
+ * kv_capacity < 2^31.  FP8 index keys: decode (q_len == 1) only. */
 typedef struct {
     int32_t batch;        /* B */
     int32_t q_len;        /* query rows per sequence: 1 = decode, lens[b] = full prefill */
     int32_t max_kv_len;   /* upper bound on every lens[b] */
     int32_t num_q_heads;  /* H_q */
-    int32_t num_kv_heads; /* H_kv = number of GQA groups = number of index queries */
+    int32_t num_kv_heads; /* H_kv = number of GQA groups */
     int32_t head_dim;     /* D */
     int32_t index_dim;    /* d_idx */
     int32_t block_size;   /* tokens per KV block */
-    int32_t top_k;        /* blocks kept per (query row, group), own block included */
+    int32_t top_k;        /* blocks kept per (query row, index head), own block included */
     int64_t kv_capacity;  /* rows in the packed k_idx / k_cache / v_cache */
+    int32_t num_index_heads;  /* Hi; 0 means num_kv_heads (one index head per group) */
+    int32_t index_key_format; /* msa_index_key_format_t; 0 = bf16, one key per index head */
 } msa_shape_t;
 
 /* Bytes of workspace msa_index_topk needs for this shape (0 on bad shape). */
 MSA_API size_t msa_index_topk_workspace_size(const msa_shape_t *shape);
 
 /* Index branch: block max-pooled index scores and the top-k block ids of
- * every (query row, group).  See the header comment for the definition.
- *   q_idx        device bf16 [B, q_len, H_kv, index_dim]
- *   k_idx        device bf16 [kv_capacity, H_kv, index_dim]
+ * every (query row, index head).  See the header comment for the definition.
+ *   q_idx        device bf16 [B, q_len, Hi, index_dim]
+ *   k_idx        device bf16 [kv_capacity, KH, index_dim] (KH = Hi, or 1 for
+ *                MSA_INDEX_KEYS_BF16_SHARED; the FP8 formats take
+ *                msa_index_topk_fp8 and return MSA_ERR_UNSUPPORTED here)
  *   lens         device int32 [B], each in [q_len, max_kv_len]
  *   kv_offsets   device int64 [B], row of token 0 of sequence b
- *   block_ids    device int32 [B, q_len, H_kv, top_k]   (written)
- *   block_scores device float [B, q_len, H_kv, top_k]   (written)
+ *   block_ids    device int32 [B, q_len, Hi, top_k]   (written)
+ *   block_scores device float [B, q_len, Hi, top_k]   (written)
  *   workspace    device, >= msa_index_topk_workspace_size(shape) bytes */
 MSA_API msa_status_t msa_index_topk(const msa_shape_t *shape, const void *q_idx, const void *k_idx,
                             const int32_t *lens, const int64_t *kv_offsets,
                             int32_t *block_ids, float *block_scores,
                             void *workspace, size_t workspace_bytes, msa_stream_t stream);
+
+/* Index branch on FP8 E4M3 index keys (index_key_format MSA_INDEX_KEYS_FP8
+ * or MSA_INDEX_KEYS_FP8_SHARED), decode only (q_len == 1): the score of
+ * token t for index head g is k_idx_scale[t, kh] * dot(q_idx[b,0,g,:],
+ * decoded k_idx_fp8[t, kh, :]), kh = g (or 0 when shared), accumulated in
+ * fp32.  E4M3 is the OCP 8-bit format with bias 7 and no infinities.
+ *   k_idx_fp8    device uint8 [kv_capacity, KH, index_dim] (E4M3 codes)
+ *   k_idx_scale  device float [kv_capacity, KH]
+ * Other arguments, layouts, results and errors are those of msa_index_topk. */
+MSA_API msa_status_t msa_index_topk_fp8(const msa_shape_t *shape, const void *q_idx,
+                                        const void *k_idx_fp8, const float *k_idx_scale,
+                                        const int32_t *lens, const int64_t *kv_offsets,
+                                        int32_t *block_ids, float *block_scores, void *workspace,
+                                        size_t workspace_bytes, msa_stream_t stream);
 
 /* Bytes of workspace msa_sparse_attention needs for this shape (0 on bad shape). */
 MSA_API size_t msa_sparse_attention_workspace_size(const msa_shape_t *shape);
@@ -120,10 +158,11 @@ MSA_API size_t msa_sparse_attention_workspace_size(const msa_shape_t *shape);
 /* Sparse branch: exact softmax attention of every query head over the keys
  * of its group's kept blocks (ids as written by msa_index_topk; -1 entries
  * are skipped; every id must be a visible block, the own block included).
+ * Group g takes the ids of index head g / (H_kv / Hi).
  *   q            device bf16 [B, q_len, H_q, head_dim]
  *   k_cache      device bf16 [kv_capacity, H_kv, head_dim]
  *   v_cache      device bf16 [kv_capacity, H_kv, head_dim]
- *   block_ids    device int32 [B, q_len, H_kv, top_k]
+ *   block_ids    device int32 [B, q_len, Hi, top_k]
  *   softmax_scale  multiplies q.k before the softmax (1/sqrt(head_dim) usual)
  *   out          device bf16 [B, q_len, H_q, head_dim]  (written)
  *   workspace    device, >= msa_sparse_attention_workspace_size(shape) bytes */
@@ -157,8 +196,10 @@ MSA_API msa_status_t msa_sparse_attention_paged(const msa_shape_t *shape, const 
                                                 float softmax_scale, void *out, void *workspace,
                                                 size_t workspace_bytes, msa_stream_t stream);
 
-/* Appends n_new tokens to every sequence: new_k_idx, new_k, new_v are device
- * bf16 [B, n_new, H_kv, 128]; token i of sequence b is written at position
+/* Appends n_new tokens to every sequence: new_k, new_v are device bf16
+ * [B, n_new, H_kv, 128], new_k_idx device bf16 [B, n_new, KH, 128] (bf16
+ * index-key formats only; the FP8 formats return MSA_ERR_UNSUPPORTED); token
+ * i of sequence b is written at position
  * lens[b] + i of the packed (kv_offsets) or paged (page_table, pages_per_seq)
  * caches -- pass exactly one of kv_offsets / page_table.  lens is not
  * changed; the caller advances it.  A token that would land at or past
@@ -178,7 +219,7 @@ MSA_API msa_status_t msa_kv_append(const msa_shape_t *shape, int32_t n_new, cons
  * has no counterpart; this is a library convenience.
  *   Scratch: a file-scope device array of 256 B + 4 MiB that every GPU which
  *   loads the library holds until the process exits.  Shapes whose
- *   msa_index_topk_workspace_size exceeds that (batch * q_len * num_kv_heads
+ *   msa_index_topk_workspace_size exceeds that (batch * q_len * index heads
  *   * ceil(max_kv_len / 128) > 1,048,576 block scores) are rejected with
  *   MSA_ERR_WORKSPACE; nothing is launched and nothing is allocated.
  *   Set-up: the first call on each device looks up the array's device

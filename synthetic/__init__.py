@@ -5,4 +5,4 @@ both the CUDA library's tests/benchmark and the CPU oracle consume the bytes it
 produces (the oracle after a device-to-host copy).
 """
 from .inputs import (WORKLOADS, Workload, bf16_bits, make_inputs, make_workload,  # noqa: F401
-                     ragged_lens)
+                     quantize_e4m3_rows, ragged_lens)

@@ -159,3 +159,15 @@ def make_workload(name: str, device) -> Workload:
 def bf16_bits(t: torch.Tensor):
     """bf16 tensor -> numpy uint16 view of its bits (host copy)."""
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view("uint16")
+
+
+def quantize_e4m3_rows(x):
+    """FP8 E4M3 codes of x with one fp32 scale per row of the last dim: scale =
+    max|x| / 448 (the largest E4M3 magnitude), codes = x / scale rounded by
+    torch's E4M3 cast.  Returns (uint8 codes shaped like x, float32 scales
+    shaped like x without its last dim).  Input preparation only."""
+    xf = x.float()
+    amax = xf.abs().amax(dim=-1)
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    codes = (xf / scale.unsqueeze(-1)).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.contiguous(), scale.contiguous()

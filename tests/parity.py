@@ -47,11 +47,13 @@ def compare_index(oracle_mod, w, gpu_ids, gpu_scores, rows=None, host=None):
     the oracle's index branch.  Returns (rows, gpu ids of those rows, report)."""
     a = host if host is not None else host_inputs(w)
     R = w.B * w.Sq
+    H = a["q_idx"].shape[2]                    # index heads (k_idx may be shared or E4M3)
     rows_a = np.arange(R, dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
     ref = oracle_mod.index_topk(a["q_idx"], a["k_idx"], a["lens"], a["kv_offsets"],
-                                block=w.block, top_k=w.top_k, rows=rows_a)
-    g_ids = gpu_ids.reshape(R, w.H_kv, w.top_k)[rows_a]
-    g_sc = gpu_scores.reshape(R, w.H_kv, w.top_k)[rows_a]
+                                block=w.block, top_k=w.top_k, rows=rows_a,
+                                k_scale=a.get("k_scale"))
+    g_ids = gpu_ids.reshape(R, H, w.top_k)[rows_a]
+    g_sc = gpu_scores.reshape(R, H, w.top_k)[rows_a]
     o_ids, o_sc, bnd = ref["block_ids"], ref["block_scores"], ref["boundary"]
 
     same = (g_ids == o_ids).all(axis=-1)
@@ -85,10 +87,12 @@ def compare(oracle_mod, w, gpu_ids, gpu_scores, gpu_out, rows=None, host=None):
 
     # Outputs: oracle attention on the GPU's own selection (identical to the
     # oracle's except at near ties).
-    full_ids = np.full((R, w.H_kv, w.top_k), -1, np.int32)
+    H = a["q_idx"].shape[2]
+    full_ids = np.full((R, H, w.top_k), -1, np.int32)
     full_ids[rows_a] = g_ids
     o_out = oracle_mod.sparse_attention(a["q"], a["k"], a["v"], full_ids, a["lens"],
-                                        a["kv_offsets"], block=w.block, scale=w.scale, rows=rows_a)
+                                        a["kv_offsets"], block=w.block, scale=w.scale, rows=rows_a,
+                                        num_index_heads=H)
     g_out = gpu_out.reshape(R, w.H_q, w.D)[rows_a].astype(np.float64)
     assert np.isfinite(g_out).all(), "non-finite output"
     d = np.abs(g_out - o_out)

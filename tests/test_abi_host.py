@@ -108,3 +108,27 @@ def test_paged_and_append_arguments_are_checked(m):
                                P(0x50000), 8192, *caches, None, None) == 1
     assert m.lib.msa_kv_append(ctypes.byref(s), 0, *ptrs[:3], P(0x30000), P(0x40000), None, 0,
                                *caches, None, None) == 1
+
+
+def test_index_variant_shapes_are_checked(m):
+    P = ctypes.c_void_p
+    nb = (1 << 20) // 128
+    # 4 index heads for 8 groups: block scores per index head
+    assert m.msa_index_topk_workspace_size(_shape(m, num_index_heads=4)) == 256 + 4 * 4 * nb * 4
+    assert m.msa_index_topk_workspace_size(_shape(m, num_index_heads=3)) == 0     # does not divide 8
+    assert m.msa_index_topk_workspace_size(_shape(m, num_index_heads=16)) == 0    # more heads than groups
+    assert m.msa_index_topk_workspace_size(_shape(m, index_key_format=4)) == 0
+    assert m.msa_sparse_attention_workspace_size(_shape(m, num_index_heads=2)) > 256
+    good = [0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 0x60000]
+    # E4M3 formats go through msa_index_topk_fp8, bf16 formats through msa_index_topk
+    assert _call_index(m, _shape(m, index_key_format=m.INDEX_KEYS_FP8), good) == 2
+    s = _shape(m, index_key_format=m.INDEX_KEYS_BF16_SHARED)
+    args = [P(x) for x in (0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 0x60000, 0x70000)]
+    assert m.lib.msa_index_topk_fp8(ctypes.byref(s), *args, P(0x100000), 1 << 40, None) == 1
+    s8 = _shape(m, index_key_format=m.INDEX_KEYS_FP8_SHARED)
+    assert m.lib.msa_index_topk_fp8(ctypes.byref(s8), P(0x10000), P(0x20000), None,
+                                    *args[3:], P(0x100000), 1 << 40, None) == 1  # no scales
+    assert m.lib.msa_index_topk_fp8(ctypes.byref(s8), P(0x10000), P(0x20000), P(0x30002),
+                                    *args[3:], P(0x100000), 1 << 40, None) == 7  # misaligned scales
+    s8p = _shape(m, q_len=64, index_key_format=m.INDEX_KEYS_FP8)
+    assert m.lib.msa_index_topk_fp8(ctypes.byref(s8p), *args, P(0x100000), 1 << 40, None) == 2
