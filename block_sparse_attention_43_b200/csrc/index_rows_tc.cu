@@ -109,7 +109,32 @@ __device__ __forceinline__ float key_score(unsigned long long key) {
     return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
 }
 
-template <int LIST>
+// E4M3 -> bf16, 16 codes per thread-step (every E4M3 value is a bf16 value).
+__global__ void widen_e4m3_kernel(const uint4 *src, uint4 *dst, long long n16) {
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const uint4 w = src[i];
+        const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+        uint32_t o[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t f16;
+                const uint16_t pair = static_cast<uint16_t>(in[q] >> (16 * h));
+                asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(f16) : "h"(pair));
+                float lo, hi;
+                asm("{\n\t.reg .f16 l, u;\n\tmov.b32 {l, u}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, u;\n\t}"
+                    : "=f"(lo), "=f"(hi) : "r"(f16));
+                o[2 * q + h] = pack_bf16x2(lo, hi);
+            }
+        }
+        dst[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+}
+
+template <int LIST, bool SCALED>
 __global__ void __launch_bounds__(kThreads, 1)
     index_rows_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK, const IndexRowsArgs P) {
@@ -279,6 +304,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const long long t0 = static_cast<long long>(J) * kBlock;
                         const bool full = t0 + kBlock - 1 <= x.p_first;   // no masking for any row
                         float m = -INFINITY;
+                        if (SCALED) {
+                            // E4M3 keys (widened exactly to bf16 for the MMA): each
+                            // token's score is its row scale times the dot.
+                            const long long krow = kv_block_row(P.kv, x.b, J, P.status);
+                            const float *sc = P.k_scale + krow * P.KH + (P.KH == 1 ? 0 : x.g);
+#pragma unroll
+                            for (int c = 0; c < 4; c += 2) {
+                                uint32_t va[32], vb[32];
+                                tmem_ld32r(lane_addr + a * 256 + jj * 128 + c * 32, va);
+                                tmem_ld32r(lane_addr + a * 256 + jj * 128 + c * 32 + 32, vb);
+                                tmem_wait_ld(va);
+                                tmem_tie(vb);
+#pragma unroll
+                                for (int e = 0; e < 32; ++e) {
+                                    const int c0 = c * 32 + e, c1 = c0 + 32;
+                                    if (t0 + c0 <= p) m = fmaxf(m, __uint_as_float(va[e]) * __ldg(sc + c0 * P.KH));
+                                    if (t0 + c1 <= p) m = fmaxf(m, __uint_as_float(vb[e]) * __ldg(sc + c1 * P.KH));
+                                }
+                            }
+                        } else
 #pragma unroll
                         for (int c = 0; c < 4; c += 2) {
                             uint32_t va[32], vb[32];
@@ -361,6 +406,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+cudaError_t launch_widen_e4m3(const void *src, void *dst, long long rows, cudaStream_t s) {
+    const long long n16 = rows * (kDim / 16);
+    TraceScope trace(s, "index_widen_e4m3");
+    widen_e4m3_kernel<<<device_sm_count() * 8, 256, 0, s>>>(static_cast<const uint4 *>(src),
+                                                            static_cast<uint4 *>(dst), n16);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_index_rows_tc(const IndexRowsArgs &a, cudaStream_t s) {
     static_assert(sizeof(Smem<64>) + 1024 <= 227 * 1024, "shared memory budget");
     CUtensorMap tq, tk;
@@ -378,9 +431,16 @@ cudaError_t launch_index_rows_tc(const IndexRowsArgs &a, cudaStream_t s) {
         kern<<<static_cast<unsigned>(grid), kThreads, smem, s>>>(tq, tk, a);
         return cudaGetLastError();
     };
-    if (a.K <= 16) return go(index_rows_tc_kernel<16>, sizeof(Smem<16>) + 1024);
-    if (a.K <= 32) return go(index_rows_tc_kernel<32>, sizeof(Smem<32>) + 1024);
-    if (a.K <= 64) return go(index_rows_tc_kernel<64>, sizeof(Smem<64>) + 1024);
+    // E4M3 keys (row scales on the scores) get their own instantiation so the
+    // bf16 kernels keep their register allocation.
+    if (a.k_scale) {
+        if (a.K <= 16) return go(index_rows_tc_kernel<16, true>, sizeof(Smem<16>) + 1024);
+        if (a.K <= 32) return go(index_rows_tc_kernel<32, true>, sizeof(Smem<32>) + 1024);
+        if (a.K <= 64) return go(index_rows_tc_kernel<64, true>, sizeof(Smem<64>) + 1024);
+    }
+    if (a.K <= 16) return go(index_rows_tc_kernel<16, false>, sizeof(Smem<16>) + 1024);
+    if (a.K <= 32) return go(index_rows_tc_kernel<32, false>, sizeof(Smem<32>) + 1024);
+    if (a.K <= 64) return go(index_rows_tc_kernel<64, false>, sizeof(Smem<64>) + 1024);
     return cudaErrorInvalidValue;
 }
 

@@ -126,9 +126,13 @@ long long rows_of(const msa_shape_t *s) { return static_cast<long long>(s->batch
 int nb_max_of(const msa_shape_t *s) { return (s->max_kv_len + kBlock - 1) / kBlock; }
 
 // Decode keeps one fp32 score per (sequence, index head, block) for the top-k
-// pass; prefill selects inside the tensor-core kernel and needs only the header.
+// pass; prefill selects inside the tensor-core kernel and needs only the
+// header, plus a bf16 copy of E4M3 index keys for the MMA.
 size_t index_ws_bytes(const msa_shape_t *s) {
-    if (s->q_len > 1) return kWsHeaderBytes;
+    if (s->q_len > 1)
+        return kWsHeaderBytes + (key_fp8(s) ? round_up(static_cast<size_t>(s->kv_capacity) *
+                                                       key_heads(s) * kDim * 2)
+                                            : 0);
     return kWsHeaderBytes +
            round_up(static_cast<size_t>(rows_of(s)) * index_heads(s) * nb_max_of(s) * sizeof(float));
 }
@@ -209,7 +213,6 @@ msa_status_t index_topk_impl(const msa_shape_t *shape, const void *q_idx, const 
     const bool fp8 = key_fp8(shape);
     if (fp8 && !k_scale) return MSA_ERR_INVALID_ARG;
     if (fp8 && (reinterpret_cast<uintptr_t>(k_scale) & 3)) return MSA_ERR_MISALIGNED;
-    if (fp8 && shape->q_len > 1) return MSA_ERR_UNSUPPORTED;
     const int hi = index_heads(shape), kh = key_heads(shape);
     msa_status_t st = check_ws(workspace, workspace_bytes, index_ws_bytes(shape));
     if (st != MSA_OK) return st;
@@ -222,7 +225,17 @@ msa_status_t index_topk_impl(const msa_shape_t *shape, const void *q_idx, const 
     if (cudaMemsetAsync(ws, 0, kWsHeaderBytes, s) != cudaSuccess) return MSA_ERR_CUDA;
     if (shape->q_len > 1) {
         IndexRowsArgs a;
-        a.q_idx = q_idx; a.k_idx = k_idx; a.lens = lens; a.kv = kv;
+        a.q_idx = q_idx; a.k_idx = k_idx; a.lens = lens; a.kv = kv; a.k_scale = nullptr;
+        if (fp8) {
+            // E4M3 keys widened exactly to bf16 in the workspace; the kernel
+            // applies the row scales to the scores.
+            void *wide = ws + kWsHeaderBytes;
+            if (launch_widen_e4m3(k_idx, wide, static_cast<long long>(shape->kv_capacity) * kh, s) !=
+                cudaSuccess)
+                return MSA_ERR_CUDA;
+            a.k_idx = wide;
+            a.k_scale = k_scale;
+        }
         a.ids = block_ids; a.out_scores = block_scores; a.status = status;
         a.B = shape->batch; a.Sq = shape->q_len; a.H_kv = hi; a.K = shape->top_k;
         a.max_kv_len = shape->max_kv_len; a.KH = kh;

@@ -77,7 +77,10 @@ struct IndexRowsArgs {
     int *status;
     int B, Sq, H_kv, K, max_kv_len;   // H_kv here: index heads
     int KH;                           // index-key rows per token: H_kv, or 1 (shared)
+    const float *k_scale;             // E4M3 keys (widened to bf16 in k_idx): row scales [T][KH]
 };
+// E4M3 codes [rows][128] -> bf16 [rows][128], exact (index_rows_tc.cu).
+cudaError_t launch_widen_e4m3(const void *src, void *dst, long long rows, cudaStream_t s);
 // tcgen05 tensor-core kernel (index_rows_tc.cu).
 cudaError_t launch_index_rows_tc(const IndexRowsArgs &a, cudaStream_t s);
 

@@ -103,7 +103,7 @@ typedef enum {
  * block_size == 128, 1 <= top_k <= 64, num_kv_heads in {1, 2, 4, 8, 16},
  * num_q_heads / num_kv_heads in {1, 2, 4, 8, 16}, index heads in {1, 2, 4,
  * 8, 16} dividing num_kv_heads, batch <= 4096, max_kv_len <= 2^27,
- * kv_capacity < 2^31.  FP8 index keys: decode (q_len == 1) only. */
+ * kv_capacity < 2^31. */
 typedef struct {
     int32_t batch;        /* B */
     int32_t q_len;        /* query rows per sequence: 1 = decode, lens[b] = full prefill */
@@ -139,10 +139,12 @@ MSA_API msa_status_t msa_index_topk(const msa_shape_t *shape, const void *q_idx,
                             void *workspace, size_t workspace_bytes, msa_stream_t stream);
 
 /* Index branch on FP8 E4M3 index keys (index_key_format MSA_INDEX_KEYS_FP8
- * or MSA_INDEX_KEYS_FP8_SHARED), decode only (q_len == 1): the score of
- * token t for index head g is k_idx_scale[t, kh] * dot(q_idx[b,0,g,:],
- * decoded k_idx_fp8[t, kh, :]), kh = g (or 0 when shared), accumulated in
- * fp32.  E4M3 is the OCP 8-bit format with bias 7 and no infinities.
+ * or MSA_INDEX_KEYS_FP8_SHARED): the score of token t for index head g is
+ * k_idx_scale[t, kh] * dot(q_idx[b,i,g,:], decoded k_idx_fp8[t, kh, :]),
+ * kh = g (or 0 when shared), accumulated in fp32.  E4M3 is the OCP 8-bit
+ * format with bias 7 and no infinities.  For q_len > 1 the workspace also
+ * holds an exact bf16 copy of all kv_capacity key rows (see
+ * msa_index_topk_workspace_size).
  *   k_idx_fp8    device uint8 [kv_capacity, KH, index_dim] (E4M3 codes)
  *   k_idx_scale  device float [kv_capacity, KH]
  * Other arguments, layouts, results and errors are those of msa_index_topk. */

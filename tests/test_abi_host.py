@@ -130,5 +130,9 @@ def test_index_variant_shapes_are_checked(m):
                                     *args[3:], P(0x100000), 1 << 40, None) == 1  # no scales
     assert m.lib.msa_index_topk_fp8(ctypes.byref(s8), P(0x10000), P(0x20000), P(0x30002),
                                     *args[3:], P(0x100000), 1 << 40, None) == 7  # misaligned scales
-    s8p = _shape(m, q_len=64, index_key_format=m.INDEX_KEYS_FP8)
-    assert m.lib.msa_index_topk_fp8(ctypes.byref(s8p), *args, P(0x100000), 1 << 40, None) == 2
+    # prefill on E4M3 keys: the workspace also holds a bf16 copy of every key row
+    cap = 4 << 20
+    assert m.msa_index_topk_workspace_size(_shape(m, q_len=64, index_key_format=m.INDEX_KEYS_FP8)) \
+        == 256 + cap * 8 * 128 * 2
+    assert m.msa_index_topk_workspace_size(
+        _shape(m, q_len=64, index_key_format=m.INDEX_KEYS_FP8_SHARED)) == 256 + cap * 128 * 2

@@ -1,6 +1,6 @@
 """GPU parity of the index-branch variants through the C ABI: fewer index
 heads than groups, index keys shared by every index head, and FP8 E4M3 index
-keys with per-row scales (decode), each against the CPU oracle on the same
+keys with per-row scales, in decode and prefill, each against the CPU oracle on the same
 bytes with the tolerances of tests/parity.py.  The sparse branch runs on the
 variant's selection (group g uses index head g / (H_kv / Hi))."""
 import numpy as np
@@ -80,14 +80,15 @@ def test_decode_variants(oracle_mod, fmt, B, lens, H_q, H_kv, Hi, top_k):
 
 
 PREFILL = [
-    # (B, Sq, lens, H_q, H_kv, Hi, top_k): tensor-core index path (bf16 keys)
+    # (B, Sq, lens, H_q, H_kv, Hi, top_k): tensor-core index path (E4M3 keys
+    # widened to bf16 in the workspace, row scales applied to the scores)
     (1, 1000, [1000], 64, 8, 4, 16),        # block-outer attention path (groups of 8)
     (2, 300, [700, 300], 16, 4, 1, 4),      # row attention path, one index head
     (1, 2000, [2000], 64, 8, 8, 8),
 ]
 
 
-@pytest.mark.parametrize("fmt", ["bf16", "bf16_shared"])
+@pytest.mark.parametrize("fmt", list(FORMATS))
 @pytest.mark.parametrize("B,Sq,lens,H_q,H_kv,Hi,top_k", PREFILL)
 def test_prefill_variants(oracle_mod, fmt, B, Sq, lens, H_q, H_kv, Hi, top_k):
     from synthetic import make_inputs
@@ -95,13 +96,3 @@ def test_prefill_variants(oracle_mod, fmt, B, Sq, lens, H_q, H_kv, Hi, top_k):
                     device=DEV)
     rep = _run(w, Hi, FORMATS[fmt], 2)
     print(fmt, (B, Sq, H_kv, Hi), rep)
-
-
-def test_fp8_keys_in_prefill_are_refused():
-    shape = m.make_shape(batch=1, q_len=64, max_kv_len=64, num_q_heads=8, num_kv_heads=8,
-                         top_k=4, kv_capacity=64, index_key_format=m.INDEX_KEYS_FP8)
-    ws = m.alloc_workspace(m.msa_index_topk_workspace_size(shape), DEV)
-    t = torch.zeros(1 << 16, dtype=torch.uint8, device=DEV)
-    with pytest.raises(m.MSAError) as e:
-        m.msa_index_topk_fp8(shape, t, t, t, t, t, t, t, ws)
-    assert e.value.code == 2
