@@ -7,7 +7,8 @@ blocks, top-k with the own block kept and ties to the lower id; sparse branch:
 exact softmax attention over the kept blocks, shared by the group's heads).
 Index-branch variants: fewer index heads than groups (contiguous sets of
 groups share one index head's selection), index keys shared by every index
-head, and FP8 E4M3 index keys with one fp32 scale per key row.
+head, and FP8 E4M3 index keys with one fp32 scale per key row.  The sparse
+branch's backward (dQ, dK, dV over the kept keys) is here too.
 The sources are the cloud.tencent.com MSA article, sections 二 and 六, and the
 mlqm.cn guide's configuration-file passage.
 
@@ -58,6 +59,9 @@ def _load():
         lib.oracle_sparse_attention_ex.argtypes = [I, I, I, I, I, I, I, I, P, P, P, P, P, P, L,
                                                    ctypes.c_double, P, L, P, P, I]
         lib.oracle_sparse_attention_ex.restype = I
+        lib.oracle_sparse_attention_backward.argtypes = [I, I, I, I, I, I, I, I, P, P, P, P, P, P,
+                                                         P, L, ctypes.c_double, P, P, P, I]
+        lib.oracle_sparse_attention_backward.restype = I
         lib.oracle_e4m3_to_double.argtypes = [I]
         lib.oracle_e4m3_to_double.restype = ctypes.c_double
         _lib = lib
@@ -158,3 +162,35 @@ def sparse_attention(q, k, v, block_ids, lens, kv_offsets, *, block=128, scale=N
     if rc != 0:
         raise ValueError(f"oracle_sparse_attention rejected its input (code {rc})")
     return (out, ws) if want_wsum else out
+
+
+def sparse_attention_backward(q, k, v, dout, block_ids, lens, kv_offsets, *, block=128,
+                              scale=None, num_index_heads=None, n_threads=None):
+    """Backward of the sparse branch.  Shapes as sparse_attention, plus dout
+    [B,Sq,H_q,D] (uint16 bf16 bits).  Returns (dq [B*Sq,H_q,D], dk [T,H_kv,D],
+    dv [T,H_kv,D]), float64; dk/dv are zero on keys no row kept."""
+    q = _c(q, np.uint16)
+    k = _c(k, np.uint16)
+    v = _c(v, np.uint16)
+    dout = _c(dout, np.uint16)
+    lens = _c(lens, np.int32)
+    kv_offsets = _c(kv_offsets, np.int64)
+    B, Sq, H_q, D = q.shape
+    T, H_kv, _ = k.shape
+    assert dout.shape == q.shape
+    n_idx = H_kv if num_index_heads is None else int(num_index_heads)
+    ids = _c(block_ids, np.int32).reshape(B * Sq, n_idx, -1)
+    top_k = ids.shape[-1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    dq = np.empty((B * Sq, H_q, D), np.float64)
+    dk = np.zeros((T, H_kv, D), np.float64)
+    dv = np.zeros((T, H_kv, D), np.float64)
+    rc = _load().oracle_sparse_attention_backward(B, Sq, H_q, H_kv, n_idx, D, block, top_k,
+                                                  _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(ids),
+                                                  _ptr(lens), _ptr(kv_offsets), T, float(scale),
+                                                  _ptr(dq), _ptr(dk), _ptr(dv),
+                                                  n_threads or default_threads())
+    if rc != 0:
+        raise ValueError(f"oracle_sparse_attention_backward rejected its input (code {rc})")
+    return dq, dk, dv

@@ -380,3 +380,143 @@ int oracle_sparse_attention(int B, int Sq, int H_q, int H_kv, int D, int block, 
                                       lens, kv_offsets, kv_capacity, scale, rows, n_rows, out, wsum,
                                       n_threads);
 }
+
+/* ------------------------------------------------------------------ backward
+ * Gradient of the sparse branch (the index branch's selection is piecewise
+ * constant in its inputs and passes no gradient).  For one (row, head) with
+ * kept keys K (t in a kept block, t <= p), z_t = scale * q.k_t,
+ * P = softmax(z), O = sum_t P_t v_t, and an upstream gradient dO:
+ *   dV_t += P_t dO                 dP_t = dO . v_t
+ *   Delta = sum_t P_t dP_t (= dO . O)
+ *   dZ_t = P_t (dP_t - Delta)
+ *   dQ   = scale * sum_t dZ_t k_t  dK_t += scale * dZ_t q
+ * dK and dV of a key sum over every (row, head) of its group that kept it.
+ * A job is one (sequence, group): it owns the dK/dV rows of that sequence
+ * and group, so jobs never write the same element. */
+typedef struct {
+    int B, Sq, H_q, H_kv, n_idx, D, block, top_k;
+    int64_t kv_capacity;
+    const uint16_t *q, *k, *v, *dout;
+    const int32_t *lens, *block_ids;
+    const int64_t *kv_offsets;
+    double scale;
+    double *dq;      /* [B*Sq, H_q, D] */
+    double *dk, *dv; /* [kv_capacity, H_kv, D], zeroed by the caller */
+    int err;
+} bjob_t;
+
+typedef struct { bjob_t *job; int first, stride; } bslice_t;
+
+static void bwd_seq_group(bjob_t *J, int b, int g)
+{
+    const int K = J->top_k, blk = J->block, D = J->D, G = J->H_q / J->H_kv;
+    const int64_t L = J->lens[b];
+    if (L < J->Sq || J->kv_offsets[b] < 0 || J->kv_offsets[b] + L > J->kv_capacity) {
+        J->err = 1;
+        return;
+    }
+    const int64_t off = J->kv_offsets[b];
+    const int gi = g / (J->H_kv / J->n_idx);
+    int64_t max_keys = (int64_t)K * blk;
+    int64_t *keys = (int64_t *)malloc(sizeof(int64_t) * max_keys);
+    double *z = (double *)malloc(sizeof(double) * max_keys);
+    double *dp = (double *)malloc(sizeof(double) * max_keys);
+    for (int i = 0; i < J->Sq; ++i) {
+        const int64_t r = (int64_t)b * J->Sq + i;
+        const int64_t p = L - J->Sq + i;
+        const int own = (int)(p / blk);
+        const int32_t *ids = J->block_ids + (r * J->n_idx + gi) * (int64_t)K;
+        int64_t nk = 0;
+        for (int q = 0; q < K; ++q) {
+            int j = ids[q];
+            if (j < 0) continue;
+            if (j > own) { J->err = 2; continue; }
+            int64_t t_end = (int64_t)(j + 1) * blk;
+            if (t_end > p + 1) t_end = p + 1;
+            for (int64_t t = (int64_t)j * blk; t < t_end && nk < max_keys; ++t) keys[nk++] = t;
+        }
+        for (int hh = 0; hh < G; ++hh) {
+            const int h = g * G + hh;
+            const uint16_t *qh = J->q + (r * J->H_q + h) * (int64_t)D;
+            const uint16_t *doh = J->dout + (r * J->H_q + h) * (int64_t)D;
+            /* forward: softmax weights */
+            double m = -INFINITY;
+            for (int64_t a = 0; a < nk; ++a) {
+                const uint16_t *kt = J->k + ((off + keys[a]) * J->H_kv + g) * (int64_t)D;
+                double s = 0.0;
+                for (int d = 0; d < D; ++d) s += bf16_to_double(qh[d]) * bf16_to_double(kt[d]);
+                z[a] = s * J->scale;
+                if (z[a] > m) m = z[a];
+            }
+            double l = 0.0;
+            for (int64_t a = 0; a < nk; ++a) { z[a] = exp(z[a] - m); l += z[a]; }
+            for (int64_t a = 0; a < nk; ++a) z[a] /= l;          /* z now holds P */
+            /* dP, Delta, dV */
+            double delta = 0.0;
+            for (int64_t a = 0; a < nk; ++a) {
+                const int64_t kr = (off + keys[a]) * J->H_kv + g;
+                const uint16_t *vt = J->v + kr * (int64_t)D;
+                double s = 0.0;
+                for (int d = 0; d < D; ++d) {
+                    const double dod = bf16_to_double(doh[d]);
+                    s += dod * bf16_to_double(vt[d]);
+                    J->dv[kr * D + d] += z[a] * dod;
+                }
+                dp[a] = s;
+                delta += z[a] * s;
+            }
+            /* dZ, dQ, dK */
+            double *dqh = J->dq + (r * J->H_q + h) * (int64_t)D;
+            for (int d = 0; d < D; ++d) dqh[d] = 0.0;
+            for (int64_t a = 0; a < nk; ++a) {
+                const double dz = z[a] * (dp[a] - delta);
+                const int64_t kr = (off + keys[a]) * J->H_kv + g;
+                const uint16_t *kt = J->k + kr * (int64_t)D;
+                for (int d = 0; d < D; ++d) {
+                    dqh[d] += J->scale * dz * bf16_to_double(kt[d]);
+                    J->dk[kr * D + d] += J->scale * dz * bf16_to_double(qh[d]);
+                }
+            }
+        }
+    }
+    free(keys); free(z); free(dp);
+}
+
+static void *bwd_worker(void *arg)
+{
+    bslice_t *s = (bslice_t *)arg;
+    const int n = s->job->B * s->job->H_kv;
+    for (int jb = s->first; jb < n; jb += s->stride) bwd_seq_group(s->job, jb / s->job->H_kv, jb % s->job->H_kv);
+    return NULL;
+}
+
+/* Backward of the sparse branch for all B*Sq rows: dq [B*Sq, H_q, D] is
+ * written; dk, dv [kv_capacity, H_kv, D] (double) are accumulated into and
+ * must start at zero.  block_ids [B*Sq, n_idx, top_k] as for the forward. */
+int oracle_sparse_attention_backward(int B, int Sq, int H_q, int H_kv, int n_idx, int D, int block,
+                                     int top_k, const uint16_t *q, const uint16_t *k,
+                                     const uint16_t *v, const uint16_t *dout,
+                                     const int32_t *block_ids, const int32_t *lens,
+                                     const int64_t *kv_offsets, int64_t kv_capacity, double scale,
+                                     double *dq, double *dk, double *dv, int n_threads)
+{
+    if (B < 1 || Sq < 1 || H_q < 1 || H_kv < 1 || H_q % H_kv || D < 1 || block < 1 || top_k < 1)
+        return -1;
+    if (n_idx < 1 || H_kv % n_idx) return -1;
+    bjob_t J;
+    memset(&J, 0, sizeof J);
+    J.B = B; J.Sq = Sq; J.H_q = H_q; J.H_kv = H_kv; J.n_idx = n_idx; J.D = D; J.block = block;
+    J.top_k = top_k; J.kv_capacity = kv_capacity; J.q = q; J.k = k; J.v = v; J.dout = dout;
+    J.lens = lens; J.block_ids = block_ids; J.kv_offsets = kv_offsets; J.scale = scale;
+    J.dq = dq; J.dk = dk; J.dv = dv;
+    int nt = n_threads < 1 ? 1 : (n_threads > 512 ? 512 : n_threads);
+    if (nt > B * H_kv) nt = B * H_kv;
+    pthread_t th[512];
+    bslice_t sl[512];
+    for (int t = 0; t < nt; ++t) {
+        sl[t].job = &J; sl[t].first = t; sl[t].stride = nt;
+        pthread_create(&th[t], NULL, bwd_worker, &sl[t]);
+    }
+    for (int t = 0; t < nt; ++t) pthread_join(th[t], NULL);
+    return J.err;
+}
