@@ -2,12 +2,14 @@
 (index score + block max-pool, top-k, sparse attention with split-K merge)
 for one batch, through the C ABI; a decode run also times the same decode
 step on the index-branch variants (fewer index heads, shared index keys,
-E4M3 index keys) and one 128k-token prefill (index GEMM + fused top-k,
-sparse attention) as sub-objects.
+E4M3 index keys), the sparse branch's backward on the 2k-row prefill, and one
+128k-token prefill (index GEMM + fused top-k, sparse attention) as
+sub-objects.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode_1m]
                     [--impl msa|reference] [--no-cpu-baseline] [--no-e2e]
-                    [--no-prefill] [--no-variants] [--prefill-steps S] [--prefill-len N]
+                    [--no-prefill] [--no-variants] [--no-backward] [--prefill-steps S]
+                    [--prefill-len N]
 
 Prints ONE JSON line (rank 0).  N > 1 runs under torchrun: every rank runs
 its own independent batch (weak scaling, no data-path collective).
@@ -51,6 +53,8 @@ def parse():
                     help="skip the prefill_128k measurement attached to a decode run")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the index-branch variant measurement attached to a decode run")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the sparse-branch backward measurement attached to a decode run")
     ap.add_argument("--prefill-steps", type=int, default=5)
     ap.add_argument("--prefill-len", type=int, default=None,
                     help="override the prefill length (profiling captures of a smaller case)")
@@ -159,6 +163,60 @@ def measure_prefill(name, dev, steps, warmup, seq_len=None):
            "index_tflop": idx_flops / 1e12, "index_ms": idx_ms,
            "index_tflops": idx_flops / (idx_ms / 1e3) / 1e12,
            "kernel_ms": per, "gpu_launches_per_step": len(trace) / steps}
+    del eng, w
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_backward(name, dev, steps, warmup):
+    """Times msa_sparse_attention_backward on a prefill workload's own
+    selection.  Useful FLOPs: 10*D per (row, head, visible kept key) -- the
+    five products S = QK^T, dP = dO V^T, dV += P^T dO, dK += dZ^T Q,
+    dQ += dZ K; reduction bytes: the fp32 dK and dV rows every (row, group,
+    kept block) adds (valid tokens x 128 dims x 4 B x 2)."""
+    import block_sparse_attention_43_b200 as msa
+    from synthetic import make_workload
+    w = make_workload(name, dev)
+    eng = msa.MSA(batch=w.B, q_len=w.Sq, max_kv_len=max(w.lens_host), num_q_heads=w.H_q,
+                  num_kv_heads=w.H_kv, top_k=w.top_k, kv_capacity=w.kv_capacity, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    eng.index_topk(w.q_idx, w.k_idx, w.lens, w.kv_offsets, stream)
+    g = torch.Generator(device=dev).manual_seed(1)
+    dout = torch.randn(w.q.shape, generator=g, device=dev).to(torch.bfloat16)
+    dq = torch.empty_like(w.q)
+    dk = torch.zeros(w.k.shape, dtype=torch.float32, device=dev)
+    dv = torch.zeros(w.v.shape, dtype=torch.float32, device=dev)
+    ws = msa.alloc_workspace(msa.msa_sparse_attention_backward_workspace_size(eng.shape), dev)
+
+    def step():
+        msa.msa_sparse_attention_backward(eng.shape, w.q, w.k, w.v, eng.block_ids, w.lens,
+                                          w.kv_offsets, w.scale, dout, dq, dk, dv, ws, stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    st = msa.msa_read_device_status(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"backward device status {msa.STATUS_NAMES.get(st, st)}")
+    ids = eng.block_ids.cpu().numpy()
+    fwd_useful = prefill_useful_flops(w, ids)             # 4*D per (row, head, key)
+    useful = fwd_useful * 10 // 4
+    keys_per_group = fwd_useful // (4 * w.D * (w.H_q // w.H_kv))
+    red_bytes = keys_per_group * w.D * 4 * 2
+    msa.msa_trace_enable(True)
+    for _ in range(steps):
+        step()
+    torch.cuda.synchronize()
+    trace = msa.msa_trace_read()
+    msa.msa_trace_enable(False)
+    ms = float(np.mean([t for n, t in trace if n == "sparse_attention_backward"]))
+    _, tf_burst, _, kind = measured_peaks()
+    res = {"workload": w.name, "rows": w.B * w.Sq, "H_q": w.H_q, "H_kv": w.H_kv, "top_k": w.top_k,
+           "ms": ms, "useful_tflop": useful / 1e12, "tflops": useful / (ms / 1e3) / 1e12,
+           "frac_of_bf16_burst": useful / (ms / 1e3) / 1e12 / tf_burst,
+           "dk_dv_reduction_bytes": red_bytes, "reduction_gbs": red_bytes / (ms / 1e3) / 1e9,
+           "bound": "fp32 dK/dV reductions (one 128-row block per row and kept block)",
+           "peak_kind": kind}
     del eng, w
     torch.cuda.empty_cache()
     return res
@@ -506,6 +564,10 @@ def main():
     if not args.no_variants and world == 1:
         variants = measure_index_variants(w, dev, 20, 3)
 
+    backward = None
+    if not args.no_backward and world == 1:
+        backward = measure_backward("prefill_2k", dev, 20, 3)
+
     prefill = None
     if not args.no_prefill and world == 1:
         del eng
@@ -546,6 +608,7 @@ def main():
             "cpu_baseline": cpu,
             "prefill_128k": prefill,
             "index_variants": variants,
+            "prefill_backward": backward,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

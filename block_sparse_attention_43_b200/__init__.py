@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
 EXPORTS = ("msa_index_topk_workspace_size", "msa_index_topk", "msa_index_topk_fp8",
            "msa_sparse_attention_workspace_size", "msa_sparse_attention",
            "msa_index_topk_paged", "msa_sparse_attention_paged", "msa_kv_append",
-           "msa_index_topk_static", "msa_read_device_status", "msa_trace_enable",
+           "msa_index_topk_static", "msa_sparse_attention_backward_workspace_size",
+           "msa_sparse_attention_backward", "msa_read_device_status", "msa_trace_enable",
            "msa_trace_read",
            "msa_status_string")
 
@@ -74,6 +75,11 @@ def _load():
     lib.msa_kv_append.restype = ctypes.c_int
     lib.msa_index_topk_static.argtypes = [S, P, P, P, P, P, P, P]
     lib.msa_index_topk_static.restype = ctypes.c_int
+    lib.msa_sparse_attention_backward_workspace_size.argtypes = [S]
+    lib.msa_sparse_attention_backward_workspace_size.restype = Z
+    lib.msa_sparse_attention_backward.argtypes = [S, P, P, P, P, P, P, ctypes.c_float, P, P, P, P,
+                                                  P, Z, P]
+    lib.msa_sparse_attention_backward.restype = ctypes.c_int
     lib.msa_read_device_status.argtypes = [P, P]
     lib.msa_read_device_status.restype = ctypes.c_int
     lib.msa_trace_enable.argtypes = [ctypes.c_int]
@@ -194,6 +200,22 @@ def msa_index_topk_static(shape, q_idx, k_idx, lens, kv_offsets, block_ids, bloc
                                      _ptr(kv_offsets), _ptr(block_ids), _ptr(block_scores),
                                      _stream(stream)),
            "msa_index_topk_static")
+
+
+def msa_sparse_attention_backward_workspace_size(shape: msa_shape_t) -> int:
+    return lib.msa_sparse_attention_backward_workspace_size(ctypes.byref(shape))
+
+
+def msa_sparse_attention_backward(shape, q, k_cache, v_cache, block_ids, lens, kv_offsets,
+                                  softmax_scale, d_out, dq, dk, dv, workspace, stream=None) -> None:
+    """Backward of the sparse branch: writes dq (bf16), adds into dk and dv
+    (float32, [kv_capacity, H_kv, 128]); see include/msa.h."""
+    _check(lib.msa_sparse_attention_backward(ctypes.byref(shape), _ptr(q), _ptr(k_cache),
+                                             _ptr(v_cache), _ptr(block_ids), _ptr(lens),
+                                             _ptr(kv_offsets), float(softmax_scale), _ptr(d_out),
+                                             _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                                             workspace.numel(), _stream(stream)),
+           "msa_sparse_attention_backward")
 
 
 def msa_read_device_status(workspace, stream=None) -> int:

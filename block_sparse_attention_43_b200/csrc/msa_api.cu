@@ -418,6 +418,41 @@ msa_status_t msa_kv_append(const msa_shape_t *shape, int32_t n_new, const void *
                                                                                      : MSA_ERR_CUDA;
 }
 
+size_t msa_sparse_attention_backward_workspace_size(const msa_shape_t *shape) {
+    if (check_shape(shape) != MSA_OK) return 0;
+    return kWsHeaderBytes;
+}
+
+msa_status_t msa_sparse_attention_backward(const msa_shape_t *shape, const void *q,
+                                           const void *k_cache, const void *v_cache,
+                                           const int32_t *block_ids, const int32_t *lens,
+                                           const int64_t *kv_offsets, float softmax_scale,
+                                           const void *d_out, void *dq, float *dk, float *dv,
+                                           void *workspace, size_t workspace_bytes,
+                                           msa_stream_t stream) {
+    msa_status_t st = check_shape(shape);
+    if (st != MSA_OK) return st;
+    if (!q || !k_cache || !v_cache || !block_ids || !lens || !kv_offsets || !d_out || !dq || !dk ||
+        !dv)
+        return MSA_ERR_INVALID_ARG;
+    if (!(softmax_scale == softmax_scale) || softmax_scale == INFINITY || softmax_scale == -INFINITY)
+        return MSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(d_out) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return MSA_ERR_MISALIGNED;
+    if ((st = check_ws(workspace, workspace_bytes, kWsHeaderBytes)) != MSA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(workspace, 0, kWsHeaderBytes, s) != cudaSuccess) return MSA_ERR_CUDA;
+    AttnBwdArgs a;
+    a.q = q; a.k_cache = k_cache; a.v_cache = v_cache; a.dout = d_out; a.ids = block_ids;
+    a.lens = lens; a.kv = packed_map(shape, kv_offsets); a.dq = dq; a.dk = dk; a.dv = dv;
+    a.status = static_cast<int *>(workspace);
+    a.B = shape->batch; a.Sq = shape->q_len; a.H_q = shape->num_q_heads;
+    a.H_kv = shape->num_kv_heads; a.n_idx = index_heads(shape); a.K = shape->top_k;
+    a.max_kv_len = shape->max_kv_len; a.softmax_scale = softmax_scale;
+    return launch_attn_bwd(a, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+}
+
 msa_status_t msa_read_device_status(const void *workspace, msa_stream_t stream) {
     if (!workspace) return MSA_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

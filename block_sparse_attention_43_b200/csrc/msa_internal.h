@@ -165,6 +165,23 @@ bool encode_q_gather_map(CUtensorMap *map, const void *q, int H_q, long long row
 
 // Appends n_new tokens per sequence after its current length (kv_append.cu):
 // src[i] [B][n_new][H_kv][128] -> dst[i] at rows of tokens lens[b] .. + n_new - 1.
+// Backward of the sparse branch (attn_bwd.cu): one CTA per (row, group).
+struct AttnBwdArgs {
+    const void *q;          // [B][Sq][H_q][128]
+    const void *k_cache;
+    const void *v_cache;
+    const void *dout;       // [B][Sq][H_q][128]
+    const int32_t *ids;     // [B*Sq][n_idx][K]
+    const int32_t *lens;
+    KvMap kv;
+    void *dq;               // [B][Sq][H_q][128] bf16, written
+    float *dk, *dv;         // [capacity][H_kv][128] fp32, added to
+    int *status;
+    int B, Sq, H_q, H_kv, n_idx, K, max_kv_len;
+    float softmax_scale;
+};
+cudaError_t launch_attn_bwd(const AttnBwdArgs &a, cudaStream_t s);
+
 struct KvAppendArgs {
     const void *src[3];
     void *dst[3];

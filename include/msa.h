@@ -174,6 +174,34 @@ MSA_API msa_status_t msa_sparse_attention(const msa_shape_t *shape, const void *
                                   float softmax_scale, void *out,
                                   void *workspace, size_t workspace_bytes, msa_stream_t stream);
 
+/* Backward of the sparse branch (training; the pages say MSA is trained
+ * natively, "百万token上下文提速近10倍..." section 五).  The index branch's
+ * selection is piecewise constant and passes no gradient, so block_ids are an
+ * input, as in the forward.  For each (row, head) over its kept keys t:
+ *   P = softmax(softmax_scale * q.k_t), dP_t = d_out.v_t,
+ *   Delta = sum_t P_t dP_t, dZ_t = P_t (dP_t - Delta),
+ *   dq = softmax_scale * sum_t dZ_t k_t,
+ *   dk_t += softmax_scale * dZ_t q,   dv_t += P_t d_out.
+ * The forward softmax is recomputed (no saved statistics are needed).
+ *   q, k_cache, v_cache, block_ids, lens, kv_offsets: as msa_sparse_attention
+ *   d_out        device bf16 [B, q_len, H_q, head_dim], gradient of out
+ *   dq           device bf16 [B, q_len, H_q, head_dim]  (written)
+ *   dk, dv       device float [kv_capacity, H_kv, head_dim]: the gradients of
+ *                this call are ADDED (fp32 atomics, so their summation order
+ *                and last bits vary by run); start them at zero.
+ *   workspace    >= msa_sparse_attention_backward_workspace_size bytes
+ * This is a first, row-oriented implementation (one CTA per row and group):
+ * every (row, kept block) adds a 128 x 128 block to dk and dv, which bounds
+ * it at large q_len. */
+MSA_API size_t msa_sparse_attention_backward_workspace_size(const msa_shape_t *shape);
+MSA_API msa_status_t msa_sparse_attention_backward(const msa_shape_t *shape, const void *q,
+                                                   const void *k_cache, const void *v_cache,
+                                                   const int32_t *block_ids, const int32_t *lens,
+                                                   const int64_t *kv_offsets, float softmax_scale,
+                                                   const void *d_out, void *dq, float *dk,
+                                                   float *dv, void *workspace,
+                                                   size_t workspace_bytes, msa_stream_t stream);
+
 /* Paged caches (a block-table layout for serving): the index keys, keys and
  * values of all sequences live in pools of 128-token pages, [kv_capacity,
  * H_kv, dim] with page p = rows p*128 .. p*128+127, and block j of sequence b

@@ -1,0 +1,104 @@
+"""GPU parity of the sparse branch's backward (dQ, dK, dV over the kept
+blocks) through the C ABI against the CPU oracle's exact derivative, on the
+same bf16 inputs and the same selection.
+
+Tolerance: relative L2 <= 1e-2 and max-abs <= 2 % of the largest reference
+magnitude, per gradient.  The kernel rounds P and dZ to bf16 as operands of
+the products (2^-9 relative each) and writes dQ as bf16; dK and dV are fp32
+sums of those products.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_43_b200 as m
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+REL_L2 = 1e-2
+MAX_ABS_FRAC = 2e-2
+
+
+def _check(name, got, ref):
+    got = np.asarray(got, np.float64)
+    assert np.isfinite(got).all(), f"{name}: non-finite"
+    err = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    mx = np.abs(got - ref).max()
+    assert err <= REL_L2, f"{name}: rel-L2 {err}"
+    assert mx <= MAX_ABS_FRAC * max(np.abs(ref).max(), 1e-6), f"{name}: max-abs {mx}"
+    return err
+
+
+def _run(oracle_mod, w, n_idx=None, padded_nan=False):
+    from synthetic import bf16_bits
+    n_idx = n_idx or w.H_kv
+    q_idx = w.q_idx[:, :, :n_idx].contiguous()
+    k_idx = w.k_idx[:, :n_idx].contiguous()
+    eng = m.MSA(batch=w.B, q_len=w.Sq, max_kv_len=max(w.lens_host), num_q_heads=w.H_q,
+                num_kv_heads=w.H_kv, top_k=w.top_k, kv_capacity=w.kv_capacity, device=DEV,
+                num_index_heads=n_idx)
+    eng.index_topk(q_idx, k_idx, w.lens, w.kv_offsets)
+    g = torch.Generator(device=DEV).manual_seed(77)
+    dout = torch.randn(w.q.shape, generator=g, device=DEV).to(torch.bfloat16)
+    dq = torch.empty_like(w.q)
+    dk = torch.zeros(w.k.shape, dtype=torch.float32, device=DEV)
+    dv = torch.zeros(w.v.shape, dtype=torch.float32, device=DEV)
+    ws = m.alloc_workspace(m.msa_sparse_attention_backward_workspace_size(eng.shape), DEV)
+    m.msa_sparse_attention_backward(eng.shape, w.q, w.k, w.v, eng.block_ids, w.lens,
+                                    w.kv_offsets, w.scale, dout, dq, dk, dv, ws)
+    torch.cuda.synchronize()
+    assert m.msa_read_device_status(ws) == 0
+    ids = eng.block_ids.cpu().numpy()
+    k_host, v_host = bf16_bits(w.k), bf16_bits(w.v)
+    if padded_nan:
+        # the oracle reads only tokens < lens; NaN padding becomes 0 in its copy
+        k_host = np.where(np.isnan(w.k.float().cpu().numpy()), 0, k_host).astype(np.uint16)
+        v_host = np.where(np.isnan(w.v.float().cpu().numpy()), 0, v_host).astype(np.uint16)
+    rq, rk, rv = oracle_mod.sparse_attention_backward(
+        bf16_bits(w.q), k_host, v_host, bf16_bits(dout), ids, w.lens.cpu().numpy(),
+        w.kv_offsets.cpu().numpy(), scale=w.scale, num_index_heads=n_idx)
+    gq = dq.float().cpu().numpy().reshape(rq.shape)
+    gk, gv = dk.cpu().numpy(), dv.cpu().numpy()
+    rep = dict(dq=_check("dq", gq, rq), dk=_check("dk", gk, rk), dv=_check("dv", gv, rv))
+    # keys no row kept get no gradient at all
+    untouched = (rk == 0).all(axis=-1) & (rv == 0).all(axis=-1)
+    assert (gk[untouched] == 0).all() and (gv[untouched] == 0).all()
+    return rep
+
+
+CASES = [
+    # (B, Sq, lens, H_q, H_kv, top_k)
+    (1, 300, [300], 8, 2, 4),              # full prefill, ragged last block
+    (2, 64, [500, 64], 16, 4, 3),          # chunked prefill after a cached prefix
+    (1, 1000, [1000], 64, 8, 16),          # groups of 8, every block kept
+    (1, 700, [700], 32, 2, 4),             # groups of 16 (two n8 tiles)
+    (3, 1, [5000, 129, 2000], 16, 2, 8),   # decode rows
+    (1, 2000, [2000], 8, 8, 16),           # one head per group (7 padding heads)
+]
+
+
+@pytest.mark.parametrize("B,Sq,lens,H_q,H_kv,top_k", CASES)
+def test_backward_matches_oracle(oracle_mod, B, Sq, lens, H_q, H_kv, top_k):
+    from synthetic import make_inputs
+    w = make_inputs(B=B, Sq=Sq, lens=lens, H_q=H_q, H_kv=H_kv, top_k=top_k, seed=700 + Sq,
+                    device=DEV)
+    print((B, Sq, H_q, H_kv, top_k), _run(oracle_mod, w))
+
+
+def test_backward_with_fewer_index_heads(oracle_mod):
+    from synthetic import make_inputs
+    w = make_inputs(B=1, Sq=600, lens=[600], H_q=64, H_kv=8, top_k=4, seed=71, device=DEV)
+    print(_run(oracle_mod, w, n_idx=2))
+
+
+def test_backward_ignores_nan_padding(oracle_mod):
+    """Padded cache (offset b*4096) with NaN past each length: nothing past a
+    sequence's query position may reach a gradient."""
+    from synthetic import make_inputs
+    lens = [1000, 300]
+    w = make_inputs(B=2, Sq=300, lens=lens, H_q=16, H_kv=2, top_k=4, seed=72, device=DEV,
+                    padded_to=1024)
+    for t in (w.k, w.v):
+        for b, L in enumerate(lens):
+            t[b * 1024 + L:(b + 1) * 1024] = float("nan")
+    print(_run(oracle_mod, w, padded_nan=True))
