@@ -128,6 +128,8 @@ struct Smem {
     uint64_t kv_full[2], kv_empty[2], q_full[2], q_empty[2];
     uint64_t s_full, s_empty, o_full[2], o_empty[2];
     uint64_t p_full, p_empty;
+    float xmax[2][128];                    // pass A: each softmax warp's half-row max
+    uint64_t xbar[4];                      // pass A: the two softmax warps of a lane quarter
     uint64_t item_full[4], item_empty[4];  // work-item queue: producer -> MMA, softmax, epilogue
     Item item_q[4];                        // decoded items (n = -1: no more work)
     uint32_t tmem_base;
@@ -184,6 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&S.s_empty, kSoftWarps);
         mbar_init(&S.p_full, kSoftWarps);
         mbar_init(&S.p_empty, 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&S.xbar[i], 64);   // every lane of both warps
         for (int i = 0; i < kQueue; ++i) {
             mbar_init(&S.item_full[i], 1);
             mbar_init(&S.item_empty[i], kQueueReaders);
@@ -451,32 +454,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const uint32_t sa = lane_addr + kColS;
                 long long lim = 127;                   // last visible column of the row
-                if (MODE == 0) {
-                    // own block: causal mask t <= p, exact max of the visible logits
-                    const long long p = static_cast<long long>(x.L) - P.Sq +
-                                        (row - static_cast<long long>(x.b) * P.Sq);
-                    lim = p - static_cast<long long>(x.j) * 128;
-                    float mx = -INFINITY;
-#pragma unroll
-                    for (int c = 0; c < 4; c += 2) {
-                        uint32_t a[32], b[32];
-                        tmem_ld32r(sa + c * 32, a);
-                        tmem_ld32r(sa + c * 32 + 32, b);
-                        tmem_wait_ld(a);
-                        tmem_tie(b);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            if (c * 32 + e <= lim) mx = fmaxf(mx, __uint_as_float(a[e]) * sl2);
-                            if (c * 32 + 32 + e <= lim) mx = fmaxf(mx, __uint_as_float(b[e]) * sl2);
-                        }
-                    }
-                    shift = valid ? mx : 0.f;
-                }
                 uint32_t a[32], b[32];
                 tmem_ld32r(sa + ch * 64, a);
                 tmem_ld32r(sa + ch * 64 + 32, b);
                 tmem_wait_ld(a);
                 tmem_tie(b);
+                if (MODE == 0) {
+                    // own block: causal mask t <= p, exact max of the visible
+                    // logits.  Each warp of the pair takes the max of its own
+                    // 64 columns and swaps it with its partner (same TMEM
+                    // lanes, other half) through shared memory.
+                    const long long p = static_cast<long long>(x.L) - P.Sq +
+                                        (row - static_cast<long long>(x.b) * P.Sq);
+                    lim = p - static_cast<long long>(x.j) * 128;
+                    float mx = -INFINITY;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        if (ch * 64 + e <= lim) mx = fmaxf(mx, __uint_as_float(a[e]) * sl2);
+                        if (ch * 64 + 32 + e <= lim) mx = fmaxf(mx, __uint_as_float(b[e]) * sl2);
+                    }
+                    // One buffer suffices: a warp writes the next tile's value
+                    // only once S of that tile exists, i.e. after both warps
+                    // of the pair arrived on s_empty below, after this read.
+                    S.xmax[ch][m] = mx;
+                    mbar_arrive(&S.xbar[warp & 3]);
+                    bool xok = !*abort_flag && mbar_wait(&S.xbar[warp & 3], qt & 1, P.status);
+                    xok = __all_sync(0xffffffffu, xok);
+                    if (!xok) { ok = false; break; }
+                    mx = fmaxf(mx, S.xmax[ch ^ 1][m]);
+                    shift = valid ? mx : 0.f;
+                }
                 // S is in registers: the next tile's QK may overwrite it.
                 tc_fence_before();
                 __syncwarp();
