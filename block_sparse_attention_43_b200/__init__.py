@@ -26,7 +26,8 @@ EXPORTS = ("msa_index_topk_workspace_size", "msa_index_topk", "msa_index_topk_fp
            "msa_sparse_attention_workspace_size", "msa_sparse_attention",
            "msa_index_topk_paged", "msa_sparse_attention_paged", "msa_kv_append",
            "msa_index_topk_static", "msa_sparse_attention_backward_workspace_size",
-           "msa_sparse_attention_backward", "msa_read_device_status", "msa_trace_enable",
+           "msa_sparse_attention_backward", "msa_decode_step_workspace_size",
+           "msa_decode_step", "msa_read_device_status", "msa_trace_enable",
            "msa_trace_read",
            "msa_status_string")
 
@@ -80,6 +81,10 @@ def _load():
     lib.msa_sparse_attention_backward.argtypes = [S, P, P, P, P, P, P, ctypes.c_float, P, P, P, P,
                                                   P, Z, P]
     lib.msa_sparse_attention_backward.restype = ctypes.c_int
+    lib.msa_decode_step_workspace_size.argtypes = [S]
+    lib.msa_decode_step_workspace_size.restype = Z
+    lib.msa_decode_step.argtypes = [S, P, P, P, P, P, P, P, ctypes.c_float, P, P, P, P, Z, P]
+    lib.msa_decode_step.restype = ctypes.c_int
     lib.msa_read_device_status.argtypes = [P, P]
     lib.msa_read_device_status.restype = ctypes.c_int
     lib.msa_trace_enable.argtypes = [ctypes.c_int]
@@ -218,6 +223,21 @@ def msa_sparse_attention_backward(shape, q, k_cache, v_cache, block_ids, lens, k
            "msa_sparse_attention_backward")
 
 
+def msa_decode_step_workspace_size(shape: msa_shape_t) -> int:
+    return lib.msa_decode_step_workspace_size(ctypes.byref(shape))
+
+
+def msa_decode_step(shape, q_idx, k_idx, q, k_cache, v_cache, lens, kv_offsets, softmax_scale,
+                    block_ids, block_scores, out, workspace, stream=None) -> None:
+    """Index branch, top-k and sparse branch of a decode step in one launch;
+    see include/msa.h."""
+    _check(lib.msa_decode_step(ctypes.byref(shape), _ptr(q_idx), _ptr(k_idx), _ptr(q),
+                               _ptr(k_cache), _ptr(v_cache), _ptr(lens), _ptr(kv_offsets),
+                               float(softmax_scale), _ptr(block_ids), _ptr(block_scores),
+                               _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "msa_decode_step")
+
+
 def msa_read_device_status(workspace, stream=None) -> int:
     return lib.msa_read_device_status(_ptr(workspace), _stream(stream))
 
@@ -283,6 +303,19 @@ class MSA:
     def forward(self, q_idx, k_idx, q, k_cache, v_cache, lens, kv_offsets, stream=None):
         self.index_topk(q_idx, k_idx, lens, kv_offsets, stream)
         return self.sparse_attention(q, k_cache, v_cache, lens, kv_offsets, stream=stream)
+
+    def decode_step(self, q_idx, k_idx, q, k_cache, v_cache, lens, kv_offsets, stream=None):
+        """The fused single-launch decode step (q_len 1); same results as
+        forward().  Its workspace is allocated on first use."""
+        if getattr(self, "ws_step", None) is None:
+            n = msa_decode_step_workspace_size(self.shape)
+            if n == 0:
+                raise MSAError(2, "shape rejected by msa_decode_step")
+            self.ws_step = alloc_workspace(n, self.device)
+        msa_decode_step(self.shape, q_idx, k_idx, q, k_cache, v_cache, lens, kv_offsets,
+                        self.softmax_scale, self.block_ids, self.block_scores, self.out,
+                        self.ws_step, stream)
+        return self.out
 
     def device_status(self, stream=None) -> int:
         a = msa_read_device_status(self.ws_index, stream)

@@ -1,0 +1,588 @@
+// decode_fused.cu -- the whole MSA decode step in one persistent launch:
+// index scores + block max-pool, top-k per (sequence, group), and sparse
+// attention over the kept blocks.
+//
+// Method: "百万token上下文提速近10倍，MiniMax M3的稀疏注意力凭什么这么快"
+// (cloud.tencent.com), section 二 (index branch, Block Max Pool, top-k; exact
+// attention over the kept blocks) and section 六 (the group's heads share its
+// blocks); the step's cost is the index keys streamed from HBM (section 四).
+//
+// Why one launch: with separate kernels, top-k and attention of every
+// sequence wait for the index scores of all sequences.  Here they overlap the
+// index streaming of the later sequences:
+//   - CTAs (one per SM, cooperative launch so all are resident) claim index
+//     units (one 128-token block of one sequence, all groups) from a global
+//     counter in sequence order, so sequences finish one after another;
+//   - the CTA that finishes a sequence's last unit runs that sequence's top-k
+//     (one warp per group, the warp selection of topk.cu) and publishes one
+//     attention item per (group, kept block);
+//   - between index units a CTA takes published attention items: the block's
+//     K/V tiles (TMA, 128-byte swizzle), S^T = K Q^T and O^T = V^T P^T on
+//     mma.sync for the group's heads, a partial (max, sum, O) per kept block;
+//     the CTA finishing a (sequence, group)'s last block merges its partials
+//     and writes the output.
+// Attention items are claimed with a compare-and-swap only while the claim
+// index is below the published count, so a claimed item is either published
+// or about to be by a CTA inside its (wait-free) publishing step; every other
+// wait is bounded.
+#include "msa_device.cuh"
+#include "msa_internal.h"
+#include "topk_warp.cuh"
+
+namespace msa {
+namespace {
+
+constexpr int kWarps = 8;                     // consumer warps
+constexpr int kConsumers = kWarps * 32;
+constexpr int kThreads = kConsumers + 32;     // + producer warp
+constexpr int kStages = 5;
+constexpr int kStageBytes = 32768;
+constexpr int kQueue = 4;
+constexpr int kMaxBatch = 4096;
+constexpr int kRec = 132;                     // partial record per head: m, l, 2 pad, O[128]
+constexpr float kLog2e = 1.4426950408889634f;
+
+enum { kWorkIndex = 0, kWorkAttn = 1, kWorkEnd = 2 };
+
+struct Smem {
+    uint8_t ring[kStages][kStageBytes];       // index-key stages / K and V tiles of a block
+    float om[kWarps][8][kDim];                // attention: per-warp O^T; top-k scratch
+    float mw[kWarps][8], lw[kWarps][8];
+    uint64_t full[kStages], empty[kStages];
+    uint64_t wq_full[kQueue], wq_empty[kQueue];
+    uint64_t cbar;                            // consumer-wide sync (all 256 threads arrive)
+    int4 wq[kQueue];                          // {kind, a, b, c}
+    int prefix[kMaxBatch + 1];
+    float red[2][16];
+    int bcast[2];
+    int total_attn;
+    int abort_flag;
+};
+
+__device__ __forceinline__ bool seq_valid(const DecodeFusedArgs &P, int b, int L) {
+    return L >= 1 && L <= P.max_kv_len && kv_seq_ok(P.kv, b, L);
+}
+
+__device__ __forceinline__ int ld_volatile(const int *p) { return *reinterpret_cast<const volatile int *>(p); }
+
+__device__ __forceinline__ unsigned long long now_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+constexpr unsigned long long kWaitNs = 2000000000ull;   // bounded waits give up after 2 s
+
+// Score rows padded to 32 floats: rows of different (sequence, group) never
+// share a cache line, so no SM can hold a stale copy of a row it reads.
+__host__ __device__ __forceinline__ int score_stride(int nb_max) { return (nb_max + 31) & ~31; }
+
+// Largest b with prefix[b] <= u.
+__device__ __forceinline__ void unit_of(const int *prefix, int B, int u, int &b, int &j) {
+    int lo = 0, hi = B;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (prefix[mid] <= u) lo = mid; else hi = mid;
+    }
+    b = lo;
+    j = u - prefix[lo];
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                        const DecodeFusedArgs P) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem &S = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = P.H_kv, G = P.H_q / P.H_kv, K = P.K;
+    const int nbs = score_stride(P.nb_max);
+    volatile int *abort_flag = &S.abort_flag;
+
+    if (tid == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&S.full[i], 1);
+            mbar_init(&S.empty[i], kWarps);
+        }
+        for (int i = 0; i < kQueue; ++i) {
+            mbar_init(&S.wq_full[i], 1);
+            mbar_init(&S.wq_empty[i], kWarps);
+        }
+        mbar_init(&S.cbar, kConsumers);
+        S.abort_flag = 0;
+        fence_mbar_init();
+    }
+    // Units per sequence (exclusive prefix) and the number of attention items.
+    if (warp == 0) {
+        const int per = (P.B + 31) / 32;
+        const int lo = lane * per, hi = min(P.B, lo + per);
+        int sum = 0, items = 0;
+        for (int b = lo; b < hi; ++b) {
+            const int L = P.lens[b];
+            if (seq_valid(P, b, L)) {
+                const int nb = (L + kBlock - 1) / kBlock;
+                sum += nb;
+                items += H * min(K, nb);
+            } else if (blockIdx.x == 0) {
+                // rejected sequence: -1 / -inf selection, NaN output, status word
+                set_status(P.status, kStatusBadLens);
+                for (int q = 0; q < H * K; ++q) {
+                    P.ids[static_cast<long long>(b) * H * K + q] = -1;
+                    P.out_scores[static_cast<long long>(b) * H * K + q] = -INFINITY;
+                }
+                __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(P.out) + static_cast<long long>(b) * P.H_q * kDim;
+                for (int e = 0; e < P.H_q * kDim; ++e) o[e] = __float2bfloat16(NAN);
+            }
+        }
+        int incl = sum;
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, m);
+            if (lane >= m) incl += o;
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) items += __shfl_xor_sync(0xffffffffu, items, m);
+        int run = incl - sum;
+        for (int b = lo; b < hi; ++b) {
+            S.prefix[b] = run;
+            const int L = P.lens[b];
+            if (seq_valid(P, b, L)) run += (L + kBlock - 1) / kBlock;
+        }
+        if (lane == 31) S.prefix[P.B] = incl;
+        if (lane == 0) S.total_attn = items;
+    }
+    __syncthreads();
+    const int U = S.prefix[P.B];
+    const int total_attn = S.total_attn;
+
+    if (warp == kWarps) {
+        // ------------------------------------------------ producer: claims work,
+        // publishes it to the consumers and issues its loads
+        if (lane != 0) return;
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+        const uint64_t pol = l2_policy_evict_first();
+        const __nv_bfloat16 *kbase = static_cast<const __nv_bfloat16 *>(P.k_idx);
+        const int tps = 128 / H;                 // tokens per index stage
+        int n = 0, it = 0;                        // work entries pushed, stages issued
+        bool index_left = true, ok = true;
+        auto push = [&](int4 w) -> bool {
+            const int slot = n % kQueue;
+            if (n >= kQueue && (*abort_flag || !mbar_wait(&S.wq_empty[slot], ((n / kQueue) - 1) & 1, P.status)))
+                return false;
+            S.wq[slot] = w;
+            mbar_arrive(&S.wq_full[slot]);
+            ++n;
+            return true;
+        };
+        auto stage = [&](int &slot) -> bool {
+            slot = it % kStages;
+            if (it >= kStages && (*abort_flag || !mbar_wait(&S.empty[slot], ((it / kStages) - 1) & 1, P.status)))
+                return false;
+            ++it;
+            return true;
+        };
+        // Claims attention item h when h < published; returns -1 if none is
+        // available now, -2 when every item has been claimed.
+        auto try_claim = [&]() -> int {
+            int h = ld_volatile(P.ctr + 2);
+            while (true) {
+                if (h >= total_attn) return -2;
+                if (h >= ld_volatile(P.ctr + 3)) return -1;
+                const int prev = atomicCAS(P.ctr + 2, h, h + 1);
+                if (prev == h) return h;
+                h = prev;
+            }
+        };
+        const unsigned long long t0 = now_ns();
+        while (ok) {
+            int item = -1;
+            if (index_left) {
+                item = try_claim();
+                if (item < 0) {
+                    const int u = atomicAdd(P.ctr, 1);
+                    if (u >= U) { index_left = false; continue; }
+                    int b, j;
+                    unit_of(S.prefix, P.B, u, b, j);
+                    const int L = P.lens[b];
+                    const int ntok = min(kBlock, L - j * kBlock);
+                    if (!push(make_int4(kWorkIndex, b, j, ntok))) { ok = false; break; }
+                    const long long t_first = kv_block_row(P.kv, b, j, P.status);
+                    for (int t0s = 0; t0s < ntok; t0s += tps) {
+                        int slot;
+                        if (!stage(slot)) { ok = false; break; }
+                        const uint32_t bytes = static_cast<uint32_t>(min(tps, ntok - t0s)) * H * kDim * 2;
+                        mbar_arrive_expect_tx(&S.full[slot], bytes);
+                        bulk_g2s(S.ring[slot], kbase + (t_first + t0s) * H * kDim, bytes, &S.full[slot], pol);
+                    }
+                    continue;
+                }
+            } else {
+                item = try_claim();
+                if (item == -2) break;
+                if (item == -1) {
+                    if (*abort_flag || now_ns() - t0 > kWaitNs) {
+                        set_status(P.status, kStatusTimeout);
+                        ok = false;
+                        break;
+                    }
+                    __nanosleep(256);
+                    continue;
+                }
+            }
+            // Attention item: its flag is set, or about to be, by a publisher.
+            const unsigned long long tw = now_ns();
+            while (ld_volatile(P.aq_flag + item) == 0) {
+                if (*abort_flag || now_ns() - tw > kWaitNs) { set_status(P.status, kStatusTimeout); ok = false; break; }
+                __nanosleep(64);
+            }
+            if (!ok) break;
+            __threadfence();
+            const int payload = __ldcg(P.aq_item + item);
+            const int bg = payload / K, s = payload % K;
+            const int b = bg / H, g = bg % H;
+            const int j = __ldcg(P.ids + static_cast<long long>(bg) * K + s);
+            if (!push(make_int4(kWorkAttn, payload, j, 0))) { ok = false; break; }
+            const int tok = static_cast<int>(kv_block_row(P.kv, b, j, P.status));
+            int sk, sv;
+            if (!stage(sk)) { ok = false; break; }
+            mbar_arrive_expect_tx(&S.full[sk], kStageBytes);
+            tma_load_3d(S.ring[sk], &tmK, 0, g, tok, &S.full[sk]);
+            tma_load_3d(S.ring[sk] + 16384, &tmK, 64, g, tok, &S.full[sk]);
+            if (!stage(sv)) { ok = false; break; }
+            mbar_arrive_expect_tx(&S.full[sv], kStageBytes);
+            tma_load_3d(S.ring[sv], &tmV, 0, g, tok, &S.full[sv]);
+            tma_load_3d(S.ring[sv] + 16384, &tmV, 64, g, tok, &S.full[sv]);
+        }
+        if (!ok) *abort_flag = 1;
+        push(make_int4(kWorkEnd, 0, 0, 0));      // best effort: consumers also stop on abort
+        // let every copy already issued land before the CTA can exit
+        for (int k = max(0, it - kStages); k < it; ++k)
+            mbar_wait(&S.full[k % kStages], (k / kStages) & 1, nullptr);
+        return;
+    }
+
+    // ---------------------------------------------------- consumers
+    // CTA-wide syncs among the consumers are a bounded mbarrier that every
+    // consumer thread arrives on, so a warp that stops early cannot hang the
+    // others: their wait gives up, raises the abort flag and they stop too.
+    int cb = 0;
+    auto cbar = [&]() {
+        mbar_arrive(&S.cbar);
+        if (!*abort_flag && !mbar_wait(&S.cbar, cb & 1, P.status)) *abort_flag = 1;
+        ++cb;
+    };
+    const int c16 = tid & 15, r16 = tid >> 4;     // index rows: 16-byte chunk, row slot 0..15
+    const int gi = r16 % H;                        // group of this thread's index rows
+    const int gq = lane >> 2, tq = lane & 3;
+    const int r0 = warp * 16;                      // attention: this warp's 16 tokens
+    const int tps = 128 / H;
+    const float sl2 = P.softmax_scale * kLog2e;
+    const __nv_bfloat16 *qibase = static_cast<const __nv_bfloat16 *>(P.q_idx);
+    float qf[8];
+    int cur_b = -1, it = 0, unit_iter = 0;
+    auto wait_stage = [&](int &slot) -> bool {
+        slot = it % kStages;
+        bool have = !*abort_flag && mbar_wait(&S.full[slot], (it / kStages) & 1, P.status);
+        have = __all_sync(0xffffffffu, have);
+        ++it;
+        if (!have) *abort_flag = 1;
+        return have;
+    };
+    auto release_stage = [&](int slot) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.empty[slot]);
+    };
+
+    // Top-k of sequence b for every group (warp per group), then one
+    // attention item per (group, kept block) published to the global queue.
+    auto topk_and_publish = [&](int b) {
+        __threadfence();                           // other CTAs' scores of b are visible
+        const int L = P.lens[b];
+        const int nb = (L + kBlock - 1) / kBlock;
+        const int own = nb - 1;                    // decode: the query is token L-1
+        const int n_kept = min(K, nb);
+        unsigned long long *keys = reinterpret_cast<unsigned long long *>(&S.om[warp][0][0]);
+        int *sel = reinterpret_cast<int *>(&S.om[warp][2][0]);
+        for (int g = warp; g < H; g += kWarps) {
+            const long long bg = static_cast<long long>(b) * H + g;
+            const float *sc = P.scores + bg * nbs;
+            int n = 0;
+            if (nb <= K) {
+                for (int q = lane; q < nb; q += 32) sel[q] = q;
+                n = nb;
+            } else {
+                const int m = K - 1;
+                warp_select([&](int jj) { return topk_key(__ldcg(sc + jj), jj); }, 0, own, m, lane, keys);
+                for (int q = lane; q < m; q += 32) sel[q] = topk_key_id(keys[q]);
+                if (lane == 0) sel[m] = own;
+                n = K;
+            }
+            __syncwarp();
+            emit_sorted(sel, n, sc, K, lane, P.ids + bg * K, P.out_scores + bg * K);
+            __syncwarp();
+        }
+        __threadfence();
+        cbar();
+        const int count = H * n_kept;
+        if (tid == 0) S.bcast[1] = atomicAdd(P.ctr + 1, count);
+        cbar();
+        const int base = S.bcast[1];
+        for (int e = tid; e < count; e += kConsumers)
+            P.aq_item[base + e] = (b * H + e / n_kept) * K + e % n_kept;
+        __threadfence();
+        for (int e = tid; e < count; e += kConsumers)
+            *reinterpret_cast<volatile int *>(P.aq_flag + base + e) = 1;
+        __threadfence();
+        cbar();
+        if (tid == 0) atomicAdd(P.ctr + 3, count);
+    };
+
+    for (int n = 0;; ++n) {
+        const int wslot = n % kQueue;
+        bool have = !*abort_flag && mbar_wait(&S.wq_full[wslot], (n / kQueue) & 1, P.status);
+        have = __all_sync(0xffffffffu, have);
+        if (!have) { *abort_flag = 1; break; }
+        const int4 w = S.wq[wslot];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.wq_empty[wslot]);
+        if (w.x == kWorkEnd) break;
+
+        if (w.x == kWorkIndex) {
+            // ---- index unit: block j of sequence b, every group
+            const int b = w.y, j = w.z, ntok = w.w;
+            if (b != cur_b) {
+                const uint4 qv = *reinterpret_cast<const uint4 *>(qibase + ((long long)b * H + gi) * kDim + c16 * 8);
+                qf[0] = bf16lo(qv.x); qf[1] = bf16hi(qv.x);
+                qf[2] = bf16lo(qv.y); qf[3] = bf16hi(qv.y);
+                qf[4] = bf16lo(qv.z); qf[5] = bf16hi(qv.z);
+                qf[6] = bf16lo(qv.w); qf[7] = bf16hi(qv.w);
+                cur_b = b;
+            }
+            float runmax = -INFINITY;
+            for (int t0 = 0; t0 < ntok; t0 += tps) {
+                const int rows_valid = min(tps, ntok - t0) * H;
+                int slot;
+                if (wait_stage(slot)) {
+                    const uint8_t *sb = S.ring[slot];
+#pragma unroll
+                    for (int pass = 0; pass < 8; ++pass) {
+                        const int row = r16 + 16 * pass;
+                        const uint4 kv = *reinterpret_cast<const uint4 *>(sb + row * 256 + c16 * 16);
+                        float d = qf[0] * bf16lo(kv.x);
+                        d = fmaf(qf[1], bf16hi(kv.x), d);
+                        d = fmaf(qf[2], bf16lo(kv.y), d);
+                        d = fmaf(qf[3], bf16hi(kv.y), d);
+                        d = fmaf(qf[4], bf16lo(kv.z), d);
+                        d = fmaf(qf[5], bf16hi(kv.z), d);
+                        d = fmaf(qf[6], bf16lo(kv.w), d);
+                        d = fmaf(qf[7], bf16hi(kv.w), d);
+                        d += __shfl_xor_sync(0xffffffffu, d, 8);
+                        d += __shfl_xor_sync(0xffffffffu, d, 4);
+                        d += __shfl_xor_sync(0xffffffffu, d, 2);
+                        d += __shfl_xor_sync(0xffffffffu, d, 1);
+                        if (row < rows_valid) runmax = fmaxf(runmax, d);
+                    }
+                    release_stage(slot);
+                }
+            }
+            const int par = unit_iter++ & 1;
+            if (c16 == 0) S.red[par][r16] = runmax;
+            cbar();
+            if (tid < H && !*abort_flag) {
+                float m = -INFINITY;
+                for (int r = tid; r < 16; r += H) m = fmaxf(m, S.red[par][r]);
+                P.scores[((long long)b * H + tid) * nbs + j] = m;
+                __threadfence();
+            }
+            cbar();
+            if (tid == 0) {
+                const int L = P.lens[b];
+                const int done = atomicAdd(P.seq_done + b, 1) + 1;
+                S.bcast[0] = done == (L + kBlock - 1) / kBlock;
+            }
+            cbar();
+            if (S.bcast[0] && !*abort_flag) topk_and_publish(b);
+            continue;
+        }
+
+        // ---- attention item: kept block j (slot s) of (sequence b, group g)
+        const int payload = w.y, j = w.z;
+        const int bg = payload / K, s = payload % K;
+        const int b = bg / H, g = bg % H;
+        const int L = P.lens[b];
+        const int nvalid = min(kBlock, L - j * kBlock);
+        const int n_kept = min(K, (L + kBlock - 1) / kBlock);
+        uint32_t qb[8][2];                          // Q^T of the group's heads (zero past G)
+        {
+            const __nv_bfloat16 *qh = static_cast<const __nv_bfloat16 *>(P.q) +
+                                      ((long long)b * P.H_q + (long long)g * G + gq) * kDim + tq * 2;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                qb[kk][0] = gq < G ? *reinterpret_cast<const uint32_t *>(qh + kk * 16) : 0u;
+                qb[kk][1] = gq < G ? *reinterpret_cast<const uint32_t *>(qh + kk * 16 + 8) : 0u;
+            }
+        }
+        int sk, sv;
+        const bool hk = wait_stage(sk);
+        const bool hv = wait_stage(sv);
+        float m2[2] = {-INFINITY, -INFINITY}, l2[2] = {0.f, 0.f};
+        float acc[8][4];
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
+        if (hk && hv) {
+            const uint32_t kb = smem_u32(S.ring[sk]), vb = smem_u32(S.ring[sv]);
+            if (nvalid < r0 + 16) {
+                // value rows past the query: weight 0, but padding may hold NaN
+                for (int e = lane; e < 16 * 16; e += 32) {
+                    const int r = r0 + (e >> 4), c = e & 15;
+                    if (r >= nvalid)
+                        *reinterpret_cast<uint4 *>(S.ring[sv] + (c >> 3) * 16384 + r * 128 + (c & 7) * 16) =
+                            make_uint4(0, 0, 0, 0);
+                }
+                __syncwarp();
+            }
+            float sv4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const int chunk = ((kk & 3) << 1) | (lane >> 4);
+                uint32_t a[4];
+                ldsm_x4(kb + (kk >> 2) * 16384 + swz128(r0 + (lane & 15), chunk), a[0], a[1], a[2], a[3]);
+                mma_bf16_16816(sv4, a, qb[kk][0], qb[kk][1]);
+            }
+            float p[4];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const float x0 = r0 + gq < nvalid ? sv4[c] * sl2 : -INFINITY;
+                const float x1 = r0 + gq + 8 < nvalid ? sv4[2 + c] * sl2 : -INFINITY;
+                float cm = fmaxf(x0, x1);
+                cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 4));
+                cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 8));
+                cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 16));
+                const float mref = cm == -INFINITY ? 0.f : cm;
+                p[c] = exp2f(x0 - mref);
+                p[2 + c] = exp2f(x1 - mref);
+                m2[c] = cm;
+                l2[c] = p[c] + p[2 + c];
+            }
+            const uint32_t pb0 = movmatrix_t(pack_bf16x2(p[0], p[1]));
+            const uint32_t pb1 = movmatrix_t(pack_bf16x2(p[2], p[3]));
+            const int mi = lane >> 3;
+            const int r = r0 + ((mi >> 1) << 3) + (lane & 7);
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                const int d = mt * 16 + ((mi & 1) << 3);
+                uint32_t a[4];
+                ldsm_x4_t(vb + (d >> 6) * 16384 + swz128(r, (d & 63) >> 3), a[0], a[1], a[2], a[3]);
+                mma_bf16_16816(acc[mt], a, pb0, pb1);
+            }
+            fence_proxy_async_smem();              // zeroed rows before the next TMA write
+        }
+        if (hk) release_stage(sk);
+        if (hv) release_stage(sv);
+        // per-warp partials to shared memory: heads 2tq + c
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            float l = l2[c];
+            l += __shfl_xor_sync(0xffffffffu, l, 4);
+            l += __shfl_xor_sync(0xffffffffu, l, 8);
+            l += __shfl_xor_sync(0xffffffffu, l, 16);
+            const int h = 2 * tq + c;
+            if (gq == 0) { S.mw[warp][h] = m2[c]; S.lw[warp][h] = l; }
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                S.om[warp][h][mt * 16 + gq] = acc[mt][c];
+                S.om[warp][h][mt * 16 + gq + 8] = acc[mt][2 + c];
+            }
+        }
+        cbar();
+        // merge the 8 warps into this block's record
+        float *rec0 = P.partials + (static_cast<long long>(bg) * K + s) * 8 * kRec;
+        for (int e = tid; e < G * kDim; e += kConsumers) {
+            const int h = e / kDim, d = e % kDim;
+            float M = -INFINITY;
+#pragma unroll
+            for (int w8 = 0; w8 < kWarps; ++w8) M = fmaxf(M, S.mw[w8][h]);
+            const float Mr = M == -INFINITY ? 0.f : M;
+            float o = 0.f, l = 0.f;
+#pragma unroll
+            for (int w8 = 0; w8 < kWarps; ++w8) {
+                const float f = exp2f(S.mw[w8][h] - Mr);
+                o += S.om[w8][h][d] * f;
+                l += S.lw[w8][h] * f;
+            }
+            float *rec = rec0 + h * kRec;
+            rec[4 + d] = o;
+            if (d == 0) { rec[0] = M; rec[1] = l; }
+        }
+        __threadfence();
+        cbar();
+        if (tid == 0) {
+            const int t = atomicAdd(P.tickets + bg, 1);
+            S.bcast[0] = t == n_kept - 1;
+            __threadfence();
+        }
+        cbar();
+        if (S.bcast[0] && !*abort_flag) {
+            // last block of (b, g): merge its kept blocks' records, write out
+            __threadfence();
+            const float *base = P.partials + static_cast<long long>(bg) * K * 8 * kRec;
+            __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(P.out) + ((long long)b * P.H_q + (long long)g * G) * kDim;
+            for (int e = tid; e < G * kDim; e += kConsumers) {
+                const int h = e / kDim, d = e % kDim;
+                float M = -INFINITY;
+                for (int q = 0; q < n_kept; ++q) M = fmaxf(M, __ldcg(base + (q * 8 + h) * kRec));
+                const float Mr = M == -INFINITY ? 0.f : M;
+                float o = 0.f, l = 0.f;
+                for (int q = 0; q < n_kept; ++q) {
+                    const float *rec = base + (q * 8 + h) * kRec;
+                    const float f = exp2f(__ldcg(rec) - Mr);
+                    o += __ldcg(rec + 4 + d) * f;
+                    l += __ldcg(rec + 1) * f;
+                }
+                out[e] = __float2bfloat16(o / l);
+            }
+        }
+        cbar();                                     // om, mw, lw and bcast are reused
+    }
+}
+
+}  // namespace
+
+size_t decode_fused_layout(int B, int H_q, int H_kv, int K, int max_kv_len, DecodeFusedLayout *L) {
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    const size_t nb_max = score_stride((max_kv_len + kBlock - 1) / kBlock);
+    const size_t items = static_cast<size_t>(B) * H_kv * K;
+    size_t o = kWsHeaderBytes;
+    L->scores = o;   o += up(static_cast<size_t>(B) * H_kv * nb_max * 4);
+    L->partials = o; o += up(items * 8 * kRec * 4);
+    L->zero_lo = o;                                 // cleared per call: counters and flags
+    L->seq_done = o; o += up(static_cast<size_t>(B) * 4);
+    L->tickets = o;  o += up(static_cast<size_t>(B) * H_kv * 4);
+    L->aq_flag = o;  o += up(items * 4);
+    L->zero_hi = o;
+    L->aq_item = o;  o += up(items * 4);
+    L->total = o;
+    (void)H_q;
+    return o;
+}
+
+cudaError_t launch_decode_fused(const DecodeFusedArgs &a, cudaStream_t s) {
+    static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory budget");
+    CUtensorMap tk, tv;
+    if (!encode_kv_tensor_map(&tk, a.k_cache, a.H_kv, a.kv.capacity) ||
+        !encode_kv_tensor_map(&tv, a.v_cache, a.H_kv, a.kv.capacity))
+        return cudaErrorInvalidValue;
+    const size_t smem = sizeof(Smem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    TraceScope trace(s, "decode_fused_step");
+    DecodeFusedArgs args = a;
+    void *params[] = {&tk, &tv, &args};
+    // Cooperative: every CTA resident at once (they hand work to each other).
+    return cudaLaunchCooperativeKernel(reinterpret_cast<void *>(decode_fused_kernel),
+                                       dim3(device_sm_count()), dim3(kThreads), params, smem, s);
+}
+
+}  // namespace msa

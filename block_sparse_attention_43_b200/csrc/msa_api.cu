@@ -453,6 +453,69 @@ msa_status_t msa_sparse_attention_backward(const msa_shape_t *shape, const void 
     return launch_attn_bwd(a, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
 }
 
+// The fused decode step takes one bf16 index key per group, q_len 1 and
+// groups of at most 8 heads (one n8 tile of the attention products).
+static msa_status_t check_decode_step(const msa_shape_t *s) {
+    msa_status_t st = check_shape(s);
+    if (st != MSA_OK) return st;
+    if (s->q_len != 1 || index_heads(s) != s->num_kv_heads ||
+        s->index_key_format != MSA_INDEX_KEYS_BF16 || s->num_q_heads / s->num_kv_heads > 8)
+        return MSA_ERR_UNSUPPORTED;
+    return MSA_OK;
+}
+
+static DecodeFusedLayout decode_step_layout(const msa_shape_t *s) {
+    DecodeFusedLayout L;
+    decode_fused_layout(s->batch, s->num_q_heads, s->num_kv_heads, s->top_k, s->max_kv_len, &L);
+    return L;
+}
+
+size_t msa_decode_step_workspace_size(const msa_shape_t *shape) {
+    if (check_decode_step(shape) != MSA_OK) return 0;
+    return decode_step_layout(shape).total;
+}
+
+msa_status_t msa_decode_step(const msa_shape_t *shape, const void *q_idx, const void *k_idx,
+                             const void *q, const void *k_cache, const void *v_cache,
+                             const int32_t *lens, const int64_t *kv_offsets, float softmax_scale,
+                             int32_t *block_ids, float *block_scores, void *out, void *workspace,
+                             size_t workspace_bytes, msa_stream_t stream) {
+    msa_status_t st = check_decode_step(shape);
+    if (st != MSA_OK) return st;
+    if (!q_idx || !k_idx || !q || !k_cache || !v_cache || !lens || !kv_offsets || !block_ids ||
+        !block_scores || !out)
+        return MSA_ERR_INVALID_ARG;
+    if (!(softmax_scale == softmax_scale) || softmax_scale == INFINITY || softmax_scale == -INFINITY)
+        return MSA_ERR_INVALID_ARG;
+    if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(q) || !aligned16(k_cache) ||
+        !aligned16(v_cache) || !aligned16(out))
+        return MSA_ERR_MISALIGNED;
+    const DecodeFusedLayout L = decode_step_layout(shape);
+    if ((st = check_ws(workspace, workspace_bytes, L.total)) != MSA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    // status word and claim counters (header), then the per-call flags
+    if (cudaMemsetAsync(ws, 0, kWsHeaderBytes, s) != cudaSuccess ||
+        cudaMemsetAsync(ws + L.zero_lo, 0, L.zero_hi - L.zero_lo, s) != cudaSuccess)
+        return MSA_ERR_CUDA;
+    DecodeFusedArgs a;
+    a.q_idx = q_idx; a.k_idx = k_idx; a.q = q; a.k_cache = k_cache; a.v_cache = v_cache;
+    a.lens = lens; a.kv = packed_map(shape, kv_offsets);
+    a.ids = block_ids; a.out_scores = block_scores; a.out = out;
+    a.status = reinterpret_cast<int *>(ws);
+    a.ctr = reinterpret_cast<int *>(ws + 64);
+    a.scores = reinterpret_cast<float *>(ws + L.scores);
+    a.partials = reinterpret_cast<float *>(ws + L.partials);
+    a.seq_done = reinterpret_cast<int *>(ws + L.seq_done);
+    a.tickets = reinterpret_cast<int *>(ws + L.tickets);
+    a.aq_item = reinterpret_cast<int *>(ws + L.aq_item);
+    a.aq_flag = reinterpret_cast<int *>(ws + L.aq_flag);
+    a.B = shape->batch; a.H_q = shape->num_q_heads; a.H_kv = shape->num_kv_heads;
+    a.K = shape->top_k; a.nb_max = nb_max_of(shape); a.max_kv_len = shape->max_kv_len;
+    a.softmax_scale = softmax_scale;
+    return launch_decode_fused(a, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+}
+
 msa_status_t msa_read_device_status(const void *workspace, msa_stream_t stream) {
     if (!workspace) return MSA_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -202,6 +202,33 @@ MSA_API msa_status_t msa_sparse_attention_backward(const msa_shape_t *shape, con
                                                    float *dv, void *workspace,
                                                    size_t workspace_bytes, msa_stream_t stream);
 
+/* One whole decode step in a single persistent launch: the index branch
+ * (scores, block max-pool, top-k with the own block forced) and the sparse
+ * branch over the kept blocks, for q_len == 1.  Results are those of
+ * msa_index_topk followed by msa_sparse_attention on the same inputs (same
+ * selection; the output within the attention tolerance, its partial sums
+ * being combined in another order).  The top-k and attention work of a
+ * sequence starts as soon as its own index scores are done, overlapping the
+ * index streaming of the later sequences (MSA's decode cost is that
+ * streaming: "百万token上下文提速近10倍..." section 四).
+ * Requirements on top of the shape rules: q_len == 1, one bf16 index key per
+ * group (num_index_heads == num_kv_heads or 0, index_key_format BF16), and
+ * num_q_heads / num_kv_heads <= 8; otherwise MSA_ERR_UNSUPPORTED.  The
+ * launch is cooperative (one CTA per SM, all resident); it is not meant to
+ * share the GPU with another kernel running at the same time.
+ *   q_idx, k_idx, lens, kv_offsets, block_ids, block_scores: as msa_index_topk
+ *   q, k_cache, v_cache, softmax_scale, out: as msa_sparse_attention
+ *   workspace    device, >= msa_decode_step_workspace_size(shape) bytes,
+ *                256-byte aligned; its first word is the device status word */
+MSA_API size_t msa_decode_step_workspace_size(const msa_shape_t *shape);
+MSA_API msa_status_t msa_decode_step(const msa_shape_t *shape, const void *q_idx,
+                                     const void *k_idx, const void *q, const void *k_cache,
+                                     const void *v_cache, const int32_t *lens,
+                                     const int64_t *kv_offsets, float softmax_scale,
+                                     int32_t *block_ids, float *block_scores, void *out,
+                                     void *workspace, size_t workspace_bytes,
+                                     msa_stream_t stream);
+
 /* Paged caches (a block-table layout for serving): the index keys, keys and
  * values of all sequences live in pools of 128-token pages, [kv_capacity,
  * H_kv, dim] with page p = rows p*128 .. p*128+127, and block j of sequence b

@@ -136,3 +136,20 @@ def test_index_variant_shapes_are_checked(m):
         == 256 + cap * 8 * 128 * 2
     assert m.msa_index_topk_workspace_size(
         _shape(m, q_len=64, index_key_format=m.INDEX_KEYS_FP8_SHARED)) == 256 + cap * 128 * 2
+
+
+def test_decode_step_rejects_unsupported_shapes(m):
+    """q_len > 1, groups of 16 heads, fewer index heads than groups: the
+    workspace query returns 0 and the call returns MSA_ERR_UNSUPPORTED."""
+    for kw in (dict(q_len=2), dict(num_q_heads=32), dict(num_index_heads=1)):
+        base = dict(batch=1, q_len=1, max_kv_len=1000, num_q_heads=16, num_kv_heads=2, top_k=4,
+                    kv_capacity=1000)
+        base.update(kw)
+        s = m.make_shape(**base)
+        assert m.msa_decode_step_workspace_size(s) == 0
+        fake = [0x1000] * 7
+        assert m.lib.msa_decode_step(ctypes.byref(s), *fake, 0.1, 0x1000, 0x1000, 0x1000,
+                                     0x100000, 1 << 40, None) == 2
+    ok = m.make_shape(batch=3, q_len=1, max_kv_len=1000, num_q_heads=16, num_kv_heads=2,
+                      top_k=4, kv_capacity=3000)
+    assert m.msa_decode_step_workspace_size(ok) > 256
