@@ -16,15 +16,17 @@
 //   - the CTA that finishes a sequence's last unit runs that sequence's top-k
 //     (one warp per group, the warp selection of topk.cu) and publishes one
 //     attention item per (group, kept block);
-//   - between index units a CTA takes published attention items: the block's
-//     K/V tiles (TMA, 128-byte swizzle), S^T = K Q^T and O^T = V^T P^T on
-//     mma.sync for the group's heads, a partial (max, sum, O) per kept block;
-//     the CTA finishing a (sequence, group)'s last block merges its partials
-//     and writes the output.
-// Attention items are claimed with a compare-and-swap only while the claim
-// index is below the published count, so a claimed item is either published
-// or about to be by a CTA inside its (wait-free) publishing step; every other
-// wait is bounded.
+//   - between index units a CTA takes published attention items, one per
+//     (sequence, group): the K/V tiles of its kept blocks (TMA, 128-byte
+//     swizzle) stream through the same ring, S^T = K Q^T and O^T = V^T P^T
+//     run on mma.sync for the group's heads with a running softmax across
+//     the blocks, and the CTA writes the group's output itself (no partial
+//     records, no merge across CTAs).
+// An attention item is claimed (one atomicAdd) only while the claim counter
+// is below the published count; a claim that overtakes its publisher stays
+// pending while the CTA streams more index units.  Once a CTA has no index
+// unit left it waits for its claimed item, which the CTA that finishes that
+// sequence's index scores publishes.  Every wait is bounded.
 #include "msa_device.cuh"
 #include "msa_internal.h"
 #include "topk_warp.cuh"
@@ -39,10 +41,9 @@ constexpr int kStages = 5;
 constexpr int kStageBytes = 32768;
 constexpr int kQueue = 4;
 constexpr int kMaxBatch = 4096;
-constexpr int kRec = 132;                     // partial record per head: m, l, 2 pad, O[128]
 constexpr float kLog2e = 1.4426950408889634f;
 
-enum { kWorkIndex = 0, kWorkAttn = 1, kWorkEnd = 2 };
+enum { kWorkIndex = 0, kWorkAttn = 1, kWorkSync = 2, kWorkEnd = 3 };
 
 struct Smem {
     uint8_t ring[kStages][kStageBytes];       // index-key stages / K and V tiles of a block
@@ -55,6 +56,7 @@ struct Smem {
     int prefix[kMaxBatch + 1];
     float red[2][16];
     int bcast[2];
+    unsigned long long topk_req[2];           // (checkpoint << 32) | sequence, by checkpoint parity
     int total_attn;
     int abort_flag;
 };
@@ -64,6 +66,14 @@ __device__ __forceinline__ bool seq_valid(const DecodeFusedArgs &P, int b, int L
 }
 
 __device__ __forceinline__ int ld_volatile(const int *p) { return *reinterpret_cast<const volatile int *>(p); }
+
+// Device-scope add that publishes this thread's earlier writes and, for the
+// thread that sees the final count, acquires everyone else's.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int *p, int v) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
 
 __device__ __forceinline__ unsigned long long now_ns() {
     unsigned long long t;
@@ -107,6 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&S.wq_empty[i], kWarps);
         }
         mbar_init(&S.cbar, kConsumers);
+        S.topk_req[0] = S.topk_req[1] = ~0ull;
         S.abort_flag = 0;
         fence_mbar_init();
     }
@@ -120,7 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (seq_valid(P, b, L)) {
                 const int nb = (L + kBlock - 1) / kBlock;
                 sum += nb;
-                items += H * min(K, nb);
+                items += H;
             } else if (blockIdx.x == 0) {
                 // rejected sequence: -1 / -inf selection, NaN output, status word
                 set_status(P.status, kStatusBadLens);
@@ -180,77 +191,97 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++it;
             return true;
         };
-        // Claims attention item h when h < published; returns -1 if none is
-        // available now, -2 when every item has been claimed.
-        auto try_claim = [&]() -> int {
-            int h = ld_volatile(P.ctr + 2);
-            while (true) {
-                if (h >= total_attn) return -2;
-                if (h >= ld_volatile(P.ctr + 3)) return -1;
-                const int prev = atomicCAS(P.ctr + 2, h, h + 1);
-                if (prev == h) return h;
-                h = prev;
-            }
-        };
+        // Work claiming.  Attention items are claimed with one atomicAdd
+        // (never a compare-and-swap loop, which a hundred polling CTAs turn
+        // into a serial storm), and only while the claim counter is below the
+        // published count; a claim may still overtake the publisher that
+        // owns the item, so the item stays pending (this CTA goes on
+        // streaming index units) until its flag is set.  The next index unit
+        // and the counters are fetched one unit ahead, so their latency hides
+        // behind the unit in flight.
+        int *const c_unit = P.ctr, *const c_claim = P.ctr + 2 * kCtrStride;
+        int *const c_pub = P.ctr + 3 * kCtrStride;
+        int pending = -1, pending_flag = 0;
+        bool attn_left = total_attn > 0;
+        int u_next = atomicAdd(c_unit, 1);
+        int seen_claim = 0, seen_pub = 0;
         const unsigned long long t0 = now_ns();
         while (ok) {
-            int item = -1;
+            if (pending < 0 && attn_left) {
+                if (!index_left) seen_claim = ld_volatile(c_claim);
+                if (seen_claim >= total_attn) {
+                    attn_left = false;
+                } else if (!index_left || seen_claim < seen_pub) {
+                    const int h = atomicAdd(c_claim, 1);
+                    if (h >= total_attn) attn_left = false;
+                    else { pending = h; pending_flag = 0; }
+                    seen_claim = h + 1;
+                }
+            }
+            if (pending >= 0 && (!index_left || pending_flag != 0)) {
+                // Attention item: its flag is set, or will be once the index
+                // units of its sequence are done.  Before waiting, let this
+                // CTA's consumers pass a checkpoint: the top-k that publishes
+                // the item may be theirs to run.
+                const int item = pending;
+                pending = -1;
+                if (ld_volatile(P.aq_flag + item) == 0) {
+                    if (!push(make_int4(kWorkSync, 0, 0, 0))) { ok = false; break; }
+                    while (ld_volatile(P.aq_flag + item) == 0) {
+                        if (*abort_flag || now_ns() - t0 > kWaitNs) { set_status(P.status, kStatusTimeout); ok = false; break; }
+                        __nanosleep(128);
+                    }
+                    if (!ok) break;
+                }
+                __threadfence();
+                const int bg = __ldcg(P.aq_item + item);
+                const int b = bg / H, g = bg % H;
+                const int nb = (P.lens[b] + kBlock - 1) / kBlock;
+                const int n_kept = min(K, nb);
+                if (!push(make_int4(kWorkAttn, bg, n_kept, 0))) { ok = false; break; }
+                // K and V tiles of every kept block, the next id loaded ahead
+                const int32_t *idrow = P.ids + static_cast<long long>(bg) * K;
+                int jn = __ldcg(idrow);
+                for (int sl = 0; sl < n_kept && ok; ++sl) {
+                    const int j = jn;
+                    if (sl + 1 < n_kept) jn = __ldcg(idrow + sl + 1);
+                    const int tok = static_cast<int>(kv_block_row(P.kv, b, j, P.status));
+                    int sk, sv;
+                    if (!stage(sk)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&S.full[sk], kStageBytes);
+                    tma_load_3d(S.ring[sk], &tmK, 0, g, tok, &S.full[sk]);
+                    tma_load_3d(S.ring[sk] + 16384, &tmK, 64, g, tok, &S.full[sk]);
+                    if (!stage(sv)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&S.full[sv], kStageBytes);
+                    tma_load_3d(S.ring[sv], &tmV, 0, g, tok, &S.full[sv]);
+                    tma_load_3d(S.ring[sv] + 16384, &tmV, 64, g, tok, &S.full[sv]);
+                }
+                continue;
+            }
             if (index_left) {
-                item = try_claim();
-                if (item < 0) {
-                    const int u = atomicAdd(P.ctr, 1);
-                    if (u >= U) { index_left = false; continue; }
-                    int b, j;
-                    unit_of(S.prefix, P.B, u, b, j);
-                    const int L = P.lens[b];
-                    const int ntok = min(kBlock, L - j * kBlock);
-                    if (!push(make_int4(kWorkIndex, b, j, ntok))) { ok = false; break; }
-                    const long long t_first = kv_block_row(P.kv, b, j, P.status);
-                    for (int t0s = 0; t0s < ntok; t0s += tps) {
-                        int slot;
-                        if (!stage(slot)) { ok = false; break; }
-                        const uint32_t bytes = static_cast<uint32_t>(min(tps, ntok - t0s)) * H * kDim * 2;
-                        mbar_arrive_expect_tx(&S.full[slot], bytes);
-                        bulk_g2s(S.ring[slot], kbase + (t_first + t0s) * H * kDim, bytes, &S.full[slot], pol);
-                    }
-                    continue;
+                const int u = u_next;
+                if (u >= U) { index_left = false; continue; }
+                u_next = atomicAdd(c_unit, 1);
+                // read now, used at the next pass of the loop
+                if (pending >= 0) pending_flag = ld_volatile(P.aq_flag + pending);
+                else if (attn_left) { seen_claim = ld_volatile(c_claim); seen_pub = ld_volatile(c_pub); }
+                int b, j;
+                unit_of(S.prefix, P.B, u, b, j);
+                const int L = P.lens[b];
+                const int ntok = min(kBlock, L - j * kBlock);
+                if (!push(make_int4(kWorkIndex, b, j, ntok))) { ok = false; break; }
+                const long long t_first = kv_block_row(P.kv, b, j, P.status);
+                for (int t0s = 0; t0s < ntok; t0s += tps) {
+                    int slot;
+                    if (!stage(slot)) { ok = false; break; }
+                    const uint32_t bytes = static_cast<uint32_t>(min(tps, ntok - t0s)) * H * kDim * 2;
+                    mbar_arrive_expect_tx(&S.full[slot], bytes);
+                    bulk_g2s(S.ring[slot], kbase + (t_first + t0s) * H * kDim, bytes, &S.full[slot], pol);
                 }
-            } else {
-                item = try_claim();
-                if (item == -2) break;
-                if (item == -1) {
-                    if (*abort_flag || now_ns() - t0 > kWaitNs) {
-                        set_status(P.status, kStatusTimeout);
-                        ok = false;
-                        break;
-                    }
-                    __nanosleep(256);
-                    continue;
-                }
+                continue;
             }
-            // Attention item: its flag is set, or about to be, by a publisher.
-            const unsigned long long tw = now_ns();
-            while (ld_volatile(P.aq_flag + item) == 0) {
-                if (*abort_flag || now_ns() - tw > kWaitNs) { set_status(P.status, kStatusTimeout); ok = false; break; }
-                __nanosleep(64);
-            }
-            if (!ok) break;
-            __threadfence();
-            const int payload = __ldcg(P.aq_item + item);
-            const int bg = payload / K, s = payload % K;
-            const int b = bg / H, g = bg % H;
-            const int j = __ldcg(P.ids + static_cast<long long>(bg) * K + s);
-            if (!push(make_int4(kWorkAttn, payload, j, 0))) { ok = false; break; }
-            const int tok = static_cast<int>(kv_block_row(P.kv, b, j, P.status));
-            int sk, sv;
-            if (!stage(sk)) { ok = false; break; }
-            mbar_arrive_expect_tx(&S.full[sk], kStageBytes);
-            tma_load_3d(S.ring[sk], &tmK, 0, g, tok, &S.full[sk]);
-            tma_load_3d(S.ring[sk] + 16384, &tmK, 64, g, tok, &S.full[sk]);
-            if (!stage(sv)) { ok = false; break; }
-            mbar_arrive_expect_tx(&S.full[sv], kStageBytes);
-            tma_load_3d(S.ring[sv], &tmV, 0, g, tok, &S.full[sv]);
-            tma_load_3d(S.ring[sv] + 16384, &tmV, 64, g, tok, &S.full[sv]);
+            if (!attn_left) break;
+            if (*abort_flag || now_ns() - t0 > kWaitNs) { set_status(P.status, kStatusTimeout); ok = false; break; }
         }
         if (!ok) *abort_flag = 1;
         push(make_int4(kWorkEnd, 0, 0, 0));      // best effort: consumers also stop on abort
@@ -293,13 +324,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     // Top-k of sequence b for every group (warp per group), then one
-    // attention item per (group, kept block) published to the global queue.
+    // attention item per group published to the global queue.
     auto topk_and_publish = [&](int b) {
         __threadfence();                           // other CTAs' scores of b are visible
         const int L = P.lens[b];
         const int nb = (L + kBlock - 1) / kBlock;
         const int own = nb - 1;                    // decode: the query is token L-1
-        const int n_kept = min(K, nb);
         unsigned long long *keys = reinterpret_cast<unsigned long long *>(&S.om[warp][0][0]);
         int *sel = reinterpret_cast<int *>(&S.om[warp][2][0]);
         for (int g = warp; g < H; g += kWarps) {
@@ -322,18 +352,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __threadfence();
         cbar();
-        const int count = H * n_kept;
-        if (tid == 0) S.bcast[1] = atomicAdd(P.ctr + 1, count);
+        const int count = H;                       // one attention item per group
+        if (tid == 0) S.bcast[1] = atomicAdd(P.ctr + kCtrStride, count);
         cbar();
         const int base = S.bcast[1];
-        for (int e = tid; e < count; e += kConsumers)
-            P.aq_item[base + e] = (b * H + e / n_kept) * K + e % n_kept;
+        for (int e = tid; e < count; e += kConsumers) P.aq_item[base + e] = b * H + e;
         __threadfence();
         for (int e = tid; e < count; e += kConsumers)
             *reinterpret_cast<volatile int *>(P.aq_flag + base + e) = 1;
         __threadfence();
         cbar();
-        if (tid == 0) atomicAdd(P.ctr + 3, count);
+        if (tid == 0) atomicAdd(P.ctr + 3 * kCtrStride, count);
+    };
+
+    // Checkpoints follow a consumer-wide sync, so every consumer thread reads
+    // the same request: a top-k asked for since the previous checkpoint (the
+    // request carries the checkpoint number it is for, and the slots
+    // alternate, so a request written after this read waits for the next).
+    int ck = 0;
+    auto checkpoint = [&]() {
+        const unsigned long long v = *reinterpret_cast<volatile unsigned long long *>(&S.topk_req[ck & 1]);
+        const bool hit = static_cast<int>(v >> 32) == ck;
+        ++ck;
+        if (hit && !*abort_flag) topk_and_publish(static_cast<int>(v & 0xffffffffu));
     };
 
     for (int n = 0;; ++n) {
@@ -344,7 +385,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int4 w = S.wq[wslot];
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.wq_empty[wslot]);
-        if (w.x == kWorkEnd) break;
+        if (w.x == kWorkSync || w.x == kWorkEnd) {
+            cbar();
+            checkpoint();
+            if (w.x == kWorkEnd) break;
+            continue;
+        }
 
         if (w.x == kWorkIndex) {
             // ---- index unit: block j of sequence b, every group
@@ -387,30 +433,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int par = unit_iter++ & 1;
             if (c16 == 0) S.red[par][r16] = runmax;
             cbar();
+            checkpoint();
+            // One thread per group stores the block score and counts it; the
+            // rest of the CTA goes straight on.  The thread that sees the
+            // sequence's last score requests its top-k at the next checkpoint.
             if (tid < H && !*abort_flag) {
                 float m = -INFINITY;
                 for (int r = tid; r < 16; r += H) m = fmaxf(m, S.red[par][r]);
                 P.scores[((long long)b * H + tid) * nbs + j] = m;
-                __threadfence();
+                const int target = H * ((P.lens[b] + kBlock - 1) / kBlock);
+                if (atom_add_acq_rel_gpu(P.seq_done + b, 1) + 1 == target)
+                    *reinterpret_cast<volatile unsigned long long *>(&S.topk_req[ck & 1]) =
+                        (static_cast<unsigned long long>(ck) << 32) | static_cast<unsigned>(b);
             }
-            cbar();
-            if (tid == 0) {
-                const int L = P.lens[b];
-                const int done = atomicAdd(P.seq_done + b, 1) + 1;
-                S.bcast[0] = done == (L + kBlock - 1) / kBlock;
-            }
-            cbar();
-            if (S.bcast[0] && !*abort_flag) topk_and_publish(b);
             continue;
         }
 
-        // ---- attention item: kept block j (slot s) of (sequence b, group g)
-        const int payload = w.y, j = w.z;
-        const int bg = payload / K, s = payload % K;
+        // ---- attention item: every kept block of (sequence b, group g).
+        // Warp w takes tokens 16w..16w+15 of each block, with a running
+        // (max, sum, O^T) per head across the blocks; the blocks arrive in
+        // ascending id order, so only the last one (the own block) is partial.
+        const int bg = w.y, n_kept = w.z;
         const int b = bg / H, g = bg % H;
         const int L = P.lens[b];
-        const int nvalid = min(kBlock, L - j * kBlock);
-        const int n_kept = min(K, (L + kBlock - 1) / kBlock);
+        const int last_valid = L - ((L - 1) / kBlock) * kBlock;
         uint32_t qb[8][2];                          // Q^T of the group's heads (zero past G)
         {
             const __nv_bfloat16 *qh = static_cast<const __nv_bfloat16 *>(P.q) +
@@ -421,16 +467,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 qb[kk][1] = gq < G ? *reinterpret_cast<const uint32_t *>(qh + kk * 16 + 8) : 0u;
             }
         }
-        int sk, sv;
-        const bool hk = wait_stage(sk);
-        const bool hv = wait_stage(sv);
         float m2[2] = {-INFINITY, -INFINITY}, l2[2] = {0.f, 0.f};
         float acc[8][4];
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
-        if (hk && hv) {
+        for (int sl = 0; sl < n_kept; ++sl) {
+            int sk, sv;
+            const bool hk = wait_stage(sk);
+            const bool hv = wait_stage(sv);
+            if (!(hk && hv)) break;
+            const int nvalid = sl == n_kept - 1 ? last_valid : kBlock;
             const uint32_t kb = smem_u32(S.ring[sk]), vb = smem_u32(S.ring[sv]);
             if (nvalid < r0 + 16) {
                 // value rows past the query: weight 0, but padding may hold NaN
@@ -440,15 +488,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         *reinterpret_cast<uint4 *>(S.ring[sv] + (c >> 3) * 16384 + r * 128 + (c & 7) * 16) =
                             make_uint4(0, 0, 0, 0);
                 }
+                fence_proxy_async_smem();          // before the next TMA write of this stage
                 __syncwarp();
             }
             float sv4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const int chunk = ((kk & 3) << 1) | (lane >> 4);
-                uint32_t a[4];
-                ldsm_x4(kb + (kk >> 2) * 16384 + swz128(r0 + (lane & 15), chunk), a[0], a[1], a[2], a[3]);
-                mma_bf16_16816(sv4, a, qb[kk][0], qb[kk][1]);
+                uint32_t a4[4];
+                ldsm_x4(kb + (kk >> 2) * 16384 + swz128(r0 + (lane & 15), chunk), a4[0], a4[1], a4[2], a4[3]);
+                mma_bf16_16816(sv4, a4, qb[kk][0], qb[kk][1]);
             }
             float p[4];
 #pragma unroll
@@ -459,11 +508,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 4));
                 cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 8));
                 cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 16));
-                const float mref = cm == -INFINITY ? 0.f : cm;
+                const float mnew = fmaxf(m2[c], cm);
+                const float mref = mnew == -INFINITY ? 0.f : mnew;
+                const float alpha = exp2f(m2[c] - mref);
+                m2[c] = mnew;
                 p[c] = exp2f(x0 - mref);
                 p[2 + c] = exp2f(x1 - mref);
-                m2[c] = cm;
-                l2[c] = p[c] + p[2 + c];
+                l2[c] = l2[c] * alpha + p[c] + p[2 + c];
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                    acc[mt][c] *= alpha;
+                    acc[mt][2 + c] *= alpha;
+                }
             }
             const uint32_t pb0 = movmatrix_t(pack_bf16x2(p[0], p[1]));
             const uint32_t pb1 = movmatrix_t(pack_bf16x2(p[2], p[3]));
@@ -472,14 +528,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
                 const int d = mt * 16 + ((mi & 1) << 3);
-                uint32_t a[4];
-                ldsm_x4_t(vb + (d >> 6) * 16384 + swz128(r, (d & 63) >> 3), a[0], a[1], a[2], a[3]);
-                mma_bf16_16816(acc[mt], a, pb0, pb1);
+                uint32_t a4[4];
+                ldsm_x4_t(vb + (d >> 6) * 16384 + swz128(r, (d & 63) >> 3), a4[0], a4[1], a4[2], a4[3]);
+                mma_bf16_16816(acc[mt], a4, pb0, pb1);
             }
-            fence_proxy_async_smem();              // zeroed rows before the next TMA write
+            release_stage(sk);
+            release_stage(sv);
         }
-        if (hk) release_stage(sk);
-        if (hv) release_stage(sv);
         // per-warp partials to shared memory: heads 2tq + c
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
@@ -496,54 +551,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         cbar();
-        // merge the 8 warps into this block's record
-        float *rec0 = P.partials + (static_cast<long long>(bg) * K + s) * 8 * kRec;
-        for (int e = tid; e < G * kDim; e += kConsumers) {
-            const int h = e / kDim, d = e % kDim;
-            float M = -INFINITY;
-#pragma unroll
-            for (int w8 = 0; w8 < kWarps; ++w8) M = fmaxf(M, S.mw[w8][h]);
-            const float Mr = M == -INFINITY ? 0.f : M;
-            float o = 0.f, l = 0.f;
-#pragma unroll
-            for (int w8 = 0; w8 < kWarps; ++w8) {
-                const float f = exp2f(S.mw[w8][h] - Mr);
-                o += S.om[w8][h][d] * f;
-                l += S.lw[w8][h] * f;
-            }
-            float *rec = rec0 + h * kRec;
-            rec[4 + d] = o;
-            if (d == 0) { rec[0] = M; rec[1] = l; }
-        }
-        __threadfence();
-        cbar();
-        if (tid == 0) {
-            const int t = atomicAdd(P.tickets + bg, 1);
-            S.bcast[0] = t == n_kept - 1;
-            __threadfence();
-        }
-        cbar();
-        if (S.bcast[0] && !*abort_flag) {
-            // last block of (b, g): merge its kept blocks' records, write out
-            __threadfence();
-            const float *base = P.partials + static_cast<long long>(bg) * K * 8 * kRec;
+        if (!*abort_flag) {
+            // merge the 8 warps and write the group's heads
             __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(P.out) + ((long long)b * P.H_q + (long long)g * G) * kDim;
             for (int e = tid; e < G * kDim; e += kConsumers) {
                 const int h = e / kDim, d = e % kDim;
                 float M = -INFINITY;
-                for (int q = 0; q < n_kept; ++q) M = fmaxf(M, __ldcg(base + (q * 8 + h) * kRec));
+#pragma unroll
+                for (int w8 = 0; w8 < kWarps; ++w8) M = fmaxf(M, S.mw[w8][h]);
                 const float Mr = M == -INFINITY ? 0.f : M;
                 float o = 0.f, l = 0.f;
-                for (int q = 0; q < n_kept; ++q) {
-                    const float *rec = base + (q * 8 + h) * kRec;
-                    const float f = exp2f(__ldcg(rec) - Mr);
-                    o += __ldcg(rec + 4 + d) * f;
-                    l += __ldcg(rec + 1) * f;
+#pragma unroll
+                for (int w8 = 0; w8 < kWarps; ++w8) {
+                    const float f = exp2f(S.mw[w8][h] - Mr);
+                    o += S.om[w8][h][d] * f;
+                    l += S.lw[w8][h] * f;
                 }
                 out[e] = __float2bfloat16(o / l);
             }
         }
         cbar();                                     // om, mw, lw and bcast are reused
+        checkpoint();
     }
 }
 
@@ -552,18 +580,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 size_t decode_fused_layout(int B, int H_q, int H_kv, int K, int max_kv_len, DecodeFusedLayout *L) {
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
     const size_t nb_max = score_stride((max_kv_len + kBlock - 1) / kBlock);
-    const size_t items = static_cast<size_t>(B) * H_kv * K;
+    const size_t items = static_cast<size_t>(B) * H_kv;
     size_t o = kWsHeaderBytes;
     L->scores = o;   o += up(static_cast<size_t>(B) * H_kv * nb_max * 4);
-    L->partials = o; o += up(items * 8 * kRec * 4);
     L->zero_lo = o;                                 // cleared per call: counters and flags
+    L->ctr = o;      o += 4 * kCtrStride * 4;
     L->seq_done = o; o += up(static_cast<size_t>(B) * 4);
-    L->tickets = o;  o += up(static_cast<size_t>(B) * H_kv * 4);
     L->aq_flag = o;  o += up(items * 4);
     L->zero_hi = o;
     L->aq_item = o;  o += up(items * 4);
     L->total = o;
     (void)H_q;
+    (void)K;
     return o;
 }
 

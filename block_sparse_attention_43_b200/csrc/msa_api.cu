@@ -494,7 +494,7 @@ msa_status_t msa_decode_step(const msa_shape_t *shape, const void *q_idx, const 
     if ((st = check_ws(workspace, workspace_bytes, L.total)) != MSA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    // status word and claim counters (header), then the per-call flags
+    // status word (header), then the claim counters and per-call flags
     if (cudaMemsetAsync(ws, 0, kWsHeaderBytes, s) != cudaSuccess ||
         cudaMemsetAsync(ws + L.zero_lo, 0, L.zero_hi - L.zero_lo, s) != cudaSuccess)
         return MSA_ERR_CUDA;
@@ -503,11 +503,9 @@ msa_status_t msa_decode_step(const msa_shape_t *shape, const void *q_idx, const 
     a.lens = lens; a.kv = packed_map(shape, kv_offsets);
     a.ids = block_ids; a.out_scores = block_scores; a.out = out;
     a.status = reinterpret_cast<int *>(ws);
-    a.ctr = reinterpret_cast<int *>(ws + 64);
+    a.ctr = reinterpret_cast<int *>(ws + L.ctr);
     a.scores = reinterpret_cast<float *>(ws + L.scores);
-    a.partials = reinterpret_cast<float *>(ws + L.partials);
     a.seq_done = reinterpret_cast<int *>(ws + L.seq_done);
-    a.tickets = reinterpret_cast<int *>(ws + L.tickets);
     a.aq_item = reinterpret_cast<int *>(ws + L.aq_item);
     a.aq_flag = reinterpret_cast<int *>(ws + L.aq_flag);
     a.B = shape->batch; a.H_q = shape->num_q_heads; a.H_kv = shape->num_kv_heads;

@@ -167,6 +167,7 @@ bool encode_q_gather_map(CUtensorMap *map, const void *q, int H_q, long long row
 // src[i] [B][n_new][H_kv][128] -> dst[i] at rows of tokens lens[b] .. + n_new - 1.
 // Whole decode step in one persistent launch (decode_fused.cu): index
 // scores, top-k per (sequence, index head) and sparse attention.
+constexpr int kCtrStride = 32;
 struct DecodeFusedArgs {
     const void *q_idx;      // [B][H_kv][128]
     const void *k_idx;      // [T][H_kv][128]
@@ -181,17 +182,16 @@ struct DecodeFusedArgs {
     int *status;
     // workspace views
     float *scores;          // [B][H_kv][nb_max] block scores
-    float *partials;        // [B][H_kv][K][G][132] per kept block: m, l, pad, O[128]
     int *seq_done;          // [B] index units finished
-    int *tickets;           // [B][H_kv] attention blocks finished
-    int *aq_item;           // [B*H_kv*K] published attention items ((b*H_kv+g)*K + slot)
-    int *aq_flag;           // [B*H_kv*K] 1 once the item above is published
-    int *ctr;               // [0] next index unit, [1] allocated items, [2] next item claimed, [3] published
+    int *aq_item;           // [B*H_kv] published attention items (b*H_kv + g)
+    int *aq_flag;           // [B*H_kv] 1 once the item above is published
+    int *ctr;               // one 128-byte line each (stride kCtrStride ints): next index unit,
+                            // allocated items, next item claimed, items published
     int B, H_q, H_kv, K, nb_max, max_kv_len;
     float softmax_scale;
 };
 struct DecodeFusedLayout {
-    size_t scores, partials, seq_done, tickets, aq_item, aq_flag, zero_lo, zero_hi, total;
+    size_t scores, ctr, seq_done, aq_item, aq_flag, zero_lo, zero_hi, total;
 };
 size_t decode_fused_layout(int B, int H_q, int H_kv, int K, int max_kv_len, DecodeFusedLayout *L);
 cudaError_t launch_decode_fused(const DecodeFusedArgs &a, cudaStream_t s);

@@ -58,7 +58,7 @@ CASES = [
 
 
 @pytest.mark.parametrize("B,lens,H_q,H_kv,top_k", CASES)
-def test_decode_step_small_shapes(msa_lib, oracle_mod, B, lens, H_q, H_kv, top_k):
+def test_decode_step_small_shapes(oracle_mod, B, lens, H_q, H_kv, top_k):
     from synthetic import make_inputs
     w = make_inputs(B=B, Sq=1, lens=lens, H_q=H_q, H_kv=H_kv, top_k=top_k, seed=501 + B,
                     device=DEV, needles=3, amp=4.0)
@@ -66,7 +66,7 @@ def test_decode_step_small_shapes(msa_lib, oracle_mod, B, lens, H_q, H_kv, top_k
 
 
 @pytest.mark.parametrize("name", ["decode_32k", "decode_ragged", "decode_1m"])
-def test_decode_step_named_workloads(msa_lib, oracle_mod, name):
+def test_decode_step_named_workloads(oracle_mod, name):
     """The decode workloads at full size, in the configuration the benchmark
     times, every row compared."""
     from synthetic import make_workload
@@ -74,7 +74,7 @@ def test_decode_step_named_workloads(msa_lib, oracle_mod, name):
     print(name, _run_and_compare(oracle_mod, w))
 
 
-def test_decode_step_padded_cache_with_nan(msa_lib, oracle_mod):
+def test_decode_step_padded_cache_with_nan(oracle_mod):
     """Padded layout with NaN past each length: no padding token may reach a
     score or an output."""
     from synthetic import make_inputs
@@ -87,7 +87,7 @@ def test_decode_step_padded_cache_with_nan(msa_lib, oracle_mod):
     print(_run_and_compare(oracle_mod, w))
 
 
-def test_decode_step_repeat_calls(msa_lib):
+def test_decode_step_repeat_calls():
     """Selection bit-identical on every call; the output may differ only in
     the merge order of the kept blocks, within bf16 rounding."""
     from synthetic import make_inputs
@@ -103,7 +103,7 @@ def test_decode_step_repeat_calls(msa_lib):
         assert (a[2] - eng.out.float()).abs().max().item() <= 2e-2
 
 
-def test_decode_step_bad_lengths(msa_lib, oracle_mod):
+def test_decode_step_bad_lengths(oracle_mod):
     """A length past max_kv_len: that sequence gets -1 / -inf / NaN and the
     status word; the others are still computed correctly."""
     from parity import compare
