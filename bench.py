@@ -1,14 +1,16 @@
 """Benchmark of the MSA hot path on B200: one step = the whole decode path
 (index score + block max-pool, top-k, sparse attention with split-K merge)
 for one batch, through the C ABI; a decode run also times the same decode
-step on the index-branch variants (fewer index heads, shared index keys,
-E4M3 index keys), the sparse branch's backward on the 2k-row prefill, and one
+step as one fused cooperative launch, the decode step on the index-branch
+variants (fewer index heads, shared index keys, E4M3 index keys), the sparse
+branch's backward on the 2k-row prefill, and one
 128k-token prefill (index GEMM + fused top-k, sparse attention) as
 sub-objects.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode_1m]
                     [--impl msa|reference] [--no-cpu-baseline] [--no-e2e]
-                    [--no-prefill] [--no-variants] [--no-backward] [--prefill-steps S]
+                    [--no-prefill] [--no-fused] [--no-variants] [--no-backward]
+                    [--prefill-steps S]
                     [--prefill-len N]
 
 Prints ONE JSON line (rank 0).  N > 1 runs under torchrun: every rank runs
@@ -53,6 +55,8 @@ def parse():
                     help="skip the prefill_128k measurement attached to a decode run")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the index-branch variant measurement attached to a decode run")
+    ap.add_argument("--no-fused", action="store_true",
+                    help="skip the single-launch decode step attached to a decode run")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the sparse-branch backward measurement attached to a decode run")
     ap.add_argument("--prefill-steps", type=int, default=5)
@@ -300,6 +304,49 @@ def measure_index_variants(w, dev, steps, warmup):
         del eng, q_idx, keys, scale
         torch.cuda.empty_cache()
     return out
+
+
+def measure_decode_fused(w, dev, steps, warmup, step_bytes, ref_ids):
+    """The same decode step as one cooperative launch (msa_decode_step:
+    index scores, top-k and sparse attention fused); GB/s on the same
+    algorithmic bytes as the two-call step, and whether its block ids equal
+    the two-call path's."""
+    import block_sparse_attention_43_b200 as msa
+    peak, _, _, kind = measured_peaks()
+    stream = torch.cuda.Stream(device=dev)
+    eng = msa.MSA(batch=w.B, q_len=1, max_kv_len=max(w.lens_host), num_q_heads=w.H_q,
+                  num_kv_heads=w.H_kv, top_k=w.top_k, kv_capacity=w.kv_capacity, device=dev)
+
+    def step():
+        eng.decode_step(w.q_idx, w.k_idx, w.q, w.k, w.v, w.lens, w.kv_offsets, stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    st = msa.msa_read_device_status(eng.ws_step, stream)
+    if st != 0:
+        raise RuntimeError(f"decode_step: device status {msa.STATUS_NAMES.get(st, st)}")
+    same = bool(np.array_equal(eng.block_ids.cpu().numpy(), ref_ids))
+    msa.msa_trace_enable(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    trace = msa.msa_trace_read()
+    msa.msa_trace_enable(False)
+    ker = [t for n, t in trace if n == "decode_fused_step"]
+    ms = ev0.elapsed_time(ev1) / steps
+    kms = float(np.mean(ker)) if ker else float("nan")
+    gbs = step_bytes / (ms / 1e3) / 1e9
+    res = {"entry": "msa_decode_step", "ms_per_step": ms, "kernel_ms": kms,
+           "launches_per_step": len(trace) / steps, "gbs": gbs, "frac_of_hbm": gbs / peak,
+           "kernel_gbs": step_bytes / (kms / 1e3) / 1e9, "peak_kind": kind,
+           "ids_equal_two_call": same}
+    del eng
+    torch.cuda.empty_cache()
+    return res
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -560,6 +607,11 @@ def main():
         cpu = {"value": gbs, "unit": "GB/s", "cores": used, "kind": "oracle", "sample": note,
                "seconds": dt}
 
+    fused = None
+    if not args.no_fused and world == 1:
+        fused = measure_decode_fused(w, dev, max(20, args.steps // 4), 5, step_bytes, ids_host)
+        fused["two_call_ms_per_step"] = ms_step
+
     variants = None
     if not args.no_variants and world == 1:
         variants = measure_index_variants(w, dev, 20, 3)
@@ -607,6 +659,7 @@ def main():
             "e2e": e2e,
             "cpu_baseline": cpu,
             "prefill_128k": prefill,
+            "decode_step_fused": fused,
             "index_variants": variants,
             "prefill_backward": backward,
         }

@@ -13,9 +13,12 @@
 //   - CTAs (one per SM, cooperative launch so all are resident) claim index
 //     units (one 128-token block of one sequence, all groups) from a global
 //     counter in sequence order, so sequences finish one after another;
-//   - the CTA that finishes a sequence's last unit runs that sequence's top-k
-//     (one warp per group, the warp selection of topk.cu) and publishes one
-//     attention item per (group, kept block);
+//   - per unit the consumer warps hand the 16 row-slot maxima to a
+//     bookkeeper warp, which stores the block scores and counts them with a
+//     device-scope atomic, so no consumer ever waits on a global round trip;
+//     the bookkeeper that counts a sequence's last score has the producer
+//     queue that sequence's top-k (one consumer warp per group, the warp
+//     selection of topk.cu), which publishes one attention item per group;
 //   - between index units a CTA takes published attention items, one per
 //     (sequence, group): the K/V tiles of its kept blocks (TMA, 128-byte
 //     swizzle) stream through the same ring, S^T = K Q^T and O^T = V^T P^T
@@ -36,14 +39,17 @@ namespace {
 
 constexpr int kWarps = 8;                     // consumer warps
 constexpr int kConsumers = kWarps * 32;
-constexpr int kThreads = kConsumers + 32;     // + producer warp
+constexpr int kProducerWarp = kWarps, kBookWarp = kWarps + 1;
+constexpr int kThreads = kConsumers + 64;     // + producer warp + bookkeeper warp
+constexpr int kRedQ = 4;                      // index units whose row maxima await the bookkeeper
+constexpr int kFifo = 16;                     // top-k requests from the bookkeeper to the producer
 constexpr int kStages = 5;
 constexpr int kStageBytes = 32768;
 constexpr int kQueue = 4;
 constexpr int kMaxBatch = 4096;
 constexpr float kLog2e = 1.4426950408889634f;
 
-enum { kWorkIndex = 0, kWorkAttn = 1, kWorkSync = 2, kWorkEnd = 3 };
+enum { kWorkIndex = 0, kWorkAttn = 1, kWorkTopk = 2, kWorkEnd = 3 };
 
 struct Smem {
     uint8_t ring[kStages][kStageBytes];       // index-key stages / K and V tiles of a block
@@ -53,10 +59,14 @@ struct Smem {
     uint64_t wq_full[kQueue], wq_empty[kQueue];
     uint64_t cbar;                            // consumer-wide sync (all 256 threads arrive)
     int4 wq[kQueue];                          // {kind, a, b, c}
+    uint64_t red_full[kRedQ], red_empty[kRedQ];
     int prefix[kMaxBatch + 1];
-    float red[2][16];
+    float red[kRedQ][16];                     // per index unit: max of each row slot
+    int red_b[kRedQ], red_j[kRedQ];           // its (sequence, block); sequence -1 ends the stream
+    int topk_fifo[kFifo];
+    int topk_wr, topk_rd;
+    int book_done;                            // index units the bookkeeper has finished
     int bcast[2];
-    unsigned long long topk_req[2];           // (checkpoint << 32) | sequence, by checkpoint parity
     int total_attn;
     int abort_flag;
 };
@@ -117,7 +127,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&S.wq_empty[i], kWarps);
         }
         mbar_init(&S.cbar, kConsumers);
-        S.topk_req[0] = S.topk_req[1] = ~0ull;
+        for (int i = 0; i < kRedQ; ++i) {
+            mbar_init(&S.red_full[i], kWarps);
+            mbar_init(&S.red_empty[i], 1);
+        }
+        S.topk_wr = S.topk_rd = S.book_done = 0;
         S.abort_flag = 0;
         fence_mbar_init();
     }
@@ -164,7 +178,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int U = S.prefix[P.B];
     const int total_attn = S.total_attn;
 
-    if (warp == kWarps) {
+    if (warp == kBookWarp) {
+        // ------------------------------------------------ bookkeeper: block
+        // scores and sequence completion, off the consumers' path.  Per index
+        // unit: the max of the group's row slots is the block score (one lane
+        // per group), stored and counted with a device-scope atomic; the lane
+        // that counts a sequence's last score asks the producer (through a
+        // shared-memory FIFO) to queue that sequence's top-k.
+        const unsigned long long t0 = now_ns();
+        for (int k = 0;; ++k) {
+            const int slot = k % kRedQ;
+            bool have = !*abort_flag && mbar_wait(&S.red_full[slot], (k / kRedQ) & 1, P.status);
+            have = __all_sync(0xffffffffu, have);
+            if (!have) { *abort_flag = 1; break; }
+            const int b = S.red_b[slot], j = S.red_j[slot];
+            float m = -INFINITY;
+            if (lane < H)
+                for (int r = lane; r < 16; r += H) m = fmaxf(m, S.red[slot][r]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.red_empty[slot]);
+            if (b < 0) break;                       // the consumers are done
+            bool last = false;
+            if (lane < H) {
+                P.scores[((long long)b * H + lane) * nbs + j] = m;
+                const int target = H * ((P.lens[b] + kBlock - 1) / kBlock);
+                last = atom_add_acq_rel_gpu(P.seq_done + b, 1) + 1 == target;
+            }
+            if (__any_sync(0xffffffffu, last) && lane == 0) {
+                // at most kRedQ + kQueue units finish between two producer
+                // polls, so the FIFO does not fill; the wait is a safety net
+                while (S.topk_wr - ld_volatile(&S.topk_rd) >= kFifo) {
+                    if (*abort_flag || now_ns() - t0 > kWaitNs) { set_status(P.status, kStatusTimeout); *abort_flag = 1; break; }
+                    __nanosleep(64);
+                }
+                S.topk_fifo[S.topk_wr % kFifo] = b;
+                __threadfence_block();
+                *reinterpret_cast<volatile int *>(&S.topk_wr) = S.topk_wr + 1;
+            }
+            if (lane == 0) {
+                __threadfence_block();              // the FIFO entry above comes first
+                *reinterpret_cast<volatile int *>(&S.book_done) = k + 1;
+            }
+            __syncwarp();
+        }
+        return;
+    }
+
+    if (warp == kProducerWarp) {
         // ------------------------------------------------ producer: claims work,
         // publishes it to the consumers and issues its loads
         if (lane != 0) return;
@@ -204,9 +264,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         int pending = -1, pending_flag = 0;
         bool attn_left = total_attn > 0;
         int u_next = atomicAdd(c_unit, 1);
-        int seen_claim = 0, seen_pub = 0;
+        int seen_claim = 0, seen_pub = 0, units_pushed = 0;
+        // queues the top-k of every sequence the bookkeeper has completed
+        auto drain_topk = [&]() -> bool {
+            while (S.topk_rd != ld_volatile(&S.topk_wr)) {
+                __threadfence_block();
+                const int b = S.topk_fifo[S.topk_rd % kFifo];
+                if (!push(make_int4(kWorkTopk, b, 0, 0))) return false;
+                *reinterpret_cast<volatile int *>(&S.topk_rd) = S.topk_rd + 1;
+            }
+            return true;
+        };
         const unsigned long long t0 = now_ns();
         while (ok) {
+            if (!drain_topk()) { ok = false; break; }
             if (pending < 0 && attn_left) {
                 if (!index_left) seen_claim = ld_volatile(c_claim);
                 if (seen_claim >= total_attn) {
@@ -220,19 +291,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (pending >= 0 && (!index_left || pending_flag != 0)) {
                 // Attention item: its flag is set, or will be once the index
-                // units of its sequence are done.  Before waiting, let this
-                // CTA's consumers pass a checkpoint: the top-k that publishes
-                // the item may be theirs to run.
+                // units of its sequence are done.  While waiting, keep queueing
+                // this CTA's top-k requests: the one that publishes the item
+                // may be among them.
                 const int item = pending;
                 pending = -1;
-                if (ld_volatile(P.aq_flag + item) == 0) {
-                    if (!push(make_int4(kWorkSync, 0, 0, 0))) { ok = false; break; }
-                    while (ld_volatile(P.aq_flag + item) == 0) {
-                        if (*abort_flag || now_ns() - t0 > kWaitNs) { set_status(P.status, kStatusTimeout); ok = false; break; }
-                        __nanosleep(128);
+                while (ld_volatile(P.aq_flag + item) == 0) {
+                    if (!drain_topk() || *abort_flag || now_ns() - t0 > kWaitNs) {
+                        set_status(P.status, kStatusTimeout);
+                        ok = false;
+                        break;
                     }
-                    if (!ok) break;
+                    __nanosleep(128);
                 }
+                if (!ok) break;
                 __threadfence();
                 const int bg = __ldcg(P.aq_item + item);
                 const int b = bg / H, g = bg % H;
@@ -270,6 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int L = P.lens[b];
                 const int ntok = min(kBlock, L - j * kBlock);
                 if (!push(make_int4(kWorkIndex, b, j, ntok))) { ok = false; break; }
+                ++units_pushed;
                 const long long t_first = kv_block_row(P.kv, b, j, P.status);
                 for (int t0s = 0; t0s < ntok; t0s += tps) {
                     int slot;
@@ -283,6 +356,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!attn_left) break;
             if (*abort_flag || now_ns() - t0 > kWaitNs) { set_status(P.status, kStatusTimeout); ok = false; break; }
         }
+        // A top-k this CTA's bookkeeper has still to request must be queued
+        // before the end: wait until it has finished every unit pushed here.
+        while (ok && ld_volatile(&S.book_done) < units_pushed) {
+            if (!drain_topk() || *abort_flag || now_ns() - t0 > kWaitNs) {
+                set_status(P.status, kStatusTimeout);
+                ok = false;
+                break;
+            }
+            __nanosleep(64);
+        }
+        if (ok) ok = drain_topk();
         if (!ok) *abort_flag = 1;
         push(make_int4(kWorkEnd, 0, 0, 0));      // best effort: consumers also stop on abort
         // let every copy already issued land before the CTA can exit
@@ -365,16 +449,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tid == 0) atomicAdd(P.ctr + 3 * kCtrStride, count);
     };
 
-    // Checkpoints follow a consumer-wide sync, so every consumer thread reads
-    // the same request: a top-k asked for since the previous checkpoint (the
-    // request carries the checkpoint number it is for, and the slots
-    // alternate, so a request written after this read waits for the next).
-    int ck = 0;
-    auto checkpoint = [&]() {
-        const unsigned long long v = *reinterpret_cast<volatile unsigned long long *>(&S.topk_req[ck & 1]);
-        const bool hit = static_cast<int>(v >> 32) == ck;
-        ++ck;
-        if (hit && !*abort_flag) topk_and_publish(static_cast<int>(v & 0xffffffffu));
+    // Hands one index unit's row-slot maxima (or, with b = -1, the end of the
+    // stream) to the bookkeeper through the kRedQ-deep queue.
+    auto hand_over = [&](int b, int j, float runmax) -> bool {
+        const int slot = unit_iter % kRedQ;
+        bool have = unit_iter < kRedQ ||
+                    (!*abort_flag && mbar_wait(&S.red_empty[slot], ((unit_iter / kRedQ) - 1) & 1, P.status));
+        have = __all_sync(0xffffffffu, have);
+        ++unit_iter;
+        if (!have) { *abort_flag = 1; return false; }
+        if (c16 == 0) S.red[slot][r16] = runmax;
+        if (tid == 0) { S.red_b[slot] = b; S.red_j[slot] = j; }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.red_full[slot]);
+        return true;
     };
 
     for (int n = 0;; ++n) {
@@ -385,10 +473,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int4 w = S.wq[wslot];
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.wq_empty[wslot]);
-        if (w.x == kWorkSync || w.x == kWorkEnd) {
-            cbar();
-            checkpoint();
-            if (w.x == kWorkEnd) break;
+        if (w.x == kWorkEnd) break;
+        if (w.x == kWorkTopk) {
+            if (!*abort_flag) topk_and_publish(w.y);
             continue;
         }
 
@@ -430,22 +517,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     release_stage(slot);
                 }
             }
-            const int par = unit_iter++ & 1;
-            if (c16 == 0) S.red[par][r16] = runmax;
-            cbar();
-            checkpoint();
-            // One thread per group stores the block score and counts it; the
-            // rest of the CTA goes straight on.  The thread that sees the
-            // sequence's last score requests its top-k at the next checkpoint.
-            if (tid < H && !*abort_flag) {
-                float m = -INFINITY;
-                for (int r = tid; r < 16; r += H) m = fmaxf(m, S.red[par][r]);
-                P.scores[((long long)b * H + tid) * nbs + j] = m;
-                const int target = H * ((P.lens[b] + kBlock - 1) / kBlock);
-                if (atom_add_acq_rel_gpu(P.seq_done + b, 1) + 1 == target)
-                    *reinterpret_cast<volatile unsigned long long *>(&S.topk_req[ck & 1]) =
-                        (static_cast<unsigned long long>(ck) << 32) | static_cast<unsigned>(b);
-            }
+            // Row-slot maxima to the bookkeeper, which finishes the unit.
+            if (!hand_over(b, j, runmax)) break;
             continue;
         }
 
@@ -571,8 +644,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         cbar();                                     // om, mw, lw and bcast are reused
-        checkpoint();
     }
+    hand_over(-1, 0, 0.f);                          // end of the bookkeeper's stream
 }
 
 }  // namespace
@@ -581,13 +654,15 @@ size_t decode_fused_layout(int B, int H_q, int H_kv, int K, int max_kv_len, Deco
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
     const size_t nb_max = score_stride((max_kv_len + kBlock - 1) / kBlock);
     const size_t items = static_cast<size_t>(B) * H_kv;
+    // Everything cleared per call sits right after the status header, so one
+    // memset covers [0, zero_hi).
     size_t o = kWsHeaderBytes;
-    L->scores = o;   o += up(static_cast<size_t>(B) * H_kv * nb_max * 4);
-    L->zero_lo = o;                                 // cleared per call: counters and flags
+    L->zero_lo = o;
     L->ctr = o;      o += 4 * kCtrStride * 4;
     L->seq_done = o; o += up(static_cast<size_t>(B) * 4);
     L->aq_flag = o;  o += up(items * 4);
     L->zero_hi = o;
+    L->scores = o;   o += up(static_cast<size_t>(B) * H_kv * nb_max * 4);
     L->aq_item = o;  o += up(items * 4);
     L->total = o;
     (void)H_q;

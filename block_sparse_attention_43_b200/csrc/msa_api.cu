@@ -494,10 +494,8 @@ msa_status_t msa_decode_step(const msa_shape_t *shape, const void *q_idx, const 
     if ((st = check_ws(workspace, workspace_bytes, L.total)) != MSA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    // status word (header), then the claim counters and per-call flags
-    if (cudaMemsetAsync(ws, 0, kWsHeaderBytes, s) != cudaSuccess ||
-        cudaMemsetAsync(ws + L.zero_lo, 0, L.zero_hi - L.zero_lo, s) != cudaSuccess)
-        return MSA_ERR_CUDA;
+    // status word, claim counters and per-call flags: one contiguous range
+    if (cudaMemsetAsync(ws, 0, L.zero_hi, s) != cudaSuccess) return MSA_ERR_CUDA;
     DecodeFusedArgs a;
     a.q_idx = q_idx; a.k_idx = k_idx; a.q = q; a.k_cache = k_cache; a.v_cache = v_cache;
     a.lens = lens; a.kv = packed_map(shape, kv_offsets);
