@@ -699,41 +699,54 @@ def run_prefill_headline(args):
 
 
 def run_e2e(w, eng, stream, args, step_bytes, world, dist):
-    """Same step through the public API from pinned host buffers: per step the
-    new query (q, q_idx) and the new token's k/v/k_idx rows go host->device
-    (the token is appended at position L-1 of every sequence's resident cache),
-    the two calls run, and out + block ids + block scores come back."""
+    """Same step through the public API from pinned host buffers, as a decode
+    server runs it: per step ONE host->device copy brings the new query (q,
+    q_idx) and the new token's k_idx/k/v rows, `msa_kv_append` writes that
+    token at position L-1 of every sequence's resident cache, the two calls
+    run, and ONE device->host copy returns out + block ids + block scores
+    (packed into one device buffer), then the host waits for it."""
+    import block_sparse_attention_43_b200 as msa
     B = w.B
+    dev = w.q.device
     pos = [int(w.kv_offsets[b]) + w.lens_host[b] - 1 for b in range(B)]
-    h_q = w.q.cpu().pin_memory()
-    h_qi = w.q_idx.cpu().pin_memory()
-    h_tok = {n: torch.stack([getattr(w, n)[p] for p in pos]).cpu().pin_memory()
-             for n in ("k", "v", "k_idx")}
-    h_out = torch.empty(eng.out.shape, dtype=eng.out.dtype).pin_memory()
-    h_ids = torch.empty(eng.block_ids.shape, dtype=torch.int32).pin_memory()
-    h_sc = torch.empty(eng.block_scores.shape, dtype=torch.float32).pin_memory()
-    d_q = torch.empty_like(w.q)
-    d_qi = torch.empty_like(w.q_idx)
-    h2d = h_q.numel() * 2 + h_qi.numel() * 2 + sum(t.numel() * 2 for t in h_tok.values())
-    d2h = h_out.numel() * 2 + h_ids.numel() * 4 + h_sc.numel() * 4
+    rows = {n: torch.stack([getattr(w, n)[p] for p in pos]).unsqueeze(1) for n in ("k_idx", "k", "v")}
+    parts = [w.q, w.q_idx, rows["k_idx"], rows["k"], rows["v"]]
+    h_in = torch.cat([t.reshape(-1).cpu() for t in parts]).pin_memory()
+    d_in = torch.empty_like(h_in, device=dev)
+    views, o = [], 0
+    for t in parts:
+        views.append(d_in[o:o + t.numel()].view(t.shape))
+        o += t.numel()
+    d_q, d_qi, d_kidx, d_k, d_v = views
+    lens_prev = (w.lens - 1).contiguous()       # kv_append writes at lens[b] + 0
+    # outputs packed into one device buffer: out (bf16) | ids (int32) | scores (fp32)
+    n_out = eng.out.numel() * 2
+    n_ids = eng.block_ids.numel() * 4
+    d_res = torch.empty(n_out + 2 * n_ids, dtype=torch.uint8, device=dev)
+    out_v = d_res[:n_out].view(torch.bfloat16).view(eng.out.shape)
+    ids_v = d_res[n_out:n_out + n_ids].view(torch.int32).view(eng.block_ids.shape)
+    sc_v = d_res[n_out + n_ids:].view(torch.float32).view(eng.block_scores.shape)
+    h_res = torch.empty(d_res.shape, dtype=torch.uint8).pin_memory()
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    h2d = h_in.numel() * h_in.element_size()
+    d2h = h_res.numel()
 
     def one():
         with torch.cuda.stream(stream):
-            d_q.copy_(h_q, non_blocking=True)
-            d_qi.copy_(h_qi, non_blocking=True)
-            for n, t in h_tok.items():
-                dst = getattr(w, n)
-                for b, p in enumerate(pos):
-                    dst[p].copy_(t[b], non_blocking=True)
-            eng.index_topk(d_qi, w.k_idx, w.lens, w.kv_offsets, stream)
-            eng.sparse_attention(d_q, w.k, w.v, w.lens, w.kv_offsets, stream=stream)
-            h_out.copy_(eng.out, non_blocking=True)
-            h_ids.copy_(eng.block_ids, non_blocking=True)
-            h_sc.copy_(eng.block_scores, non_blocking=True)
+            d_in.copy_(h_in, non_blocking=True)
+            msa.msa_kv_append(eng.shape, d_kidx, d_k, d_v, lens_prev, w.k_idx, w.k, w.v,
+                              kv_offsets=w.kv_offsets, device_status=status, stream=stream)
+            msa.msa_index_topk(eng.shape, d_qi, w.k_idx, w.lens, w.kv_offsets, ids_v, sc_v,
+                               eng.ws_index, stream)
+            msa.msa_sparse_attention(eng.shape, d_q, w.k, w.v, ids_v, w.lens, w.kv_offsets,
+                                     eng.softmax_scale, out_v, eng.ws_attn, stream)
+            h_res.copy_(d_res, non_blocking=True)
         stream.synchronize()
 
     for _ in range(max(3, args.warmup // 4)):
         one()
+    if int(status.item()) != 0 or msa.msa_read_device_status(eng.ws_attn, stream) != 0:
+        raise RuntimeError("e2e: device status set")
     n = max(10, args.steps // 4)
     if dist is not None:
         dist.barrier()
@@ -742,7 +755,8 @@ def run_e2e(w, eng, stream, args, step_bytes, world, dist):
         one()
     rate, dt = whole_job_rate(dist, world, step_bytes, (time.perf_counter() - t0) / n, w.q.device)
     return {"value": rate / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": dt * 1e3, "steps": n}
+            "d2h_bytes_per_step": d2h, "ms_per_step": dt * 1e3, "steps": n,
+            "copies_per_step": {"h2d": 1, "d2h": 1}}
 
 
 if __name__ == "__main__":

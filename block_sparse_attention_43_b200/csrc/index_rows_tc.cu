@@ -415,6 +415,8 @@ cudaError_t launch_widen_e4m3(const void *src, void *dst, long long rows, cudaSt
 }
 
 cudaError_t launch_index_rows_tc(const IndexRowsArgs &a, cudaStream_t s) {
+    static_assert(sizeof(Smem<16>) + 1024 <= 227 * 1024, "shared memory budget");
+    static_assert(sizeof(Smem<32>) + 1024 <= 227 * 1024, "shared memory budget");
     static_assert(sizeof(Smem<64>) + 1024 <= 227 * 1024, "shared memory budget");
     CUtensorMap tq, tk;
     if (!encode_kv_tensor_map(&tq, a.q_idx, a.H_kv, static_cast<long long>(a.B) * a.Sq) ||

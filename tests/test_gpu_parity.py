@@ -95,6 +95,25 @@ def test_prefill_block_outer_path(msa_lib, oracle_mod, B, Sq, lens, H_q, H_kv, t
     print("prefill g8", (B, Sq, H_q, H_kv, top_k), rep)
 
 
+# top-k above 16 takes the index kernel's longer row lists (32, 64 slots) and
+# the block-outer attention with up to 64 kept blocks per row.
+PREFILL_LARGE_K_CASES = [
+    (1, 6000, [6000], 16, 2, 32),      # 47 blocks, 32 kept
+    (2, 4500, [9000, 4500], 16, 2, 64),  # chunk after a cached prefix (71 blocks) + 36 blocks
+    (1, 3000, [3000], 8, 2, 17),       # list of 32 slots, row attention path (groups of 4)
+]
+
+
+@pytest.mark.parametrize("B,Sq,lens,H_q,H_kv,top_k", PREFILL_LARGE_K_CASES)
+def test_prefill_large_top_k(msa_lib, oracle_mod, B, Sq, lens, H_q, H_kv, top_k):
+    from parity import sample_rows
+    from synthetic import make_inputs
+    w = make_inputs(B=B, Sq=Sq, lens=lens, H_q=H_q, H_kv=H_kv, top_k=top_k, seed=500 + top_k,
+                    device=DEV)
+    rep = _run_and_compare(oracle_mod, w, rows=sample_rows(B * Sq, 600, seed=6))
+    print("prefill large k", (B, Sq, H_q, H_kv, top_k), rep)
+
+
 def test_prefill_large_logit_block_takes_exact_shift(msa_lib, oracle_mod):
     """A kept non-own block whose keys are 40x larger: its logits dwarf the
     own block's, the norm bound cannot prove the own-block shift safe, and the
