@@ -28,8 +28,11 @@
 // An attention item is claimed (one atomicAdd) only while the claim counter
 // is below the published count; a claim that overtakes its publisher stays
 // pending while the CTA streams more index units.  Once a CTA has no index
-// unit left it waits for its claimed item, which the CTA that finishes that
-// sequence's index scores publishes.  Every wait is bounded.
+// unit left it waits for its claimed item, which the CTA whose bookkeeper
+// counts that sequence's last score publishes; while it waits, its producer
+// keeps queueing its own CTA's top-k requests, and it ends only after its
+// bookkeeper has finished every unit it handed out, so no request is left
+// behind.  Every wait is bounded.
 #include "msa_device.cuh"
 #include "msa_internal.h"
 #include "topk_warp.cuh"
