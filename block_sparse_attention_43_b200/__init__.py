@@ -27,7 +27,8 @@ EXPORTS = ("msa_index_topk_workspace_size", "msa_index_topk", "msa_index_topk_fp
            "msa_index_topk_paged", "msa_sparse_attention_paged", "msa_kv_append",
            "msa_index_topk_static", "msa_sparse_attention_backward_workspace_size",
            "msa_sparse_attention_backward", "msa_decode_step_workspace_size",
-           "msa_decode_step", "msa_read_device_status", "msa_trace_enable",
+           "msa_decode_step", "msa_decode_step_paged", "msa_read_device_status",
+           "msa_trace_enable",
            "msa_trace_read",
            "msa_status_string")
 
@@ -85,6 +86,9 @@ def _load():
     lib.msa_decode_step_workspace_size.restype = Z
     lib.msa_decode_step.argtypes = [S, P, P, P, P, P, P, P, ctypes.c_float, P, P, P, P, Z, P]
     lib.msa_decode_step.restype = ctypes.c_int
+    lib.msa_decode_step_paged.argtypes = [S, P, P, P, P, P, P, P, I32, ctypes.c_float, P, P, P, P,
+                                          Z, P]
+    lib.msa_decode_step_paged.restype = ctypes.c_int
     lib.msa_read_device_status.argtypes = [P, P]
     lib.msa_read_device_status.restype = ctypes.c_int
     lib.msa_trace_enable.argtypes = [ctypes.c_int]
@@ -236,6 +240,19 @@ def msa_decode_step(shape, q_idx, k_idx, q, k_cache, v_cache, lens, kv_offsets, 
                                float(softmax_scale), _ptr(block_ids), _ptr(block_scores),
                                _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)),
            "msa_decode_step")
+
+
+def msa_decode_step_paged(shape, q_idx, k_idx_pool, q, k_pool, v_pool, lens, page_table,
+                          softmax_scale, block_ids, block_scores, out, workspace,
+                          stream=None) -> None:
+    """msa_decode_step on paged caches (page_table [B, pages_per_seq])."""
+    pps = int(page_table.shape[-1])
+    _check(lib.msa_decode_step_paged(ctypes.byref(shape), _ptr(q_idx), _ptr(k_idx_pool), _ptr(q),
+                                     _ptr(k_pool), _ptr(v_pool), _ptr(lens), _ptr(page_table), pps,
+                                     float(softmax_scale), _ptr(block_ids), _ptr(block_scores),
+                                     _ptr(out), _ptr(workspace), workspace.numel(),
+                                     _stream(stream)),
+           "msa_decode_step_paged")
 
 
 def msa_read_device_status(workspace, stream=None) -> int:

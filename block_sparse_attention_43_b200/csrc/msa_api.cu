@@ -475,15 +475,14 @@ size_t msa_decode_step_workspace_size(const msa_shape_t *shape) {
     return decode_step_layout(shape).total;
 }
 
-msa_status_t msa_decode_step(const msa_shape_t *shape, const void *q_idx, const void *k_idx,
-                             const void *q, const void *k_cache, const void *v_cache,
-                             const int32_t *lens, const int64_t *kv_offsets, float softmax_scale,
-                             int32_t *block_ids, float *block_scores, void *out, void *workspace,
-                             size_t workspace_bytes, msa_stream_t stream) {
-    msa_status_t st = check_decode_step(shape);
-    if (st != MSA_OK) return st;
-    if (!q_idx || !k_idx || !q || !k_cache || !v_cache || !lens || !kv_offsets || !block_ids ||
-        !block_scores || !out)
+static msa_status_t decode_step_impl(const msa_shape_t *shape, const void *q_idx,
+                                     const void *k_idx, const void *q, const void *k_cache,
+                                     const void *v_cache, const int32_t *lens, const KvMap &kv,
+                                     float softmax_scale, int32_t *block_ids, float *block_scores,
+                                     void *out, void *workspace, size_t workspace_bytes,
+                                     msa_stream_t stream) {
+    if (!q_idx || !k_idx || !q || !k_cache || !v_cache || !lens || !block_ids || !block_scores ||
+        !out)
         return MSA_ERR_INVALID_ARG;
     if (!(softmax_scale == softmax_scale) || softmax_scale == INFINITY || softmax_scale == -INFINITY)
         return MSA_ERR_INVALID_ARG;
@@ -491,14 +490,15 @@ msa_status_t msa_decode_step(const msa_shape_t *shape, const void *q_idx, const 
         !aligned16(v_cache) || !aligned16(out))
         return MSA_ERR_MISALIGNED;
     const DecodeFusedLayout L = decode_step_layout(shape);
-    if ((st = check_ws(workspace, workspace_bytes, L.total)) != MSA_OK) return st;
+    msa_status_t st = check_ws(workspace, workspace_bytes, L.total);
+    if (st != MSA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     // status word, claim counters and per-call flags: one contiguous range
     if (cudaMemsetAsync(ws, 0, L.zero_hi, s) != cudaSuccess) return MSA_ERR_CUDA;
     DecodeFusedArgs a;
     a.q_idx = q_idx; a.k_idx = k_idx; a.q = q; a.k_cache = k_cache; a.v_cache = v_cache;
-    a.lens = lens; a.kv = packed_map(shape, kv_offsets);
+    a.lens = lens; a.kv = kv;
     a.ids = block_ids; a.out_scores = block_scores; a.out = out;
     a.status = reinterpret_cast<int *>(ws);
     a.ctr = reinterpret_cast<int *>(ws + L.ctr);
@@ -510,6 +510,34 @@ msa_status_t msa_decode_step(const msa_shape_t *shape, const void *q_idx, const 
     a.K = shape->top_k; a.nb_max = nb_max_of(shape); a.max_kv_len = shape->max_kv_len;
     a.softmax_scale = softmax_scale;
     return launch_decode_fused(a, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+}
+
+msa_status_t msa_decode_step(const msa_shape_t *shape, const void *q_idx, const void *k_idx,
+                             const void *q, const void *k_cache, const void *v_cache,
+                             const int32_t *lens, const int64_t *kv_offsets, float softmax_scale,
+                             int32_t *block_ids, float *block_scores, void *out, void *workspace,
+                             size_t workspace_bytes, msa_stream_t stream) {
+    msa_status_t st = check_decode_step(shape);
+    if (st != MSA_OK) return st;
+    if (!kv_offsets) return MSA_ERR_INVALID_ARG;
+    return decode_step_impl(shape, q_idx, k_idx, q, k_cache, v_cache, lens,
+                            packed_map(shape, kv_offsets), softmax_scale, block_ids, block_scores,
+                            out, workspace, workspace_bytes, stream);
+}
+
+msa_status_t msa_decode_step_paged(const msa_shape_t *shape, const void *q_idx,
+                                   const void *k_idx_pool, const void *q, const void *k_pool,
+                                   const void *v_pool, const int32_t *lens,
+                                   const int32_t *page_table, int32_t pages_per_seq,
+                                   float softmax_scale, int32_t *block_ids, float *block_scores,
+                                   void *out, void *workspace, size_t workspace_bytes,
+                                   msa_stream_t stream) {
+    msa_status_t st = check_decode_step(shape);
+    if (st != MSA_OK) return st;
+    if ((st = check_paged(shape, page_table, pages_per_seq)) != MSA_OK) return st;
+    return decode_step_impl(shape, q_idx, k_idx_pool, q, k_pool, v_pool, lens,
+                            paged_map(shape, page_table, pages_per_seq), softmax_scale, block_ids,
+                            block_scores, out, workspace, workspace_bytes, stream);
 }
 
 msa_status_t msa_read_device_status(const void *workspace, msa_stream_t stream) {

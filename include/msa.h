@@ -229,6 +229,21 @@ MSA_API msa_status_t msa_decode_step(const msa_shape_t *shape, const void *q_idx
                                      void *workspace, size_t workspace_bytes,
                                      msa_stream_t stream);
 
+/* msa_decode_step on paged caches (the layout described below): index keys,
+ * keys and values in pools of 128-token pages, block j of sequence b in page
+ * page_table[b * pages_per_seq + j].  Same requirements, results, workspace
+ * size and errors as msa_decode_step, plus the paged checks below; the
+ * results equal msa_decode_step's on a packed copy of the same tokens, bit for
+ * bit (the kernel's summation order does not depend on where a block lives). */
+MSA_API msa_status_t msa_decode_step_paged(const msa_shape_t *shape, const void *q_idx,
+                                           const void *k_idx_pool, const void *q,
+                                           const void *k_pool, const void *v_pool,
+                                           const int32_t *lens, const int32_t *page_table,
+                                           int32_t pages_per_seq, float softmax_scale,
+                                           int32_t *block_ids, float *block_scores, void *out,
+                                           void *workspace, size_t workspace_bytes,
+                                           msa_stream_t stream);
+
 /* Paged caches (a block-table layout for serving): the index keys, keys and
  * values of all sequences live in pools of 128-token pages, [kv_capacity,
  * H_kv, dim] with page p = rows p*128 .. p*128+127, and block j of sequence b

@@ -153,3 +153,9 @@ def test_decode_step_rejects_unsupported_shapes(m):
     ok = m.make_shape(batch=3, q_len=1, max_kv_len=1000, num_q_heads=16, num_kv_heads=2,
                       top_k=4, kv_capacity=3000)
     assert m.msa_decode_step_workspace_size(ok) > 256
+    # paged: a pool that is not whole pages, or a table row too short for max_kv_len
+    for cap, pps in ((3000, 8), (3072, 7)):
+        s = m.make_shape(batch=3, q_len=1, max_kv_len=1000, num_q_heads=16, num_kv_heads=2,
+                         top_k=4, kv_capacity=cap)
+        assert m.lib.msa_decode_step_paged(ctypes.byref(s), *([0x1000] * 7), pps, 0.1, 0x1000,
+                                           0x1000, 0x1000, 0x100000, 1 << 40, None) == 1

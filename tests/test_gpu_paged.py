@@ -175,3 +175,35 @@ def test_kv_append_past_max_len_is_refused(m):
     torch.cuda.synchronize()
     assert int(status.item()) == 1
     assert torch.equal(w.k, before)
+
+
+@pytest.mark.parametrize("B,lens,H_q,H_kv,top_k", [
+    (3, [5000, 129, 20000], 64, 8, 16),
+    (2, [4096, 300], 16, 4, 4),
+])
+def test_fused_decode_step_paged_equals_packed(m, oracle_mod, B, lens, H_q, H_kv, top_k):
+    """msa_decode_step_paged on shuffled pages (NaN page padding) gives the
+    packed msa_decode_step's ids, scores and outputs bit for bit."""
+    from parity import compare
+    from synthetic import make_inputs
+    w = make_inputs(B=B, Sq=1, lens=lens, H_q=H_q, H_kv=H_kv, top_k=top_k, seed=650 + B,
+                    device=DEV, needles=2)
+    eng = m.MSA(batch=B, q_len=1, max_kv_len=max(lens), num_q_heads=H_q, num_kv_heads=H_kv,
+                top_k=top_k, kv_capacity=w.kv_capacity, device=DEV)
+    eng.decode_step(w.q_idx, w.k_idx, w.q, w.k, w.v, w.lens, w.kv_offsets)
+    torch.cuda.synchronize()
+    assert m.msa_read_device_status(eng.ws_step) == 0
+    pools, table, n_pages = _paged_copy(w)
+    shape = m.make_shape(batch=B, q_len=1, max_kv_len=max(lens), num_q_heads=H_q,
+                         num_kv_heads=H_kv, top_k=top_k, kv_capacity=n_pages * 128)
+    ids = torch.empty_like(eng.block_ids)
+    sc = torch.empty_like(eng.block_scores)
+    out = torch.empty_like(eng.out)
+    ws = m.alloc_workspace(m.msa_decode_step_workspace_size(shape), DEV)
+    m.msa_decode_step_paged(shape, w.q_idx, pools["k_idx"], w.q, pools["k"], pools["v"], w.lens,
+                            table, w.scale, ids, sc, out, ws)
+    torch.cuda.synchronize()
+    assert m.msa_read_device_status(ws) == 0
+    assert torch.equal(ids, eng.block_ids) and torch.equal(sc, eng.block_scores)
+    assert torch.equal(out, eng.out)
+    compare(oracle_mod, w, ids.cpu().numpy(), sc.cpu().numpy(), out.float().cpu().numpy())
