@@ -556,7 +556,7 @@ const char *msa_status_string(msa_status_t status) {
     switch (status) {
         case MSA_OK: return "MSA_OK";
         case MSA_ERR_INVALID_ARG: return "MSA_ERR_INVALID_ARG: null pointer or invalid size";
-        case MSA_ERR_UNSUPPORTED: return "MSA_ERR_UNSUPPORTED: size not handled by this build";
+        case MSA_ERR_UNSUPPORTED: return "MSA_ERR_UNSUPPORTED: size not handled by this library";
         case MSA_ERR_WORKSPACE: return "MSA_ERR_WORKSPACE: workspace missing, short or misaligned";
         case MSA_ERR_CUDA: return "MSA_ERR_CUDA: a CUDA call or launch failed";
         case MSA_ERR_DEVICE_TIMEOUT: return "MSA_ERR_DEVICE_TIMEOUT: a device wait gave up";

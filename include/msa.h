@@ -83,7 +83,7 @@ typedef struct CUstream_st *msa_stream_t;
 typedef enum {
     MSA_OK = 0,
     MSA_ERR_INVALID_ARG = 1,    /* null pointer, non-positive size, H_q % H_kv != 0 */
-    MSA_ERR_UNSUPPORTED = 2,    /* a size this build does not handle (see below) */
+    MSA_ERR_UNSUPPORTED = 2,    /* a size this library does not handle (see below) */
     MSA_ERR_WORKSPACE = 3,      /* workspace missing, too small or not 256-byte aligned */
     MSA_ERR_CUDA = 4,           /* a CUDA call or kernel launch failed */
     MSA_ERR_DEVICE_TIMEOUT = 5, /* a bounded device-side wait gave up (device status) */
@@ -99,7 +99,7 @@ typedef enum {
     MSA_INDEX_KEYS_FP8_SHARED = 3   /* E4M3 [kv_capacity, 1, index_dim] + fp32 scale [kv_capacity, 1] */
 } msa_index_key_format_t;
 
-/* Problem shape.  Supported by this build: head_dim == index_dim == 128,
+/* Problem shape.  Supported by this library: head_dim == index_dim == 128,
  * block_size == 128, 1 <= top_k <= 64, num_kv_heads in {1, 2, 4, 8, 16},
  * num_q_heads / num_kv_heads in {1, 2, 4, 8, 16}, index heads in {1, 2, 4,
  * 8, 16} dividing num_kv_heads, batch <= 4096, max_kv_len <= 2^27,
