@@ -340,7 +340,11 @@ def measure_decode_fused(w, dev, steps, warmup, step_bytes, ref_ids):
     ms = ev0.elapsed_time(ev1) / steps
     kms = float(np.mean(ker)) if ker else float("nan")
     gbs = step_bytes / (ms / 1e3) / 1e9
-    res = {"entry": "msa_decode_step", "ms_per_step": ms, "kernel_ms": kms,
+    tr = kernel_traffic("decode_fused_step",
+                        os.path.join(ROOT, "block_sparse_attention_43_b200", "csrc", "decode_fused.cu"))
+    traffic = None if tr is None else tr["dram_bytes_per_unit"] * (step_bytes / tr["bytes_per_unit_basis"])
+    res = {"entry": "msa_decode_step", "ms_per_step": ms, "kernel_ms": kms, "traffic": traffic,
+           "algorithmic_bytes": step_bytes,
            "launches_per_step": len(trace) / steps, "gbs": gbs, "frac_of_hbm": gbs / peak,
            "kernel_gbs": step_bytes / (kms / 1e3) / 1e9, "peak_kind": kind,
            "ids_equal_two_call": same}
@@ -414,15 +418,15 @@ def measured_peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def kernel_traffic():
-    """Per-launch DRAM bytes of the dominant kernel from the last ncu capture,
-    or None when the kernel source changed since."""
+def kernel_traffic(name=DOMINANT, src=DOMINANT_SRC):
+    """Per-launch DRAM bytes of a kernel from its last ncu capture, or None
+    when the kernel source changed since."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
-    d = json.load(open(TRAFFIC_FILE)).get(DOMINANT)
+    d = json.load(open(TRAFFIC_FILE)).get(name)
     if not d:
         return None
-    h = hashlib.sha256(open(DOMINANT_SRC, "rb").read()).hexdigest()
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()
     if d.get("source_sha256") != h:
         return None
     return d
