@@ -118,6 +118,10 @@ msa_status_t check_shape(const msa_shape_t *s) {
         return MSA_ERR_UNSUPPORTED;
     if (s->batch > 4096 || s->max_kv_len > (1 << 27) || s->kv_capacity >= (1LL << 31))
         return MSA_ERR_UNSUPPORTED;
+    // Work units (one 128-token block of one sequence) are counted in 32 bits;
+    // sequences may share cache rows, so bound the count by batch x blocks.
+    if (static_cast<long long>(s->batch) * ((s->max_kv_len + kBlock - 1) / kBlock) >= (1LL << 31))
+        return MSA_ERR_UNSUPPORTED;
     return MSA_OK;
 }
 

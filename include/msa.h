@@ -103,7 +103,7 @@ typedef enum {
  * block_size == 128, 1 <= top_k <= 64, num_kv_heads in {1, 2, 4, 8, 16},
  * num_q_heads / num_kv_heads in {1, 2, 4, 8, 16}, index heads in {1, 2, 4,
  * 8, 16} dividing num_kv_heads, batch <= 4096, max_kv_len <= 2^27,
- * kv_capacity < 2^31. */
+ * batch * ceil(max_kv_len / 128) < 2^31, kv_capacity < 2^31. */
 typedef struct {
     int32_t batch;        /* B */
     int32_t q_len;        /* query rows per sequence: 1 = decode, lens[b] = full prefill */

@@ -159,3 +159,16 @@ def test_decode_step_rejects_unsupported_shapes(m):
                          top_k=4, kv_capacity=cap)
         assert m.lib.msa_decode_step_paged(ctypes.byref(s), *([0x1000] * 7), pps, 0.1, 0x1000,
                                            0x1000, 0x1000, 0x100000, 1 << 40, None) == 1
+
+
+def test_block_count_bound(m):
+    """batch x ceil(max_kv_len / 128) must stay below 2^31 (work units are
+    counted in 32 bits; sequences may share cache rows, so the pool size does
+    not bound it)."""
+    big = m.make_shape(batch=4096, q_len=1, max_kv_len=1 << 27, num_q_heads=64, num_kv_heads=8,
+                       top_k=16, kv_capacity=1 << 27)
+    assert m.msa_index_topk_workspace_size(big) == 0
+    assert m.msa_decode_step_workspace_size(big) == 0
+    ok = m.make_shape(batch=4096, q_len=1, max_kv_len=(1 << 26) - 128, num_q_heads=64,
+                      num_kv_heads=8, top_k=16, kv_capacity=1 << 27)
+    assert m.msa_index_topk_workspace_size(ok) > 0
