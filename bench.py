@@ -59,6 +59,10 @@ def parse():
                     help="skip the single-launch decode step attached to a decode run")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the sparse-branch backward measurement attached to a decode run")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other four workloads attached to a decode_1m run")
+    ap.add_argument("--cpu-rows", type=int, default=4096,
+                    help="query rows of the prefill_128k oracle sample (CPU baseline)")
     ap.add_argument("--prefill-steps", type=int, default=5)
     ap.add_argument("--prefill-len", type=int, default=None,
                     help="override the prefill length (profiling captures of a smaller case)")
@@ -353,6 +357,110 @@ def measure_decode_fused(w, dev, steps, warmup, step_bytes, ref_ids):
     return res
 
 
+def measure_decode_config(name, dev, steps, warmup, with_cpu=True):
+    """One decode workload at full size: the two-call step (index + top-k,
+    sparse attention) timed with CUDA events, the dominant kernel's roofline
+    from the library's trace, the same step as one fused launch, and the
+    oracle on every sequence of the workload as the CPU baseline."""
+    import block_sparse_attention_43_b200 as msa
+    from synthetic import make_workload
+    w = make_workload(name, dev)
+    stream = torch.cuda.Stream(device=dev)
+    eng = msa.MSA(batch=w.B, q_len=1, max_kv_len=max(w.lens_host), num_q_heads=w.H_q,
+                  num_kv_heads=w.H_kv, top_k=w.top_k, kv_capacity=w.kv_capacity, device=dev)
+
+    def step():
+        eng.index_topk(w.q_idx, w.k_idx, w.lens, w.kv_offsets, stream)
+        eng.sparse_attention(w.q, w.k, w.v, w.lens, w.kv_offsets, stream=stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    st = eng.device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"{name}: device status {msa.STATUS_NAMES.get(st, st)}")
+    ids_host = eng.block_ids.cpu().numpy()
+    step_bytes, kidx_bytes = decode_step_bytes(w, ids_host)
+    msa.msa_trace_enable(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    trace = msa.msa_trace_read()
+    msa.msa_trace_enable(False)
+    ms = ev0.elapsed_time(ev1) / steps
+    per = {}
+    for n, t in trace:
+        per[n] = per.get(n, 0.0) + t / steps
+    dom = [t for n, t in trace if n == DOMINANT]
+    dom_ms = float(np.mean(dom))
+    peak, _, _, kind = measured_peaks()
+    kb = index_kernel_bytes(w)
+    gbs = step_bytes / (ms / 1e3) / 1e9
+    fused = measure_decode_fused(w, dev, steps, warmup, step_bytes, ids_host)
+    cpu = None
+    if with_cpu:
+        c_gbs, dt, used, note = oracle_sample(w, seqs=range(w.B))
+        cpu = {"value": c_gbs, "unit": "GB/s", "cores": host_cores(), "threads_used": used,
+               "kind": "oracle", "sample": note, "seconds": dt}
+    lens = w.lens_host
+    res = {"workload": name, "batch": w.B,
+           "context": lens[0] if len(set(lens)) == 1 else
+           {"min": min(lens), "max": max(lens), "total": int(sum(lens))},
+           "H_q": w.H_q, "H_kv": w.H_kv, "top_k": w.top_k,
+           "ms_per_step": ms, "value": gbs, "unit": "GB/s", "pct_of_8TBps": 100.0 * gbs / 8000.0,
+           "frac_of_hbm": gbs / peak, "step_bytes": step_bytes, "index_key_bytes": kidx_bytes,
+           "tokens_per_s": w.B / (ms / 1e3),
+           "l2": "inputs larger than L2 (index keys %.2f GiB)" % (kidx_bytes / 2**30),
+           "roofline": {"bound": "hbm", "kernel": DOMINANT, "achieved": kb / (dom_ms / 1e3) / 1e9,
+                        "peak": peak, "peak_kind": kind, "unit": "GB/s",
+                        "frac": kb / (dom_ms / 1e3) / 1e9 / peak, "algorithmic_bytes": kb,
+                        "avg_launch_ms": dom_ms, "traffic": None},
+           "kernel_ms": per, "gpu_launches_per_step": len(trace) / steps,
+           "decode_step_fused": fused, "cpu_baseline": cpu}
+    tr = kernel_traffic()
+    if tr is not None:
+        res["roofline"]["traffic"] = tr["dram_bytes_per_unit"] * (kb / tr["bytes_per_unit_basis"])
+    del eng, w
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_prefill_config(name, dev, steps, warmup, with_cpu=True, cpu_rows=4096):
+    """One prefill workload at full size (index GEMM with fused top-k, then
+    the sparse branch), its sparse branch's roofline on useful FLOPs, and the
+    oracle on a seeded row sample as the CPU baseline."""
+    from synthetic import make_workload
+    r = measure_prefill(name, dev, steps, warmup)
+    _, tf_burst, tf_sus, kind = measured_peaks()
+    r["value"] = r["sparse_attn_tflops"]
+    r["unit"] = "TFLOP/s"
+    r["tokens_per_s"] = r["rows"] / (r["ms_per_step"] / 1e3)
+    r["roofline"] = {"bound": "tensor", "kernel": "sparse branch (prefill_* kernels)",
+                     "achieved": r["sparse_attn_tflops"], "peak": tf_burst,
+                     "peak_kind": kind + " burst", "unit": "TFLOP/s",
+                     "frac": r["sparse_attn_tflops"] / tf_burst,
+                     "sparse_attn_frac_of_burst": r["sparse_attn_tflops"] / tf_burst,
+                     "index_frac_of_burst": r["index_tflops"] / tf_burst,
+                     "peak_burst": tf_burst, "peak_sustained": tf_sus, "traffic": None}
+    r["cpu_baseline"] = None
+    if with_cpu:
+        w = make_workload(name, dev)
+        rps, dt, used, n, note, _ = oracle_prefill_sample(w, cpu_rows)
+        full = w.B * w.Sq
+        r["cpu_baseline"] = {"value": rps, "unit": "query rows/s", "cores": host_cores(),
+                             "threads_used": used, "kind": "oracle", "sample": note,
+                             "seconds": dt, "sample_rows": n,
+                             "extrapolated_full_seconds": dt * full / n if n < full else dt,
+                             "extrapolation": "linear in rows" if n < full else "none (all rows)"}
+        r["gpu_rows_per_s"] = full / (r["ms_per_step"] / 1e3)
+        del w
+        torch.cuda.empty_cache()
+    return r
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -462,7 +570,8 @@ def whole_job_rate(dist, world, units_per_rank, seconds_local, device):
     return units_per_rank * world / slow, slow
 
 
-def cores_used():
+def host_cores():
+    """Cores this process may run on (sched_getaffinity)."""
     try:
         return len(os.sched_getaffinity(0))
     except AttributeError:
@@ -470,34 +579,82 @@ def cores_used():
 
 
 # ----------------------------------------------------------------------------- CPU oracle leg
-def oracle_sample(w, dev_inputs=True):
-    """The oracle, as it stands, on sequence 0 of the workload (index branch
-    over all its index keys + sparse branch), on the host's cores.  Returns
-    (GB/s of that sequence's algorithmic bytes, seconds, threads, note)."""
+def oracle_sample(w, seqs=(0,)):
+    """The oracle, as it stands, on sequences `seqs` of a decode workload
+    (index branch over all their index keys + sparse branch), on the host's
+    cores.  Returns (GB/s of those sequences' algorithmic bytes, seconds,
+    threads the oracle could keep busy, note)."""
     import oracle
     from synthetic import bf16_bits
-    L = w.lens_host[0]
-    off = int(w.kv_offsets[0])
-    sl = slice(off, off + L)
-    q_idx = bf16_bits(w.q_idx[:1])
-    k_idx = bf16_bits(w.k_idx[sl])
-    q = bf16_bits(w.q[:1])
-    k = bf16_bits(w.k[sl])
-    v = bf16_bits(w.v[sl])
-    lens = np.array([L], np.int32)
-    offs = np.zeros(1, np.int64)
+    seqs = list(seqs)
+    lens_l, offs_l, sl = [], [], []
+    acc = 0
+    for b in seqs:
+        L = w.lens_host[b]
+        off = int(w.kv_offsets[b])
+        sl.append(slice(off, off + L))
+        lens_l.append(L)
+        offs_l.append(acc)
+        acc += L
+    cat = lambda t: np.concatenate([bf16_bits(t[x]) for x in sl]) if len(sl) > 1 else bf16_bits(t[sl[0]])
+    q_idx = bf16_bits(w.q_idx[seqs])
+    q = bf16_bits(w.q[seqs])
+    k_idx, k, v = cat(w.k_idx), cat(w.k), cat(w.v)
+    lens = np.array(lens_l, np.int32)
+    offs = np.array(offs_l, np.int64)
     threads = oracle.default_threads()
     t0 = time.perf_counter()
     sel = oracle.index_topk(q_idx, k_idx, lens, offs, top_k=w.top_k, n_threads=threads)
     oracle.sparse_attention(q, k, v, sel["block_ids"], lens, offs, n_threads=threads)
     dt = time.perf_counter() - t0
-    nbytes = L * w.H_kv * w.d_idx * 2
-    kv = sum(min(128, L - 128 * int(j)) for j in sel["block_ids"].ravel() if j >= 0) * w.D * 4
+    nbytes = int(lens.sum()) * w.H_kv * w.d_idx * 2
+    ids = sel["block_ids"].reshape(len(seqs), w.H_kv, w.top_k)
+    kv = sum(min(128, lens_l[i] - 128 * int(j)) for i in range(len(seqs)) for j in ids[i].ravel()
+             if j >= 0) * w.D * 4
     gbs = (nbytes + kv) / dt / 1e9
-    # The oracle spreads (row, group) work over threads: one decode row has
+    # The oracle spreads (row, group) jobs over threads: a decode row has
     # H_kv index jobs and H_q attention jobs.
-    used = min(threads, w.H_kv)
-    return gbs, dt, used, f"sequence 0 of {w.name} ({L} tokens, all {w.H_kv} groups, both stages)"
+    used = min(threads, len(seqs) * w.H_kv)
+    what = f"sequence 0 of {w.name} ({lens_l[0]} tokens" if seqs == [0] and w.B > 1 else \
+        f"all {len(seqs)} sequences of {w.name} ({int(lens.sum())} tokens"
+    return gbs, dt, used, what + f", all {w.H_kv} groups, both stages)"
+
+
+def oracle_prefill_sample(w, n_rows=4096, seed=2):
+    """The oracle, as it stands, on a seeded sample of a prefill workload's
+    query rows (uniform without replacement plus the block-edge rows), both
+    stages.  Returns (rows/s, seconds, threads, sample rows, note); the whole
+    prefill's oracle time is extrapolated linearly from the sample (a uniform
+    row sample has the mean per-row cost)."""
+    import oracle
+    from synthetic import bf16_bits
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from parity import sample_rows
+    R = w.B * w.Sq
+    rows = sample_rows(R, min(n_rows, R), seed) if n_rows < R else np.arange(R, dtype=np.int64)
+    a = dict(q_idx=bf16_bits(w.q_idx), k_idx=bf16_bits(w.k_idx), q=bf16_bits(w.q),
+             k=bf16_bits(w.k), v=bf16_bits(w.v), lens=w.lens.cpu().numpy(),
+             offs=w.kv_offsets.cpu().numpy())
+    threads = oracle.default_threads()
+    t0 = time.perf_counter()
+    sel = oracle.index_topk(a["q_idx"], a["k_idx"], a["lens"], a["offs"], top_k=w.top_k,
+                            rows=rows, n_threads=threads)
+    ids = np.full((R, w.H_kv, w.top_k), -1, np.int32)
+    ids[rows] = sel["block_ids"]
+    oracle.sparse_attention(a["q"], a["k"], a["v"], ids, a["lens"], a["offs"], scale=w.scale,
+                            rows=rows, n_threads=threads)
+    dt = time.perf_counter() - t0
+    # useful sparse-branch FLOPs of the sampled rows (4*D per row, head, visible kept key)
+    ids_s = sel["block_ids"].astype(np.int64)
+    b_of = rows // w.Sq
+    p = rows % w.Sq + (np.asarray(w.lens_host)[b_of] - w.Sq)
+    vis = np.where(ids_s == (p // 128)[:, None, None], (p % 128 + 1)[:, None, None], 128)
+    useful = int((vis * (ids_s >= 0)).sum()) * (w.H_q // w.H_kv) * 4 * w.D
+    used = min(threads, len(rows) * w.H_kv)
+    note = (f"{len(rows)} of {R} query rows of {w.name} (seeded uniform sample + block-edge rows), "
+            f"all {w.H_kv} groups, both stages" if len(rows) < R else
+            f"all {R} query rows of {w.name}, both stages")
+    return len(rows) / dt, dt, used, len(rows), note, useful
 
 
 def run_reference(args):
@@ -507,20 +664,27 @@ def run_reference(args):
     from synthetic import make_workload
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     w = make_workload(args.workload, dev)
+    prefill = args.workload.startswith("prefill")
+    unit = "TFLOP/s" if prefill else "GB/s"
     vals = []
     for i in range(args.warmup + args.steps):
-        gbs, dt, used, note = oracle_sample(w)
+        if prefill:
+            # a bounded row sample per step (rows/s scale linearly with rows)
+            _, dt, used, _, note, useful = oracle_prefill_sample(w, min(args.cpu_rows, 256), seed=2 + i)
+            v = useful / dt / 1e12
+        else:
+            v, dt, used, note = oracle_sample(w)
         if i >= args.warmup:
-            vals.append((gbs, dt))
+            vals.append((v, dt))
     gbs = float(np.mean([v[0] for v in vals]))
     ms = float(np.mean([v[1] for v in vals])) * 1e3
-    line = {"impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+    line = {"impl": "reference", "metric": METRIC, "value": gbs, "unit": unit, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": args.workload, "sample": note},
-            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": used, "kind": "oracle",
-                             "sample": note},
-            "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "cpu_baseline": {"value": gbs, "unit": unit, "cores": host_cores(),
+                             "threads_used": used, "kind": "oracle", "sample": note},
+            "e2e": {"value": gbs, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
@@ -589,6 +753,9 @@ def main():
     msa.msa_trace_enable(False)
     clk = clocks.stop()
 
+    kb = index_kernel_bytes(w)
+    head_cfg = {"workload": args.workload, "batch": w.B, "context": max(w.lens_host),
+                "H_q": w.H_q, "H_kv": w.H_kv, "top_k": w.top_k}
     launches = len(trace)
     dom = [t for n, t in trace if n == DOMINANT]
     dom_ms = float(np.mean(dom)) if dom else float("nan")
@@ -608,8 +775,8 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         gbs, dt, used, note = oracle_sample(w)
-        cpu = {"value": gbs, "unit": "GB/s", "cores": used, "kind": "oracle", "sample": note,
-               "seconds": dt}
+        cpu = {"value": gbs, "unit": "GB/s", "cores": host_cores(), "threads_used": used,
+               "kind": "oracle", "sample": note, "seconds": dt}
 
     fused = None
     if not args.no_fused and world == 1:
@@ -625,19 +792,33 @@ def main():
         backward = measure_backward("prefill_2k", dev, 20, 3)
 
     prefill = None
-    if not args.no_prefill and world == 1:
+    configs = None
+    if world == 1 and (not args.no_prefill or not args.no_configs):
         del eng
+        del w
         torch.cuda.empty_cache()
-        prefill = measure_prefill("prefill_128k", dev, args.prefill_steps, 2)
-        _, tf_burst, tf_sus, _ = measured_peaks()
-        prefill["roofline"] = {"bound": "tensor", "unit": "TFLOP/s",
-                               "sparse_attn_frac_of_burst": prefill["sparse_attn_tflops"] / tf_burst,
-                               "index_frac_of_burst": prefill["index_tflops"] / tf_burst,
-                               "peak_burst": tf_burst, "peak_sustained": tf_sus}
+    if not args.no_prefill and world == 1:
+        prefill = measure_prefill_config("prefill_128k", dev, args.prefill_steps, 2,
+                                         with_cpu=not args.no_cpu_baseline,
+                                         cpu_rows=args.cpu_rows)
+    if not args.no_configs and world == 1:
+        configs = {}
+        for name in ("decode_32k", "decode_ragged"):
+            configs[name] = measure_decode_config(name, dev, 100, 10,
+                                                  with_cpu=not args.no_cpu_baseline)
+        configs["prefill_2k"] = measure_prefill_config("prefill_2k", dev, 50, 5,
+                                                       with_cpu=not args.no_cpu_baseline)
 
     peak, _, _, peak_kind = measured_peaks()
-    kb = index_kernel_bytes(w)
     achieved = kb / (dom_ms / 1e3) / 1e9
+    if configs is not None:
+        # all five workloads side by side (the headline's own figures first)
+        configs = {"decode_1m": {"workload": args.workload, "ms_per_step": ms_step, "value": value,
+                                 "unit": "GB/s", "pct_of_8TBps": 100.0 * value / 8000.0,
+                                 "frac_of_hbm": value / peak, "tokens_per_s": head_cfg["batch"] / (ms_step / 1e3),
+                                 "roofline_frac": achieved / peak, "cpu_baseline": cpu,
+                                 "detail": "the headline fields of this line"},
+                   **configs, "prefill_128k": prefill}
     tr = kernel_traffic()
     traffic = None
     if tr is not None:
@@ -647,8 +828,7 @@ def main():
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": args.workload, "batch": w.B, "context": max(w.lens_host),
-                       "H_q": w.H_q, "H_kv": w.H_kv, "top_k": w.top_k, "block": 128,
+            "config": {**head_cfg, "block": 128,
                        "step_bytes": step_bytes, "index_key_bytes": kidx_bytes,
                        "pct_of_8TBps": 100.0 * value / world / 8000.0,
                        "l2": "inputs larger than L2 (index keys %.1f GiB per GPU)" % (kidx_bytes / 2**30),
@@ -663,6 +843,7 @@ def main():
             "e2e": e2e,
             "cpu_baseline": cpu,
             "prefill_128k": prefill,
+            "configs": configs,
             "decode_step_fused": fused,
             "index_variants": variants,
             "prefill_backward": backward,
@@ -682,6 +863,16 @@ def run_prefill_headline(args):
     clocks.start()
     r = measure_prefill(args.workload, dev, args.steps, max(args.warmup, 1), args.prefill_len)
     clk = clocks.stop()
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.prefill_len is None:
+        from synthetic import make_workload
+        w = make_workload(args.workload, dev)
+        rps, dt, used, n, note, useful = oracle_prefill_sample(w, args.cpu_rows)
+        cpu = {"value": useful / dt / 1e12, "unit": "TFLOP/s", "rows_per_s": rps,
+               "cores": host_cores(), "threads_used": used, "kind": "oracle", "sample": note,
+               "seconds": dt, "sample_rows": n,
+               "extrapolated_full_seconds": dt * r["rows"] / n}
+        del w
     _, tf_burst, tf_sus, kind = measured_peaks()
     if rank == 0:
         line = {"metric": METRIC, "value": r["sparse_attn_tflops"], "unit": "TFLOP/s",
@@ -696,7 +887,7 @@ def run_prefill_headline(args):
                              "peak_kind": kind + " burst", "unit": "TFLOP/s",
                              "frac": r["sparse_attn_tflops"] / tf_burst, "traffic": None},
                 "prefill": r, "clocks": clk, "gpu_launches": int(r["gpu_launches_per_step"] * args.steps),
-                "e2e": None, "cpu_baseline": None}
+                "e2e": None, "cpu_baseline": cpu}
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()

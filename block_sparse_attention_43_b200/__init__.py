@@ -28,7 +28,7 @@ EXPORTS = ("msa_index_topk_workspace_size", "msa_index_topk", "msa_index_topk_fp
            "msa_index_topk_static", "msa_sparse_attention_backward_workspace_size",
            "msa_sparse_attention_backward", "msa_decode_step_workspace_size",
            "msa_decode_step", "msa_decode_step_paged", "msa_read_device_status",
-           "msa_trace_enable",
+           "msa_set_wait_controls", "msa_trace_enable",
            "msa_trace_read",
            "msa_status_string")
 
@@ -91,6 +91,8 @@ def _load():
     lib.msa_decode_step_paged.restype = ctypes.c_int
     lib.msa_read_device_status.argtypes = [P, P]
     lib.msa_read_device_status.restype = ctypes.c_int
+    lib.msa_set_wait_controls.argtypes = [ctypes.c_uint64, ctypes.c_uint32]
+    lib.msa_set_wait_controls.restype = ctypes.c_int
     lib.msa_trace_enable.argtypes = [ctypes.c_int]
     lib.msa_trace_enable.restype = ctypes.c_int
     lib.msa_trace_read.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_float),
@@ -257,6 +259,16 @@ def msa_decode_step_paged(shape, q_idx, k_idx_pool, q, k_pool, v_pool, lens, pag
 
 def msa_read_device_status(workspace, stream=None) -> int:
     return lib.msa_read_device_status(_ptr(workspace), _stream(stream))
+
+
+# msa_stall_t bits
+STALL_NONE, STALL_INDEX_DECODE, STALL_DECODE_STEP = 0, 1, 2
+
+
+def msa_set_wait_controls(wait_limit_ns: int = 0, stall_mask: int = STALL_NONE) -> None:
+    """Testing aid: the bounded device waits' limit (0 = default) and the
+    kernels that wait once on something that never happens."""
+    _check(lib.msa_set_wait_controls(int(wait_limit_ns), int(stall_mask)), "msa_set_wait_controls")
 
 
 def msa_trace_enable(on: bool) -> None:

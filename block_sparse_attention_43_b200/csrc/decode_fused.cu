@@ -93,7 +93,6 @@ __device__ __forceinline__ unsigned long long now_ns() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-constexpr unsigned long long kWaitNs = 2000000000ull;   // bounded waits give up after 2 s
 
 // Score rows padded to 32 floats: rows of different (sequence, group) never
 // share a cache line, so no SM can hold a stale copy of a row it reads.
@@ -188,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // per group), stored and counted with a device-scope atomic; the lane
         // that counts a sequence's last score asks the producer (through a
         // shared-memory FIFO) to queue that sequence's top-k.
-        const unsigned long long t0 = now_ns();
+        const unsigned long long lim = wait_limit_ns(P.status);
         for (int k = 0;; ++k) {
             const int slot = k % kRedQ;
             bool have = !*abort_flag && mbar_wait(&S.red_full[slot], (k / kRedQ) & 1, P.status);
@@ -210,8 +209,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (__any_sync(0xffffffffu, last) && lane == 0) {
                 // at most kRedQ + kQueue units finish between two producer
                 // polls, so the FIFO does not fill; the wait is a safety net
+                const unsigned long long t0 = now_ns();
                 while (S.topk_wr - ld_volatile(&S.topk_rd) >= kFifo) {
-                    if (*abort_flag || now_ns() - t0 > kWaitNs) { set_status(P.status, kStatusTimeout); *abort_flag = 1; break; }
+                    if (*abort_flag || now_ns() - t0 > lim) { set_status(P.status, kStatusTimeout); *abort_flag = 1; break; }
                     __nanosleep(64);
                 }
                 S.topk_fifo[S.topk_wr % kFifo] = b;
@@ -278,7 +278,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             return true;
         };
-        const unsigned long long t0 = now_ns();
+        const unsigned long long lim = wait_limit_ns(P.status);
+        // A test may make this CTA's first item wait on a word nothing writes.
+        bool stall = (stall_mask(P.status) & kStallDecodeFused) != 0;
+        unsigned long long t_idle = now_ns();   // start of the current idle spell
         while (ok) {
             if (!drain_topk()) { ok = false; break; }
             if (pending < 0 && attn_left) {
@@ -299,8 +302,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // may be among them.
                 const int item = pending;
                 pending = -1;
-                while (ld_volatile(P.aq_flag + item) == 0) {
-                    if (!drain_topk() || *abort_flag || now_ns() - t0 > kWaitNs) {
+                const int *flag = stall ? P.status + kCtlNeverWord : P.aq_flag + item;
+                stall = false;
+                const unsigned long long t0 = now_ns();   // this wait's own clock
+                while (ld_volatile(flag) == 0) {
+                    if (!drain_topk() || *abort_flag || now_ns() - t0 > lim) {
                         set_status(P.status, kStatusTimeout);
                         ok = false;
                         break;
@@ -331,11 +337,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_3d(S.ring[sv], &tmV, 0, g, tok, &S.full[sv]);
                     tma_load_3d(S.ring[sv] + 16384, &tmV, 64, g, tok, &S.full[sv]);
                 }
+                t_idle = now_ns();
                 continue;
             }
             if (index_left) {
                 const int u = u_next;
-                if (u >= U) { index_left = false; continue; }
+                if (u >= U) { index_left = false; t_idle = now_ns(); continue; }
                 u_next = atomicAdd(c_unit, 1);
                 // read now, used at the next pass of the loop
                 if (pending >= 0) pending_flag = ld_volatile(P.aq_flag + pending);
@@ -354,15 +361,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(&S.full[slot], bytes);
                     bulk_g2s(S.ring[slot], kbase + (t_first + t0s) * H * kDim, bytes, &S.full[slot], pol);
                 }
+                t_idle = now_ns();
                 continue;
             }
             if (!attn_left) break;
-            if (*abort_flag || now_ns() - t0 > kWaitNs) { set_status(P.status, kStatusTimeout); ok = false; break; }
+            // No work taken in this pass: an idle spell, bounded from its start.
+            if (*abort_flag || now_ns() - t_idle > lim) { set_status(P.status, kStatusTimeout); ok = false; break; }
+            continue;
         }
         // A top-k this CTA's bookkeeper has still to request must be queued
         // before the end: wait until it has finished every unit pushed here.
+        const unsigned long long t_end = now_ns();
         while (ok && ld_volatile(&S.book_done) < units_pushed) {
-            if (!drain_topk() || *abort_flag || now_ns() - t0 > kWaitNs) {
+            if (!drain_topk() || *abort_flag || now_ns() - t_end > lim) {
                 set_status(P.status, kStatusTimeout);
                 ok = false;
                 break;

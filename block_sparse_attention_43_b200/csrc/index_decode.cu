@@ -30,6 +30,7 @@ struct Smem {
     uint8_t ring[kStages][kStageBytes];
     uint64_t full[kStages];
     uint64_t empty[kStages];
+    uint64_t idle;                 // never arrived on: the test stall waits here
     int prefix[kMaxBatch + 1];
     float red[2][16];
     int abort_flag;
@@ -55,6 +56,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_decode_kernel(const IndexDe
             mbar_init(&S.full[i], 1);
             mbar_init(&S.empty[i], kConsumerWarps);
         }
+        mbar_init(&S.idle, 1);
         S.abort_flag = 0;
         fence_mbar_init();
     }
@@ -126,11 +128,10 @@ __global__ void __launch_bounds__(kThreads, 1) index_decode_kernel(const IndexDe
                              pol);
                 }
             }
-            if (!ok) {
-                // Drain: let every copy already issued land before exiting.
-                for (int k = max(0, it - kStages); k < it; ++k)
-                    mbar_wait(&S.full[k % kStages], (k / kStages) & 1, nullptr);
-            }
+            // Drain: every copy already issued lands before this thread
+            // exits (after an abort the consumers may not wait for them).
+            for (int k = max(0, it - kStages); k < it; ++k)
+                mbar_wait(&S.full[k % kStages], (k / kStages) & 1, nullptr);
         }
         return;
     }
@@ -143,6 +144,11 @@ __global__ void __launch_bounds__(kThreads, 1) index_decode_kernel(const IndexDe
     int cur_b = -1;
     int it = 0, unit_iter = 0;
     const __nv_bfloat16 *qbase = static_cast<const __nv_bfloat16 *>(P.q_idx);
+    // A test may ask the consumers to wait once on a barrier nobody arrives
+    // on: the wait gives up after the call's limit and the CTA aborts.
+    if (stall_mask(P.status) & kStallIndexDecode) {
+        if (!mbar_wait(&S.idle, 0, P.status)) *(volatile int *)&S.abort_flag = 1;
+    }
 
     for (int u = blockIdx.x; u < U; u += gridDim.x, ++unit_iter) {
         int b, j;

@@ -78,6 +78,32 @@ namespace {
 
 constexpr size_t kAlign = 256;
 
+// Wait controls set by msa_set_wait_controls, copied into every workspace
+// header a call clears (bytes 128..143; see msa_device.cuh).
+struct WaitControls {
+    unsigned long long limit_ns;
+    unsigned stall;
+    unsigned never;     // stays 0: the word a stalled wait polls
+};
+std::mutex g_ctl_mu;
+WaitControls g_ctl = {0, 0, 0};
+std::atomic<bool> g_ctl_on{false};
+
+// Clears the first `bytes` of a workspace (header first) and writes the
+// wait controls into its header when a test has set them.
+cudaError_t clear_header(void *ws, size_t bytes, cudaStream_t s) {
+    cudaError_t e = cudaMemsetAsync(ws, 0, bytes, s);
+    if (e != cudaSuccess || !g_ctl_on.load(std::memory_order_acquire)) return e;
+    WaitControls c;
+    {
+        std::lock_guard<std::mutex> lock(g_ctl_mu);
+        c = g_ctl;
+    }
+    // From pageable memory: the source is staged before this returns.
+    return cudaMemcpyAsync(static_cast<uint8_t *>(ws) + kCtlLimitWord * 4, &c, sizeof(c),
+                           cudaMemcpyHostToDevice, s);
+}
+
 size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool pow2_le16(int x) { return x == 1 || x == 2 || x == 4 || x == 8 || x == 16; }
@@ -226,7 +252,7 @@ msa_status_t index_topk_impl(const msa_shape_t *shape, const void *q_idx, const 
     float *scores = reinterpret_cast<float *>(ws + kWsHeaderBytes);
     const int nb_max = nb_max_of(shape);
 
-    if (cudaMemsetAsync(ws, 0, kWsHeaderBytes, s) != cudaSuccess) return MSA_ERR_CUDA;
+    if (clear_header(ws, kWsHeaderBytes, s) != cudaSuccess) return MSA_ERR_CUDA;
     if (shape->q_len > 1) {
         IndexRowsArgs a;
         a.q_idx = q_idx; a.k_idx = k_idx; a.lens = lens; a.kv = kv; a.k_scale = nullptr;
@@ -285,7 +311,7 @@ msa_status_t sparse_attention_impl(const msa_shape_t *shape, const void *q, cons
     if (st != MSA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    if (cudaMemsetAsync(ws, 0, kWsHeaderBytes + L.tickets_bytes, s) != cudaSuccess)
+    if (clear_header(ws, kWsHeaderBytes + L.tickets_bytes, s) != cudaSuccess)
         return MSA_ERR_CUDA;
     if (use_prefill_path(shape)) {
         PrefillArgs p;
@@ -446,7 +472,7 @@ msa_status_t msa_sparse_attention_backward(const msa_shape_t *shape, const void 
         return MSA_ERR_MISALIGNED;
     if ((st = check_ws(workspace, workspace_bytes, kWsHeaderBytes)) != MSA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(workspace, 0, kWsHeaderBytes, s) != cudaSuccess) return MSA_ERR_CUDA;
+    if (clear_header(workspace, kWsHeaderBytes, s) != cudaSuccess) return MSA_ERR_CUDA;
     AttnBwdArgs a;
     a.q = q; a.k_cache = k_cache; a.v_cache = v_cache; a.dout = d_out; a.ids = block_ids;
     a.lens = lens; a.kv = packed_map(shape, kv_offsets); a.dq = dq; a.dk = dk; a.dv = dv;
@@ -499,7 +525,7 @@ static msa_status_t decode_step_impl(const msa_shape_t *shape, const void *q_idx
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     // status word, claim counters and per-call flags: one contiguous range
-    if (cudaMemsetAsync(ws, 0, L.zero_hi, s) != cudaSuccess) return MSA_ERR_CUDA;
+    if (clear_header(ws, L.zero_hi, s) != cudaSuccess) return MSA_ERR_CUDA;
     DecodeFusedArgs a;
     a.q_idx = q_idx; a.k_idx = k_idx; a.q = q; a.k_cache = k_cache; a.v_cache = v_cache;
     a.lens = lens; a.kv = kv;
@@ -553,6 +579,17 @@ msa_status_t msa_read_device_status(const void *workspace, msa_stream_t stream) 
         return MSA_ERR_CUDA;
     if (word & kStatusTimeout) return MSA_ERR_DEVICE_TIMEOUT;
     if (word & kStatusBadLens) return MSA_ERR_BAD_LENS;
+    return MSA_OK;
+}
+
+msa_status_t msa_set_wait_controls(uint64_t wait_limit_ns, uint32_t stall_mask) {
+    {
+        std::lock_guard<std::mutex> lock(g_ctl_mu);
+        g_ctl.limit_ns = wait_limit_ns;
+        g_ctl.stall = stall_mask;
+        g_ctl.never = 0;
+    }
+    g_ctl_on.store(wait_limit_ns != 0 || stall_mask != 0, std::memory_order_release);
     return MSA_OK;
 }
 

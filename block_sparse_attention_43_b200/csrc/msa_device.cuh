@@ -19,11 +19,25 @@ constexpr int kDim = 128;       // head dim == index dim
 constexpr int kStatusBadLens = 1;   // lens / kv_offsets / block ids out of range
 constexpr int kStatusTimeout = 2;   // a bounded wait gave up
 
-// A bounded wait gives up after this long (globaltimer nanoseconds).
+// A bounded wait gives up after this long (globaltimer nanoseconds) unless
+// the workspace header sets another limit (below).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+// Waits shorter than this never read the header's limit.
+constexpr unsigned long long kWaitCheckNs = 20000ull;
 
-// Workspace header: status word + per-(row, group) arrival tickets follow.
+// Workspace header (256 bytes, cleared by every call): status word at byte 0;
+// bytes 4..127 belong to the kernels of a call; bytes 128..143 are the wait
+// controls, which a call fills right after clearing the header when a test
+// has set them (msa_set_wait_controls): the wait limit in ns (u64 at 128,
+// 0 = kWaitLimitNs), a stall mask (u32 at 136: kernels that see their bit
+// wait once on something that never happens, so their bounded-wait path
+// runs) and a word nothing ever writes (u32 at 140).
 constexpr size_t kWsHeaderBytes = 256;
+constexpr int kCtlLimitWord = 32;    // in ints from the status word
+constexpr int kCtlStallWord = 34;
+constexpr int kCtlNeverWord = 35;
+constexpr unsigned kStallIndexDecode = MSA_STALL_INDEX_DECODE;
+constexpr unsigned kStallDecodeFused = MSA_STALL_DECODE_STEP;
 
 __device__ __forceinline__ void set_status(int *status, int bit) {
     if (status) atomicOr(status, bit);
@@ -92,15 +106,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs, records kStatusTimeout and returns false; never spins forever.
+// The wait limit of the call whose status word is `status` (nullptr: the
+// default).
+__device__ __forceinline__ unsigned long long wait_limit_ns(const int *status) {
+    if (!status) return kWaitLimitNs;
+    const unsigned long long v =
+        *reinterpret_cast<const volatile unsigned long long *>(status + kCtlLimitWord);
+    return v ? v : kWaitLimitNs;
+}
+
+// The stall mask of the call (0 unless a test set it).
+__device__ __forceinline__ unsigned stall_mask(const int *status) {
+    return status ? *reinterpret_cast<const volatile unsigned *>(status + kCtlStallWord) : 0u;
+}
+
+// Wait for the phase with the given parity to complete.  Each wait gives up
+// after the call's limit (measured from the start of this wait), records
+// kStatusTimeout and returns false; it never spins forever.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *status) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_timer_ns();
+    unsigned long long lim = 0;
     while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
-            set_status(status, kStatusTimeout);
-            return false;
+        const unsigned long long dt = global_timer_ns() - t0;
+        if (dt > kWaitCheckNs) {
+            if (lim == 0) lim = wait_limit_ns(status);
+            if (dt > lim) {
+                set_status(status, kStatusTimeout);
+                return false;
+            }
         }
     }
     return true;

@@ -16,7 +16,10 @@ namespace {
 
 // 256-byte header (device status word) + 4 MiB of block scores: enough for a
 // decode batch with batch * index heads * ceil(max_kv_len / 128) <= 1,048,576
-// (e.g. 4 sequences x 8 groups at 1M tokens, or 64 x 8 at 256k).
+// (e.g. 4 sequences x 8 groups at 1M tokens, or 64 x 8 at 256k).  Prefill
+// rows with bf16 keys use only the header.  The address of the array is
+// looked up once per device and kept, so a primary-context reset between
+// calls is not supported.
 constexpr size_t kStaticScratchBytes = 256 + (size_t(4) << 20);
 
 static __device__ __align__(256) unsigned char g_scratch[kStaticScratchBytes];
@@ -47,7 +50,9 @@ extern "C" msa_status_t msa_index_topk_static(const msa_shape_t *shape, const vo
                                               const int64_t *kv_offsets, int32_t *block_ids,
                                               float *block_scores, msa_stream_t stream) {
     const size_t need = msa_index_topk_workspace_size(shape);
-    if (need == 0)   // rejected shape: let the checks report which error, nothing is launched
+    if (need == 0 || (shape->index_key_format != MSA_INDEX_KEYS_BF16 &&
+                      shape->index_key_format != MSA_INDEX_KEYS_BF16_SHARED))
+        // rejected shape or key format: msa_index_topk reports which error, nothing is launched
         return msa_index_topk(shape, q_idx, k_idx, lens, kv_offsets, block_ids, block_scores,
                               nullptr, 0, stream);
     if (need > kStaticScratchBytes) return MSA_ERR_WORKSPACE;   // shape too large for g_scratch

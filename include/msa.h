@@ -290,13 +290,23 @@ MSA_API msa_status_t msa_kv_append(const msa_shape_t *shape, int32_t n_new, cons
  * to another allocator, loops that must not stall on cudaMalloc).  The paper
  * has no counterpart; this is a library convenience.
  *   Scratch: a file-scope device array of 256 B + 4 MiB that every GPU which
- *   loads the library holds until the process exits.  Shapes whose
- *   msa_index_topk_workspace_size exceeds that (batch * q_len * index heads
- *   * ceil(max_kv_len / 128) > 1,048,576 block scores) are rejected with
- *   MSA_ERR_WORKSPACE; nothing is launched and nothing is allocated.
+ *   loads the library holds until the process exits.  What a call needs of
+ *   it depends on the rows:
+ *     - decode (q_len == 1): the 256 B header plus one fp32 block score per
+ *       (sequence, index head, block), so batch * index heads *
+ *       ceil(max_kv_len / 128) may be at most 1,048,576 (e.g. 4 sequences x
+ *       8 index heads at 1M tokens, or 64 x 8 at 256k); larger shapes are
+ *       rejected with MSA_ERR_WORKSPACE before anything is launched;
+ *     - prefill (q_len > 1): the selection happens inside the tensor-core
+ *       kernel, so only the 256 B header is used and no shape is refused
+ *       for its size.
+ *   Only the bf16 index-key formats are accepted (the E4M3 formats return
+ *   MSA_ERR_UNSUPPORTED, as msa_index_topk does).
  *   Set-up: the first call on each device looks up the array's device
- *   address with cudaGetSymbolAddress (that device must be current); make
- *   that first call before any stream capture.
+ *   address with cudaGetSymbolAddress (that device must be current) and
+ *   keeps it for later calls; make that first call before any stream
+ *   capture.  Tearing down a device's primary context between calls
+ *   (cudaDeviceReset) is not supported: the kept address would be stale.
  *   Sharing: every call on a device uses the same array and it keeps the last
  *   call's contents; calls that may overlap on the GPU (different streams,
  *   no ordering) race on it and must be serialised by the caller.
@@ -313,6 +323,36 @@ MSA_API msa_status_t msa_index_topk_static(const msa_shape_t *shape, const void 
  * MSA_ERR_DEVICE_TIMEOUT), or MSA_ERR_CUDA if the wait or copy failed.  Every
  * call clears the word when it starts. */
 MSA_API msa_status_t msa_read_device_status(const void *workspace, msa_stream_t stream);
+
+/* Kernels that msa_set_wait_controls can make wait on something that never
+ * happens (bits of stall_mask). */
+typedef enum {
+    MSA_STALL_NONE = 0,
+    MSA_STALL_INDEX_DECODE = 1, /* decode index kernel of msa_index_topk (bf16 keys, one per
+                                   index head): its consumer warps wait once on an mbarrier
+                                   nobody arrives on */
+    MSA_STALL_DECODE_STEP = 2   /* msa_decode_step: each CTA's first attention item waits on
+                                   a flag nobody sets */
+} msa_stall_t;
+
+/* Testing aid for the bounded device waits; production code never needs it.
+ * Every wait inside the kernels (an mbarrier phase, a flag another CTA sets)
+ * gives up after a limit, measured from the start of that wait, records
+ * MSA_ERR_DEVICE_TIMEOUT in the workspace's status word, lets the copies it
+ * already issued land, frees what it holds and returns.  This call sets, for
+ * the whole process and every later call until it is called again:
+ *   wait_limit_ns  the limit (0 = the default, 2 s);
+ *   stall_mask     msa_stall_t bits: the named kernels wait once on something
+ *                  that never happens, so their give-up path runs.  The call
+ *                  still returns MSA_OK; msa_read_device_status then reports
+ *                  MSA_ERR_DEVICE_TIMEOUT and that call's outputs are
+ *                  unspecified (no memory outside the caller's buffers and
+ *                  the workspace is touched).  Clear the mask and the next
+ *                  call works normally on the same workspace.
+ * The values travel to the device in the workspace header (bytes 128..143),
+ * which every call fills right after clearing it.  Not meant to be changed
+ * while other threads are issuing calls.  Returns MSA_OK. */
+MSA_API msa_status_t msa_set_wait_controls(uint64_t wait_limit_ns, uint32_t stall_mask);
 
 /* Kernel timing trace (off by default).  After msa_trace_enable(1), every
  * call records a pair of CUDA events around each kernel it launches, on that

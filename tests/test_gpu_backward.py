@@ -2,10 +2,12 @@
 blocks) through the C ABI against the CPU oracle's exact derivative, on the
 same bf16 inputs and the same selection.
 
-Tolerance: relative L2 <= 1e-2 and max-abs <= 2 % of the largest reference
-magnitude, per gradient.  The kernel rounds P and dZ to bf16 as operands of
-the products (2^-9 relative each) and writes dQ as bf16; dK and dV are fp32
-sums of those products.
+Tolerance: relative L2 <= 5e-3 (the forward's bound) and max-abs <= 2 % of
+the largest reference magnitude, per gradient.  The kernel rounds P and dZ to
+bf16 as operands of the products (at most 2^-9 relative each, about 1.1e-3
+RMS for round-to-nearest) and writes dQ as bf16 (another 2^-9); dK and dV
+are fp32 sums of those products, so the rounding adds in quadrature to about
+2e-3 RMS, inside 5e-3.
 """
 import numpy as np
 import pytest
@@ -15,7 +17,7 @@ import block_sparse_attention_43_b200 as m
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
-REL_L2 = 1e-2
+REL_L2 = 5e-3
 MAX_ABS_FRAC = 2e-2
 
 
