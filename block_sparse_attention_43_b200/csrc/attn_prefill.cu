@@ -12,21 +12,25 @@
 // Exactness: softmax is invariant to the shift subtracted before exp, so the
 // partial sums of different blocks can be added directly if they share one
 // shift per (row, head).  The shift is the row's exact max over its own block
-// (pass A).  It is safe (no overflow) whenever the Cauchy-Schwarz bound
-// scale*|q|*max|k| exceeds it by at most 64 (base 2); rows where the bound
-// does not prove that are flagged and get their exact max over all kept keys
-// from the fix-up pass before pass B adds anything.
+// (pass A) plus 4 (base 2).  Partial outputs are added in fp16: the adds at
+// L2 cost bytes, not operations, so 16-bit partials halve the pass's bound,
+// and fp16 keeps 11 significant bits (the bf16 output keeps 8).  A partial
+// is checked before it is added: if any of its values exceeds 65504 / top_k
+// (or is not finite), the sum of at most top_k partials could overflow, so
+// that (row, head) is flagged instead, its partials are dropped, and the
+// exact pass recomputes its output from scratch after the others (rare: a
+// kept block would have to beat the own block's max by about 2^9 or more).
 //
 // Passes (one stream, no host synchronisation):
-//   knorm      max token norm of k per (sequence, group)
 //   bucket_*   rows that kept block j (j != own) bucketed by (sequence, group,
 //              8192-row range, j); buckets become work items of <= 256 rows
 //   pass A     own block of every row (causal), query-outer: writes the
-//              partial output, sum and shift
-//   fixup      flagged (row, head) only: exact shift, rescale pass A's partials
+//              partial output (fp16), sum and shift
 //   pass B     the other kept blocks, block-outer: partials added into the
-//              accumulator with bulk fp32 reductions (cp.reduce.async.bulk)
+//              accumulator with bulk fp16 reductions (cp.reduce.async.bulk)
 //   finalize   out = accumulator / sum, bf16
+//   exact      flagged (row, head) only: softmax over every kept key in fp32
+//              on CUDA cores, written over finalize's output
 //
 // Passes A and B share one kernel: per 16-row tile, 16 rows x 8 heads = 128
 // TMEM lanes; the tile's Q rows are gathered by TMA (one 8-head x 64-dim box
@@ -38,8 +42,9 @@
 // output in shared memory and hands it to the bulk-copy engine as one fp32
 // add-reduction per row: the reductions, which bound pass B, then never sit
 // in the SM's load/store queue in front of the softmax's memory operations.
-// The accumulator interleaves the 8 heads of a row at 16-byte granularity,
-// so a row's partial output is one contiguous 4 KiB run.
+// The accumulator interleaves the 8 heads of a row at 16-byte granularity
+// (8 dims of one head per 16 bytes), so a row's partial output is one
+// contiguous 2 KiB run.
 #include "msa_device.cuh"
 #include "msa_internal.h"
 
@@ -58,7 +63,7 @@ constexpr uint32_t kTmemCols = 512;        // S, P and O[2]
 // TMEM columns: S (128 fp32), P (64 columns of bf16 pairs), O[2] (2 x 128 fp32).
 constexpr uint32_t kColS = 0, kColP = 128, kColO = 256;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kSafeLog2 = 64.f;          // max (bound - shift) accepted, base 2
+constexpr float kShiftPad = 4.f;           // shift = own-block max + this (base 2)
 
 __device__ __forceinline__ bool seq_ok(const PrefillArgs &P, int b, int &L) {
     L = P.lens[b];
@@ -124,7 +129,7 @@ __device__ __forceinline__ long long n_items(const PrefillArgs &P) {
 struct Smem {
     uint8_t kv[2][65536];                  // K lo, K hi, V lo, V hi (16 KiB each)
     uint8_t q[2][32768];                   // gathered Q tile, two swizzled halves
-    uint8_t ostage[kEpiWarps][8192];       // epilogue: 4 rows x 64 dims x 8 heads fp32 per warp
+    uint8_t ostage[kEpiWarps][8192];       // epilogue: 4 rows x 128 dims x 8 heads fp16 per warp
     uint64_t kv_full[2], kv_empty[2], q_full[2], q_empty[2];
     uint64_t s_full, s_empty, o_full[2], o_empty[2];
     uint64_t p_full, p_empty;
@@ -140,7 +145,11 @@ struct Smem {
 static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory over the per-block limit");
 
 constexpr int kQueue = 4;
-constexpr int kQueueReaders = 1 + kSoftWarps + kEpiWarps;   // MMA thread + one per consumer warp
+// Q loader warps: pass A one TMA thread (whole 16-row boxes), pass B two
+// warps gathering rows with cp.async.
+template <int MODE> constexpr int kLoaderWarps = MODE == 0 ? 1 : 2;
+// MMA thread + one per loader, softmax and epilogue warp
+template <int MODE> constexpr int kQueueReaders = 1 + kLoaderWarps<MODE> + kSoftWarps + kEpiWarps;
 
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
     uint64_t d = static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
@@ -162,7 +171,7 @@ __device__ __forceinline__ float fast_exp2(float x) {
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_prefill_kernel(const __grid_constant__ CUtensorMap tmQ,
+    attn_prefill_kernel(const __grid_constant__ CUtensorMap tmQ16,
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const PrefillArgs P) {
     extern __shared__ uint8_t smem_raw[];
@@ -175,10 +184,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.kv_full[i], 1);
             mbar_init(&S.kv_empty[i], 1);
-            mbar_init(&S.q_full[i], 1);
-            // Pass A reads each Q tile once more (its norms) after the MMA: the
-            // softmax warps release it; in pass B the MMA commit does.
-            mbar_init(&S.q_empty[i], MODE == 0 ? kSoftWarps : 1);
+            mbar_init(&S.q_full[i], kLoaderWarps<MODE>);
+            mbar_init(&S.q_empty[i], 1);          // released by the MMA commit
             mbar_init(&S.o_full[i], 1);
             mbar_init(&S.o_empty[i], kEpiWarps);
         }
@@ -189,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 4; ++i) mbar_init(&S.xbar[i], 64);   // every lane of both warps
         for (int i = 0; i < kQueue; ++i) {
             mbar_init(&S.item_full[i], 1);
-            mbar_init(&S.item_empty[i], kQueueReaders);
+            mbar_init(&S.item_empty[i], kQueueReaders<MODE>);
         }
         S.abort_flag = 0;
         fence_mbar_init();
@@ -224,80 +231,114 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer (whole warp:
-        // lane 0 owns the barriers, lane r gathers tile row r)
+        // ------------------------------------------------ producer (lane 0): claims
+        // and decodes items, publishes them, loads each item's K and V block
+        // lanes 1-31 go straight to the final barrier
         if (lane == 0) {
-            prefetch_tensormap(&tmQ);
             prefetch_tensormap(&tmK);
             prefetch_tensormap(&tmV);
-        }
-        int ki = 0, qt = 0;
-        bool ok = true;
-        for (int n = 0; ok; ++n) {
-            long long it = 0;
-            if (lane == 0) {
+            int ki = 0;
+            bool ok = true;
+            for (int n = 0; ok; ++n) {
                 const int slot = n % kQueue;
-                if (n >= kQueue && (*abort_flag || !mbar_wait(&S.item_empty[slot],
-                                                              ((n / kQueue) - 1) & 1, P.status))) {
-                    it = -1;
-                } else {
-                    // Decode once here; the other roles read the result.
-                    it = atomicAdd(reinterpret_cast<unsigned long long *>(counter), 1ull);
-                    Item d;
-                    if (it >= total) {
-                        it = total;
-                        d.n = -1;
-                    } else {
-                        d = item_at<MODE>(P, it);
-                    }
-                    S.item_q[slot] = d;
-                    mbar_arrive(&S.item_full[slot]);
-                }
-            }
-            it = __shfl_sync(0xffffffffu, it, 0);
-            if (it < 0) { ok = false; break; }
-            if (it >= total) break;
-            __syncwarp();
-            const Item x = S.item_q[n % kQueue];
-            if (x.n <= 0) continue;
-            const int kvs = ki & 1;
-            if (lane == 0) {
-                if (ki >= 2 &&
-                    (*abort_flag || !mbar_wait(&S.kv_empty[kvs], ((ki >> 1) - 1) & 1, P.status))) {
+                if (n >= kQueue && (*abort_flag || !mbar_wait(&S.item_empty[slot], ((n / kQueue) - 1) & 1, P.status))) {
                     ok = false;
-                } else {
-                    const int tok = static_cast<int>(kv_block_row(P.kv, x.b, x.j, P.status));
-                    mbar_arrive_expect_tx(&S.kv_full[kvs], 65536);
-                    tma_load_3d(S.kv[kvs], &tmK, 0, x.g, tok, &S.kv_full[kvs]);
-                    tma_load_3d(S.kv[kvs] + 16384, &tmK, 64, x.g, tok, &S.kv_full[kvs]);
-                    tma_load_3d(S.kv[kvs] + 32768, &tmV, 0, x.g, tok, &S.kv_full[kvs]);
-                    tma_load_3d(S.kv[kvs] + 49152, &tmV, 64, x.g, tok, &S.kv_full[kvs]);
+                    break;
                 }
+                // Decode once here; the other roles read the result.
+                long long it = atomicAdd(reinterpret_cast<unsigned long long *>(counter), 1ull);
+                Item x;
+                if (it >= total) x.n = -1;
+                else x = item_at<MODE>(P, it);
+                S.item_q[slot] = x;
+                mbar_arrive(&S.item_full[slot]);
+                if (x.n < 0) break;
+                if (x.n == 0) continue;
+                const int kvs = ki & 1;
+                if (ki >= 2 && (*abort_flag || !mbar_wait(&S.kv_empty[kvs], ((ki >> 1) - 1) & 1, P.status))) {
+                    ok = false;
+                    break;
+                }
+                const int tok = static_cast<int>(kv_block_row(P.kv, x.b, x.j, P.status));
+                mbar_arrive_expect_tx(&S.kv_full[kvs], 65536);
+                tma_load_3d(S.kv[kvs], &tmK, 0, x.g, tok, &S.kv_full[kvs]);
+                tma_load_3d(S.kv[kvs] + 16384, &tmK, 64, x.g, tok, &S.kv_full[kvs]);
+                tma_load_3d(S.kv[kvs] + 32768, &tmV, 0, x.g, tok, &S.kv_full[kvs]);
+                tma_load_3d(S.kv[kvs] + 49152, &tmV, 64, x.g, tok, &S.kv_full[kvs]);
+                ++ki;
             }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-            ++ki;
+            if (!ok) *abort_flag = 1;
+        }
+    } else if (warp == 2 || (warp == 3 && MODE == 1)) {
+        // ------------------------------------------------ Q loaders
+        // Pass A: a tile is 16 consecutive query rows, two TMA boxes of
+        // 16 rows x 8 heads x 64 dims.  Pass B: the tile's rows are scattered
+        // (bucket entries), and one small TMA box per row would be bound by
+        // the bulk engine's per-copy cost (shared with the reductions), so
+        // two warps gather each 2 KiB (row, group) slice with 16-byte
+        // cp.async copies straight into the 128-byte-swizzled layout the MMA
+        // reads; each warp signals a tile once its copies have landed.
+        const int lw = warp - 2;
+        int qt = 0, n = 0, prev_qs = -1;
+        bool ok = true;
+        if (MODE == 0 && lane == 0) prefetch_tensormap(&tmQ16);
+        Item x;
+        while (ok) {
+            if (!next_item(n++, true, x)) { ok = false; break; }
+            if (x.n < 0) break;
+            if (x.n == 0) continue;
             for (int t0 = 0; t0 < x.n; t0 += kTileRows, ++qt) {
                 const int qs = qt & 1;
-                const int nr = min(kTileRows, x.n - t0);
-                // Row index of this lane's gather, loaded before the wait.
-                const int row = lane < nr ? static_cast<int>(tile_row<MODE>(P, x, t0 + lane)) : 0;
-                if (lane == 0) {
-                    if (qt >= 2 &&
-                        (*abort_flag || !mbar_wait(&S.q_empty[qs], ((qt >> 1) - 1) & 1, P.status)))
-                        ok = false;
-                    else
-                        mbar_arrive_expect_tx(&S.q_full[qs], nr * 2 * 1024);
+                int myrow = -1;                      // lane k < 8: row of this warp's k-th slot
+                if (MODE == 1 && lane < 8 && t0 + lw + 2 * lane < x.n)
+                    myrow = P.bucket_rows[x.rows_off + t0 + lw + 2 * lane];
+                bool free_ = qt < 2 || (!*abort_flag && mbar_wait(&S.q_empty[qs], ((qt >> 1) - 1) & 1, P.status));
+                free_ = __all_sync(0xffffffffu, free_);
+                if (!free_) { ok = false; break; }
+                if (MODE == 0) {
+                    if (lane == 0) {
+                        const int row0 = x.b * P.Sq + x.i_lo + t0;
+                        mbar_arrive_expect_tx(&S.q_full[qs], 32768);
+                        tma_load_3d(S.q[qs], &tmQ16, 0, x.g * kG, row0, &S.q_full[qs]);
+                        tma_load_3d(S.q[qs] + 16384, &tmQ16, 64, x.g * kG, row0, &S.q_full[qs]);
+                    }
+                    __syncwarp();
+                    continue;
                 }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-                if (lane < nr) {
-                    tma_load_3d(S.q[qs] + lane * 1024, &tmQ, 0, x.g * kG, row, &S.q_full[qs]);
-                    tma_load_3d(S.q[qs] + 16384 + lane * 1024, &tmQ, 64, x.g * kG, row, &S.q_full[qs]);
+                const uint32_t qbase = smem_u32(S.q[qs]);
+#pragma unroll 1
+                for (int k = 0; k < 8; ++k) {
+                    const int r = __shfl_sync(0xffffffffu, myrow, k);
+                    if (r < 0) continue;
+                    const int rr = lw + 2 * k;       // tile row
+                    const uint8_t *src = static_cast<const uint8_t *>(P.q) +
+                                         (static_cast<long long>(r) * P.H_q + x.g * kG) * (kDim * 2);
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) {
+                        const int ch = lane + 32 * qq;   // 16-byte chunk of the 2 KiB slice
+                        const int h = ch >> 4, c = ch & 15, m = rr * kG + h;
+                        cp_async16(qbase + (c >> 3) * 16384 + m * 128 + (((c & 7) ^ (m & 7)) << 4),
+                                   src + ch * 16);
+                    }
                 }
+                cp_async_commit();
+                if (prev_qs >= 0) {
+                    // the previous tile's copies have landed: hand it to the MMA
+                    cp_async_wait_but1();
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.q_full[prev_qs]);
+                }
+                prev_qs = qs;
             }
         }
-        if (!ok && lane == 0) *abort_flag = 1;
+        if (MODE == 1) {
+            cp_async_wait_all();                     // nothing lands after the CTA ends
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (ok && prev_qs >= 0 && lane == 0) mbar_arrive(&S.q_full[prev_qs]);
+        }
+        if (!ok) *abort_flag = 1;
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------ MMA issuer
         const uint32_t idesc_qk = umma_idesc_bf16(128, 128);
@@ -350,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     umma_bf16_ss(tmem + kColS, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&S.s_full);
-                if (MODE == 1) umma_commit(&S.q_empty[qs]);
+                umma_commit(&S.q_empty[qs]);
                 // PV of the previous tile runs behind this tile's QK.
                 if (pv_pending >= 0 && !issue_pv(pv_pending, pv_kvs, pv_last)) { ok = false; break; }
                 pv_pending = qt;
@@ -428,32 +469,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 have = __all_sync(0xffffffffu, have);
                 if (!have) { ok = false; break; }
                 tc_fence_after();
-                float nq = 0.f;                        // pass A: |q|^2 of this (row, head)
-                if (MODE == 0) {
-                    // The Q tile goes back to the producer as soon as its norms
-                    // are read, so the next tiles' loads overlap this softmax.
-                    bool qok = !*abort_flag && mbar_wait(&S.q_full[qt & 1], (qt >> 1) & 1, P.status);
-                    qok = __all_sync(0xffffffffu, qok);
-                    if (!qok) { ok = false; break; }
-                    if (ch == 0 && valid) {
-                        const uint8_t *qs = S.q[qt & 1];
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            const uint4 w = *reinterpret_cast<const uint4 *>(
-                                qs + (c >> 3) * 16384 + swz128(m, c & 7));
-                            const uint32_t a4[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                nq = fmaf(bf16lo(a4[e]), bf16lo(a4[e]), nq);
-                                nq = fmaf(bf16hi(a4[e]), bf16hi(a4[e]), nq);
-                            }
-                        }
-                    }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&S.q_empty[qt & 1]);
-                }
                 const uint32_t sa = lane_addr + kColS;
-                long long lim = 127;                   // last visible column of the row
+                int lim = 127;                         // last visible column of the row
                 uint32_t a[32], b[32];
                 tmem_ld32r(sa + ch * 64, a);
                 tmem_ld32r(sa + ch * 64 + 32, b);
@@ -466,7 +483,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // lanes, other half) through shared memory.
                     const long long p = static_cast<long long>(x.L) - P.Sq +
                                         (row - static_cast<long long>(x.b) * P.Sq);
-                    lim = p - static_cast<long long>(x.j) * 128;
+                    // clamped: the row's position lies in this block when valid
+                    lim = static_cast<int>(max(-1LL, min(127LL, p - static_cast<long long>(x.j) * 128)));
                     float mx = -INFINITY;
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
@@ -482,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     xok = __all_sync(0xffffffffu, xok);
                     if (!xok) { ok = false; break; }
                     mx = fmaxf(mx, S.xmax[ch ^ 1][m]);
-                    shift = valid ? mx : 0.f;
+                    shift = valid ? mx + kShiftPad : 0.f;
                 }
                 // S is in registers: the next tile's QK may overwrite it.
                 tc_fence_before();
@@ -527,17 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.p_full);
                 if (valid) atomicAdd(P.l_acc + row * P.H_q + x.g * kG + h, l);
-                if (MODE == 0) {
-                    if (ch == 0 && valid) {
-                        // Shift of this (row, head) and the safety test of the bound.
-                        const float bound = fabsf(sl2) * sqrtf(nq) * P.knorm[x.b * P.H_kv + x.g];
-                        const long long idx = row * P.H_q + x.g * kG + h;
-                        P.m_arr[idx] = shift;
-                        const uint8_t fl = !(bound - shift <= kSafeLog2);   // NaN-safe
-                        P.flags[idx] = fl;
-                        if (fl) atomicAdd(P.flag_count, 1);
-                    }
-                }
+                if (MODE == 0 && ch == 0 && valid) P.m_arr[row * P.H_q + x.g * kG + h] = shift;
             }
             x = xn;
         }
@@ -545,12 +553,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp >= kEpiWarp0) {
         // ------------------------------------------------ epilogue
         // Warp w owns the TMEM lanes of w % 4 (tile rows 4(w%4) .. +3, all 8
-        // heads), one (tile row, head) per thread.  Each half of the output
-        // dims goes through the warp's 8 KiB staging slot, laid out as the
+        // heads), one (tile row, head) per thread.  A tile's partial output
+        // goes through the warp's 8 KiB staging slot in fp16, laid out as the
         // accumulator is (a row's 8 heads interleaved at 16-byte granularity),
-        // and leaves as one 2 KiB bulk copy (pass A) or bulk fp32 add (pass B)
-        // per row, issued by the row's head-0 lane: the reductions run on the
-        // bulk-copy engine.
+        // and leaves as one 2 KiB bulk copy (pass A) or bulk fp16 add (pass
+        // B) per row, issued by lane 0: the reductions run on the bulk-copy
+        // engine.  A partial with a value above P.acc_limit (or not finite)
+        // is not added: its (row, head) is flagged for the exact pass.
         const int w = warp & 3;
         const int m = w * 32 + lane;
         const int ri = m / kG, h = m % kG;
@@ -588,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!fetch(xn)) { ok = false; break; }
                     if (xn.n > 0) row_nx = load_row(xn, 0);
                 }
-                float *dst4[4];
+                __half *dst4[4];
 #pragma unroll
                 for (int r4 = 0; r4 < 4; ++r4) {
                     const long long rr = __shfl_sync(0xffffffffu, row, r4 * 8);
@@ -598,6 +607,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 have = __all_sync(0xffffffffu, have);
                 if (!have) { ok = false; break; }
                 tc_fence_after();
+                // The slot is free once the bulk engine has read the last tile's rows.
+                if (issuer) bulk_wait_read_all();
+                __syncwarp();
+                bool fits = true;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t a[32], b[32];
@@ -610,29 +623,42 @@ __global__ void __launch_bounds__(kThreads, 1)
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&S.o_empty[os]);
                     }
-                    // The slot is free once the bulk engine has read the last groups.
-                    if (issuer) bulk_wait_read_all();
-                    __syncwarp();
                     if (valid) {
 #pragma unroll
-                        for (int q4 = 0; q4 < 16; ++q4) {
-                            const uint32_t *r = q4 < 8 ? a + 4 * q4 : b + 4 * (q4 - 8);
-                            *reinterpret_cast<uint4 *>(stage + q4 * 128 + h * 16) =
-                                make_uint4(r[0], r[1], r[2], r[3]);
-                        }
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (issuer) {
+                        for (int c8 = 0; c8 < 8; ++c8) {
+                            const uint32_t *r = c8 < 4 ? a + 8 * c8 : b + 8 * (c8 - 4);
+                            uint32_t pk[4];
 #pragma unroll
-                        for (int r4 = 0; r4 < 4; ++r4) {
-                            if (!dst4[r4]) continue;
-                            float *g = dst4[r4] + half * (kDim * kG / 2);
-                            if (MODE == 0) bulk_s2g(g, stage0 + r4 * 2048, 2048);
-                            else bulk_s2g_add_f32(g, stage0 + r4 * 2048, 2048);
+                            for (int e = 0; e < 4; ++e) {
+                                const float lo = __uint_as_float(r[2 * e]);
+                                const float hi = __uint_as_float(r[2 * e + 1]);
+                                fits = fits && fabsf(lo) <= P.acc_limit && fabsf(hi) <= P.acc_limit;
+                                pk[e] = pack_f16x2(lo, hi);
+                            }
+                            *reinterpret_cast<uint4 *>(stage + ((half * 8 + c8) * kG + h) * 16) =
+                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
                         }
-                        bulk_commit();
                     }
+                }
+                if (valid && !fits) {
+                    // Too large for the fp16 sum (or not finite): add zeros and
+                    // leave this (row, head) to the exact pass.
+#pragma unroll
+                    for (int c = 0; c < 16; ++c)
+                        *reinterpret_cast<uint4 *>(stage + (c * kG + h) * 16) = make_uint4(0, 0, 0, 0);
+                    P.flags[row * P.H_q + x.g * kG + h] = 1;
+                    atomicAdd(P.flag_count, 1);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (issuer) {
+#pragma unroll
+                    for (int r4 = 0; r4 < 4; ++r4) {
+                        if (!dst4[r4]) continue;
+                        if (MODE == 0) bulk_s2g(dst4[r4], stage0 + r4 * 2048, 2048);
+                        else bulk_s2g_add_f16(dst4[r4], stage0 + r4 * 2048, 2048);
+                    }
+                    bulk_commit();
                 }
             }
             x = xn;
@@ -652,43 +678,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- helpers
-// Max token norm of k per (sequence, group); one warp per (sequence, group,
-// 128-token block).
-__global__ void knorm_kernel(const PrefillArgs P) {
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-    const int nb = P.nb_max;
-    const long long total = static_cast<long long>(P.B) * P.H_kv * nb;
-    for (long long w = warp; w < total; w += (static_cast<long long>(gridDim.x) * blockDim.x) >> 5) {
-        const int j = static_cast<int>(w % nb);
-        const int g = static_cast<int>((w / nb) % P.H_kv);
-        const int b = static_cast<int>(w / (static_cast<long long>(nb) * P.H_kv));
-        int L;
-        if (!seq_ok(P, b, L) || j * 128 >= L) continue;
-        const __nv_bfloat16 *k = static_cast<const __nv_bfloat16 *>(P.k_cache);
-        const long long row0 = kv_block_row(P.kv, b, j, P.status);
-        float best = 0.f;
-        for (int t = lane; t < min(L - j * 128, 128); t += 32) {
-            const uint4 *row = reinterpret_cast<const uint4 *>(k + ((row0 + t) * P.H_kv + g) * kDim);
-            float s = 0.f;
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const uint4 v = row[c];
-                const uint32_t a4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    s = fmaf(bf16lo(a4[e]), bf16lo(a4[e]), s);
-                    s = fmaf(bf16hi(a4[e]), bf16hi(a4[e]), s);
-                }
-            }
-            best = fmaxf(best, sqrtf(s));
-        }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
-        // Norms are >= 0, so their float bits order like ints (NaN -> flagged later).
-        if (lane == 0) atomicMax(reinterpret_cast<int *>(P.knorm) + b * P.H_kv + g, __float_as_int(best));
-    }
-}
-
 // Buckets of one (sequence, group, row range), built by one CTA: rows that
 // kept block j (j != own) are counted, given offsets in the range's own
 // region of bucket_rows, split into work items of <= kItemRows rows, and
@@ -836,62 +825,8 @@ __global__ void bucket_shift_kernel(const PrefillArgs P) {
     }
 }
 
-// Flagged (row, head): exact max logit over the row's other kept keys, then
-// the own-block partials are rescaled to the new shift.  Exits at once when
-// no row was flagged.  One warp per (row, group).
-__global__ void fixup_kernel(const PrefillArgs P) {
-    if (*P.flag_count == 0) return;
-    const int lane = threadIdx.x & 31;
-    const long long total = static_cast<long long>(P.B) * P.Sq * P.H_kv;
-    const float sl2 = P.softmax_scale * kLog2e;
-    const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(P.q);
-    const __nv_bfloat16 *kb = static_cast<const __nv_bfloat16 *>(P.k_cache);
-    for (long long pair = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-         pair < total; pair += (static_cast<long long>(gridDim.x) * blockDim.x) >> 5) {
-        const long long row = pair / P.H_kv;
-        const int g = static_cast<int>(pair % P.H_kv);
-        const int b = static_cast<int>(row / P.Sq), i = static_cast<int>(row % P.Sq);
-        int L;
-        if (!seq_ok(P, b, L)) continue;
-        const long long p = static_cast<long long>(L) - P.Sq + i;
-        for (int h = 0; h < kG; ++h) {
-            const long long idx = row * P.H_q + g * kG + h;
-            if (!P.flags[idx]) continue;
-            const __nv_bfloat16 *qh = qb + idx * kDim;
-            float mx = -INFINITY;
-            for (int s = 0; s < P.K; ++s) {
-                const int j = P.ids[(row * P.n_idx + g / (P.H_kv / P.n_idx)) * P.K + s];
-                if (j < 0 || j >= p / 128) continue;
-                const long long row0 = kv_block_row(P.kv, b, j, P.status);
-                for (int t = lane; t < 128; t += 32) {
-                    const __nv_bfloat16 *kt = kb + ((row0 + t) * P.H_kv + g) * kDim;
-                    float d = 0.f;
-                    for (int c = 0; c < kDim; ++c) d = fmaf(__bfloat162float(qh[c]), __bfloat162float(kt[c]), d);
-                    mx = fmaxf(mx, d * sl2);
-                }
-            }
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            const float m_own = P.m_arr[idx];
-            const float m_new = fmaxf(m_own, mx);
-            const float sc = exp2f(m_own - m_new);
-            float *acc = P.o_acc + (row * P.H_kv + g) * (kDim * kG) + h * 4;
-            for (int c = lane; c < kDim / 4; c += 32) {
-                float4 *v = reinterpret_cast<float4 *>(acc + c * 4 * kG);
-                float4 x = *v;
-                x.x *= sc; x.y *= sc; x.z *= sc; x.w *= sc;
-                *v = x;
-            }
-            __syncwarp();
-            if (lane == 0) {
-                P.l_acc[idx] *= sc;
-                P.m_arr[idx] = m_new;
-            }
-        }
-    }
-}
-
-// out = accumulator / sum, bf16.  One warp per (row, group): lane = (head, 32 dims).
+// out = accumulator / sum, bf16.  One warp per (row, group): lane = (head,
+// 32 dims = four 16-byte chunks of the fp16 accumulator).
 __global__ void finalize_kernel(const PrefillArgs P) {
     const int lane = threadIdx.x & 31;
     const int h = lane >> 2, qd = lane & 3;
@@ -908,17 +843,88 @@ __global__ void finalize_kernel(const PrefillArgs P) {
             continue;
         }
         const float inv = 1.f / P.l_acc[row * P.H_q + g * kG + h];
-        const float *acc = P.o_acc + pair * (kDim * kG) + h * 4;
+        const uint4 *acc = reinterpret_cast<const uint4 *>(P.o_acc + pair * (kDim * kG));
 #pragma unroll
-        for (int c = 0; c < 8; c += 2) {
-            const float4 a = *reinterpret_cast<const float4 *>(acc + (qd * 8 + c) * 4 * kG);
-            const float4 bq = *reinterpret_cast<const float4 *>(acc + (qd * 8 + c + 1) * 4 * kG);
-            uint4 w;
-            w.x = pack_bf16x2(a.x * inv, a.y * inv);
-            w.y = pack_bf16x2(a.z * inv, a.w * inv);
-            w.z = pack_bf16x2(bq.x * inv, bq.y * inv);
-            w.w = pack_bf16x2(bq.z * inv, bq.w * inv);
-            *reinterpret_cast<uint4 *>(out + c * 4) = w;
+        for (int c = 0; c < 4; ++c) {
+            const uint4 v = acc[(qd * 4 + c) * kG + h];      // dims 8(4qd+c) .. +7 of head h
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+            uint32_t o4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w4[e]));
+                o4[e] = pack_bf16x2(f.x * inv, f.y * inv);
+            }
+            *reinterpret_cast<uint4 *>(out + c * 8) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        }
+    }
+}
+
+// Flagged (row, head) pairs (a partial too large for the fp16 sum): softmax
+// over every kept key of the row, in fp32 on CUDA cores, written over the
+// finalized output.  Exits at once when nothing was flagged.  One warp per
+// (row, group); per flagged head a lane owns 4 output dims, each key's logit
+// is a warp-reduced dot product.
+__global__ void exact_rows_kernel(const PrefillArgs P) {
+    if (*P.flag_count == 0) return;
+    const int lane = threadIdx.x & 31;
+    const long long total = static_cast<long long>(P.B) * P.Sq * P.H_kv;
+    const float sl2 = P.softmax_scale * kLog2e;
+    const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(P.q);
+    const __nv_bfloat16 *kb = static_cast<const __nv_bfloat16 *>(P.k_cache);
+    const __nv_bfloat16 *vb = static_cast<const __nv_bfloat16 *>(P.v_cache);
+    for (long long pair = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+         pair < total; pair += (static_cast<long long>(gridDim.x) * blockDim.x) >> 5) {
+        const long long row = pair / P.H_kv;
+        const int g = static_cast<int>(pair % P.H_kv);
+        const int b = static_cast<int>(row / P.Sq), i = static_cast<int>(row % P.Sq);
+        int L;
+        if (!seq_ok(P, b, L)) continue;
+        const long long p = static_cast<long long>(L) - P.Sq + i;
+        const int own = static_cast<int>(p / 128);
+        const int32_t *ids = P.ids + (row * P.n_idx + g / (P.H_kv / P.n_idx)) * P.K;
+        for (int h = 0; h < kG; ++h) {
+            const long long idx = row * P.H_q + g * kG + h;
+            if (!P.flags[idx]) continue;
+            float q4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) q4[e] = __bfloat162float(qb[idx * kDim + lane * 4 + e]);
+            // logit of token t (row0 = first cache row of its block), warp-reduced
+            auto logit = [&](long long krow) -> float {
+                const __nv_bfloat16 *kt = kb + (krow * P.H_kv + g) * kDim + lane * 4;
+                float d = 0.f;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) d = fmaf(q4[e], __bfloat162float(kt[e]), d);
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+                return d * sl2;
+            };
+            float mx = -INFINITY;
+            for (int s = 0; s < P.K; ++s) {
+                const int j = ids[s];
+                if (j < 0 || j > own) continue;
+                const long long row0 = kv_block_row(P.kv, b, j, P.status);
+                const int nt = j == own ? static_cast<int>(p - 128LL * own) + 1 : 128;
+                for (int t = 0; t < nt; ++t) mx = fmaxf(mx, logit(row0 + t));
+            }
+            float l = 0.f, o4[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int s = 0; s < P.K; ++s) {
+                const int j = ids[s];
+                if (j < 0 || j > own) continue;
+                const long long row0 = kv_block_row(P.kv, b, j, P.status);
+                const int nt = j == own ? static_cast<int>(p - 128LL * own) + 1 : 128;
+                for (int t = 0; t < nt; ++t) {
+                    const float w = exp2f(logit(row0 + t) - mx);
+                    l += w;
+                    const __nv_bfloat16 *vt = vb + ((row0 + t) * P.H_kv + g) * kDim + lane * 4;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) o4[e] = fmaf(w, __bfloat162float(vt[e]), o4[e]);
+                }
+            }
+            __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(P.out) + idx * kDim + lane * 4;
+            const float inv = 1.f / l;
+            const uint2 wv = make_uint2(pack_bf16x2(o4[0] * inv, o4[1] * inv),
+                                        pack_bf16x2(o4[2] * inv, o4[3] * inv));
+            *reinterpret_cast<uint2 *>(out) = wv;
         }
     }
 }
@@ -951,11 +957,11 @@ size_t prefill_workspace_layout(int B, int Sq, int H_q, int H_kv, int K, int max
     const size_t per_range_rows = static_cast<size_t>(L->rows_per_range) * (K > 1 ? K - 1 : 1);
     L->items_per_range = static_cast<int>(L->nb_max + per_range_rows / kItemRows + 1);
     size_t o = kWsHeaderBytes;
-    L->knorm = o;        o += up(static_cast<size_t>(B) * H_kv * 4);
     L->cnt = o;          o += up(static_cast<size_t>(L->n_buckets) * 4);
     L->cur = o;          o += up(static_cast<size_t>(L->n_buckets) * 4);
     L->l_acc = o;        o += up(static_cast<size_t>(rows) * H_q * 4);
-    L->zero_end = o;                                  // [knorm, zero_end) is cleared per call
+    L->flags = o;        o += up(static_cast<size_t>(rows) * H_q);
+    L->zero_end = o;                                  // [cnt, zero_end) is cleared per call
     L->off = o;          o += up(static_cast<size_t>(L->n_buckets) * 4);
     L->item_off = o;     o += up(static_cast<size_t>(L->n_buckets) * 4);
     L->item_bucket = o;  o += up(static_cast<size_t>(L->n_ranges_total) * L->items_per_range * 4);
@@ -964,9 +970,8 @@ size_t prefill_workspace_layout(int B, int Sq, int H_q, int H_kv, int K, int max
     L->rows = o;         o += up(static_cast<size_t>(L->n_ranges_total) * per_range_rows * 4);
     L->shift = o;        o += up(static_cast<size_t>(L->n_ranges_total) * per_range_rows * kG * 4);
     L->item_desc = o;    o += up(static_cast<size_t>(L->n_ranges_total) * L->items_per_range * 32);
-    L->o_acc = o;        o += up(static_cast<size_t>(rows) * H_q * kDim * 4);
+    L->o_acc = o;        o += up(static_cast<size_t>(rows) * H_q * kDim * 2);
     L->m_arr = o;        o += up(static_cast<size_t>(rows) * H_q * 4);
-    L->flags = o;        o += up(static_cast<size_t>(rows) * H_q);
     L->total = o;
     return o;
 }
@@ -974,7 +979,6 @@ size_t prefill_workspace_layout(int B, int Sq, int H_q, int H_kv, int K, int max
 cudaError_t launch_prefill_attention(const PrefillArgs &a0, uint8_t *ws, const PrefillLayout &L,
                                      cudaStream_t s) {
     PrefillArgs a = a0;
-    a.knorm = reinterpret_cast<float *>(ws + L.knorm);
     a.bucket_cnt = reinterpret_cast<int *>(ws + L.cnt);
     a.bucket_cur = reinterpret_cast<int *>(ws + L.cur);
     a.bucket_off = reinterpret_cast<int *>(ws + L.off);
@@ -985,13 +989,14 @@ cudaError_t launch_prefill_attention(const PrefillArgs &a0, uint8_t *ws, const P
     a.bucket_rows = reinterpret_cast<int *>(ws + L.rows);
     a.bucket_shift = reinterpret_cast<float *>(ws + L.shift);
     a.item_desc = reinterpret_cast<int *>(ws + L.item_desc);
-    a.o_acc = reinterpret_cast<float *>(ws + L.o_acc);
+    a.o_acc = reinterpret_cast<__half *>(ws + L.o_acc);
     a.l_acc = reinterpret_cast<float *>(ws + L.l_acc);
     a.m_arr = reinterpret_cast<float *>(ws + L.m_arr);
     a.flags = reinterpret_cast<uint8_t *>(ws + L.flags);
     a.flag_count = reinterpret_cast<int *>(ws + 4);
     a.item_total = reinterpret_cast<long long *>(ws + 8);
     a.item_next = reinterpret_cast<long long *>(ws + 16);   // [pass A, pass B]
+    a.acc_limit = 65504.f / static_cast<float>(a.K > 0 ? a.K : 1);
     a.nb_max = L.nb_max;
     a.n_ranges = L.n_ranges;
     a.n_ranges_total = L.n_ranges_total;
@@ -999,17 +1004,13 @@ cudaError_t launch_prefill_attention(const PrefillArgs &a0, uint8_t *ws, const P
     a.items_per_range = L.items_per_range;
 
     CUtensorMap tq, tk, tv;
-    if (!encode_q_gather_map(&tq, a.q, a.H_q, static_cast<long long>(a.B) * a.Sq) ||
+    if (!encode_q_rows_map(&tq, a.q, a.H_q, static_cast<long long>(a.B) * a.Sq, kTileRows) ||
         !encode_kv_tensor_map(&tk, a.k_cache, a.H_kv, a.kv.capacity) ||
         !encode_kv_tensor_map(&tv, a.v_cache, a.H_kv, a.kv.capacity))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaMemsetAsync(ws + L.knorm, 0, L.zero_end - L.knorm, s);
+    cudaError_t e = cudaMemsetAsync(ws + L.cnt, 0, L.zero_end - L.cnt, s);
     if (e != cudaSuccess) return e;
     const int sms = device_sm_count();
-    {
-        TraceScope t(s, "prefill_knorm");
-        knorm_kernel<<<sms * 4, 256, 0, s>>>(a);
-    }
     {
         TraceScope t(s, "prefill_bucket");
         bucket_build_kernel<<<static_cast<unsigned>(L.n_ranges_total), kBuildThreads, 0, s>>>(a);
@@ -1019,10 +1020,6 @@ cudaError_t launch_prefill_attention(const PrefillArgs &a0, uint8_t *ws, const P
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_pass<0>(tq, tk, tv, a, s, "prefill_attn_own_block")) != cudaSuccess) return e;
     {
-        TraceScope t(s, "prefill_fixup");
-        fixup_kernel<<<sms * 4, 256, 0, s>>>(a);
-    }
-    {
         TraceScope t(s, "prefill_bucket_shift");
         bucket_shift_kernel<<<sms * 8, 256, 0, s>>>(a);
     }
@@ -1030,6 +1027,10 @@ cudaError_t launch_prefill_attention(const PrefillArgs &a0, uint8_t *ws, const P
     {
         TraceScope t(s, "prefill_finalize");
         finalize_kernel<<<sms * 8, 256, 0, s>>>(a);
+    }
+    {
+        TraceScope t(s, "prefill_exact_rows");
+        exact_rows_kernel<<<sms * 4, 256, 0, s>>>(a);
     }
     return cudaGetLastError();
 }

@@ -56,14 +56,14 @@ bool encode_kv_tensor_map(CUtensorMap *map, const void *base, int H_kv, long lon
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool encode_q_gather_map(CUtensorMap *map, const void *q, int H_q, long long rows) {
+bool encode_q_rows_map(CUtensorMap *map, const void *q, int H_q, long long rows, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDim), static_cast<cuuint64_t>(H_q),
                                 static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDim) * 2,
                                    static_cast<cuuint64_t>(kDim) * 2 * H_q};
-    const cuuint32_t box[3] = {64, 8, 1};
+    const cuuint32_t box[3] = {64, 8, static_cast<cuuint32_t>(box_rows)};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -134,7 +135,6 @@ struct PrefillArgs {
     int n_idx;              // index heads: group g reads ids of g / (H_kv / n_idx)
     float softmax_scale;
     // workspace views (filled by launch_prefill_attention)
-    float *knorm;
     int *bucket_cnt, *bucket_cur, *bucket_off, *bucket_rows;  // per (range, block j)
     int *item_off;          // first item of each bucket, counted inside its range
     int *item_bucket;       // [range][item] -> block j
@@ -143,15 +143,17 @@ struct PrefillArgs {
     long long *range_count, *range_item_off;
     long long *item_total;
     long long *item_next;   // claim counters of pass A and pass B (zeroed per call)
-    float *o_acc, *l_acc, *m_arr;
-    uint8_t *flags;
+    __half *o_acc;          // [rows][H_kv][128 dims x 8 heads] fp16, heads interleaved per 8 dims
+    float *l_acc, *m_arr;   // [rows][H_q] softmax sums and shifts (base 2)
+    uint8_t *flags;         // [rows][H_q] 1: recomputed by the exact pass
     int *flag_count;
+    float acc_limit;        // largest partial value added in fp16: 65504 / top_k
     int nb_max, n_ranges, rows_per_range, items_per_range;
     long long n_ranges_total;
 };
 struct PrefillLayout {
-    size_t knorm, cnt, cur, l_acc, zero_end, off, item_off, item_bucket, range_count,
-        range_item_off, rows, shift, item_desc, o_acc, m_arr, flags, total;
+    size_t cnt, cur, l_acc, flags, zero_end, off, item_off, item_bucket, range_count,
+        range_item_off, rows, shift, item_desc, o_acc, m_arr, total;
     int nb_max, n_ranges, rows_per_range, items_per_range;
     long long n_ranges_total, n_buckets;
 };
@@ -160,8 +162,9 @@ size_t prefill_workspace_layout(int B, int Sq, int H_q, int H_kv, int K, int max
                                 PrefillLayout *L);
 cudaError_t launch_prefill_attention(const PrefillArgs &a, uint8_t *ws, const PrefillLayout &L,
                                      cudaStream_t s);
-// 3-D map over q [rows, H_q, 128] with an 8-head x 64-dim box (one row).
-bool encode_q_gather_map(CUtensorMap *map, const void *q, int H_q, long long rows);
+// 3-D map over q [rows, H_q, 128] with a box of 64 dims x 8 heads x box_rows
+// rows, 128-byte swizzle.
+bool encode_q_rows_map(CUtensorMap *map, const void *q, int H_q, long long rows, int box_rows);
 
 // Appends n_new tokens per sequence after its current length (kv_append.cu):
 // src[i] [B][n_new][H_kv][128] -> dst[i] at rows of tokens lens[b] .. + n_new - 1.

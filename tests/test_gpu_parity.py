@@ -114,15 +114,42 @@ def test_prefill_large_top_k(msa_lib, oracle_mod, B, Sq, lens, H_q, H_kv, top_k)
     print("prefill large k", (B, Sq, H_q, H_kv, top_k), rep)
 
 
-def test_prefill_large_logit_block_takes_exact_shift(msa_lib, oracle_mod):
+def _flag_count(eng):
+    """(row, head) pairs the block-outer prefill path handed to its exact
+    fp32 pass (a count the kernels keep in the workspace header)."""
+    return int(eng.ws_attn[4:8].view(torch.int32).item())
+
+
+def test_prefill_large_logit_block_takes_exact_path(msa_lib, oracle_mod):
     """A kept non-own block whose keys are 40x larger: its logits dwarf the
-    own block's, the norm bound cannot prove the own-block shift safe, and the
-    fix-up pass must supply the exact shift."""
+    own block's, so its partial outputs are far beyond the fp16 sum's range;
+    those (row, head) pairs must go through the exact fp32 pass."""
     from synthetic import make_inputs
+    from parity import compare, run_gpu, to_host
     w = make_inputs(B=1, Sq=640, lens=[640], H_q=16, H_kv=2, top_k=5, seed=33, device=DEV)
     w.k[128:256].mul_(40.0)
-    rep = _run_and_compare(oracle_mod, w)
-    print("large logits", rep)
+    m, st = run_gpu(w)
+    assert st == 0
+    assert _flag_count(m) > 0, "the exact pass was not exercised"
+    rep = compare(oracle_mod, w, *to_host(m))
+    print("large logits", rep, "flagged", _flag_count(m))
+
+
+def test_prefill_sharp_logits_take_exact_path(msa_lib, oracle_mod):
+    """Queries 6x larger in one sequence (logits with a standard deviation
+    of 6): for rows whose own block holds few keys, another kept block's
+    maximum beats the own block's by far more than the fp16 sum allows, so
+    those (row, head) pairs take the exact pass; the outputs stay O(1)."""
+    from synthetic import make_inputs
+    from parity import compare, run_gpu, to_host
+    w = make_inputs(B=2, Sq=1024, lens=[1024, 1024], H_q=16, H_kv=2, top_k=4, seed=34, device=DEV)
+    w.q[0].mul_(6.0)
+    m, st = run_gpu(w)
+    assert st == 0
+    n = _flag_count(m)
+    assert n > 0, "the exact pass was not exercised"
+    rep = compare(oracle_mod, w, *to_host(m))
+    print("sharp logits", rep, "flagged", n)
 
 
 @pytest.mark.parametrize("name", ["prefill_2k", "decode_32k", "decode_ragged", "decode_1m"])
