@@ -184,7 +184,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.kv_full[i], 1);
             mbar_init(&S.kv_empty[i], 1);
-            mbar_init(&S.q_full[i], kLoaderWarps<MODE>);
+            // pass A: one expect-tx arrival (TMA); pass B: one arrival per
+            // loader thread, made by the hardware once its copies have landed
+            mbar_init(&S.q_full[i], MODE == 0 ? 1 : kLoaderWarps<MODE> * 32);
             mbar_init(&S.q_empty[i], 1);          // released by the MMA commit
             mbar_init(&S.o_full[i], 1);
             mbar_init(&S.o_empty[i], kEpiWarps);
@@ -277,9 +279,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the bulk engine's per-copy cost (shared with the reductions), so
         // two warps gather each 2 KiB (row, group) slice with 16-byte
         // cp.async copies straight into the 128-byte-swizzled layout the MMA
-        // reads; each warp signals a tile once its copies have landed.
+        // reads; the tile's barrier completes once every copy has landed.
         const int lw = warp - 2;
-        int qt = 0, n = 0, prev_qs = -1;
+        int qt = 0, n = 0;
         bool ok = true;
         if (MODE == 0 && lane == 0) prefetch_tensormap(&tmQ16);
         Item x;
@@ -321,23 +323,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    src + ch * 16);
                     }
                 }
-                cp_async_commit();
-                if (prev_qs >= 0) {
-                    // the previous tile's copies have landed: hand it to the MMA
-                    cp_async_wait_but1();
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&S.q_full[prev_qs]);
-                }
-                prev_qs = qs;
+                // Each thread's arrival on the tile's barrier fires when its
+                // copies have landed (tracked by the hardware; a software wait,
+                // proxy fence and arrive let the MMA read stale rows).
+                cp_async_arrive_noinc(&S.q_full[qs]);
             }
         }
-        if (MODE == 1) {
-            cp_async_wait_all();                     // nothing lands after the CTA ends
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (ok && prev_qs >= 0 && lane == 0) mbar_arrive(&S.q_full[prev_qs]);
-        }
+        if (MODE == 1) cp_async_wait_all();          // nothing lands after the CTA ends
         if (!ok) *abort_flag = 1;
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------ MMA issuer
@@ -377,6 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int t0 = 0; t0 < x.n; t0 += kTileRows, ++qt) {
                 const int qs = qt & 1;
                 if (*abort_flag || !mbar_wait(&S.q_full[qs], (qt >> 1) & 1, P.status)) { ok = false; break; }
+                fence_proxy_async_smem();   // pass B's Q rows were written by cp.async
                 // One S buffer: the previous tile's S must have been read.
                 if (qt >= 1 && (*abort_flag || !mbar_wait(&S.s_empty, (qt - 1) & 1, P.status))) {
                     ok = false;
