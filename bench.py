@@ -147,6 +147,9 @@ def measure_prefill(name, dev, steps, warmup, seq_len=None):
     st = eng.device_status(stream)
     if st != 0:
         raise RuntimeError(f"prefill device status {msa.STATUS_NAMES.get(st, st)}")
+    # (row, head) pairs the block-outer path handed to its exact fp32 pass
+    # (a count the kernels keep in the attention workspace header)
+    flagged = int(eng.ws_attn[4:8].view(torch.int32).item()) if w.H_q // w.H_kv == 8 else 0
     useful = prefill_useful_flops(w, eng.block_ids.cpu().numpy())
     idx_flops = prefill_index_flops(w)
     msa.msa_trace_enable(True)
@@ -170,7 +173,8 @@ def measure_prefill(name, dev, steps, warmup, seq_len=None):
            "sparse_attn_ms": att_ms, "sparse_attn_tflops": useful / (att_ms / 1e3) / 1e12,
            "index_tflop": idx_flops / 1e12, "index_ms": idx_ms,
            "index_tflops": idx_flops / (idx_ms / 1e3) / 1e12,
-           "kernel_ms": per, "gpu_launches_per_step": len(trace) / steps}
+           "kernel_ms": per, "gpu_launches_per_step": len(trace) / steps,
+           "exact_pass_row_heads": flagged}
     del eng, w
     torch.cuda.empty_cache()
     return res

@@ -59,9 +59,13 @@ constexpr int kG = 8;                      // heads per group handled by this pa
 constexpr int kTileRows = 128 / kG;        // query rows per 128-lane tile
 constexpr int kRange = 8192;               // query rows per bucket range
 constexpr int kItemRows = 256;             // max rows per pass-B work item
-constexpr uint32_t kTmemCols = 512;        // S, P and O[2]
-// TMEM columns: S (128 fp32), P (64 columns of bf16 pairs), O[2] (2 x 128 fp32).
-constexpr uint32_t kColS = 0, kColP = 128, kColO = 256;
+constexpr uint32_t kTmemCols = 512;        // S[2], P[2] and O
+// TMEM columns: S[2] (2 x 128 fp32), P[2] (2 x 64 columns of bf16 pairs),
+// O (128 fp32).  Two S buffers let the next tile's QK run while the softmax
+// still works on this one; two P buffers let the softmax write a tile's P
+// while the previous PV still reads the other; one O buffer suffices because
+// the epilogue reads it while the next QK runs, before the next PV.
+constexpr uint32_t kColS = 0, kColP = 256, kColO = 384;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kShiftPad = 4.f;           // shift = own-block max + this (base 2)
 
@@ -131,8 +135,8 @@ struct Smem {
     uint8_t q[2][32768];                   // gathered Q tile, two swizzled halves
     uint8_t ostage[kEpiWarps][8192];       // epilogue: 4 rows x 128 dims x 8 heads fp16 per warp
     uint64_t kv_full[2], kv_empty[2], q_full[2], q_empty[2];
-    uint64_t s_full, s_empty, o_full[2], o_empty[2];
-    uint64_t p_full, p_empty;
+    uint64_t s_full[2], s_empty[2], o_full, o_empty;
+    uint64_t p_full[2], p_empty[2];
     float xmax[2][128];                    // pass A: each softmax warp's half-row max
     uint64_t xbar[4];                      // pass A: the two softmax warps of a lane quarter
     uint64_t item_full[4], item_empty[4];  // work-item queue: producer -> MMA, softmax, epilogue
@@ -188,13 +192,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             // loader thread, made by the hardware once its copies have landed
             mbar_init(&S.q_full[i], MODE == 0 ? 1 : kLoaderWarps<MODE> * 32);
             mbar_init(&S.q_empty[i], 1);          // released by the MMA commit
-            mbar_init(&S.o_full[i], 1);
-            mbar_init(&S.o_empty[i], kEpiWarps);
+            mbar_init(&S.s_full[i], 1);
+            mbar_init(&S.s_empty[i], kSoftWarps);
+            mbar_init(&S.p_full[i], kSoftWarps);
+            mbar_init(&S.p_empty[i], 1);
         }
-        mbar_init(&S.s_full, 1);
-        mbar_init(&S.s_empty, kSoftWarps);
-        mbar_init(&S.p_full, kSoftWarps);
-        mbar_init(&S.p_empty, 1);
+        mbar_init(&S.o_full, 1);
+        mbar_init(&S.o_empty, kEpiWarps);
         for (int i = 0; i < 4; ++i) mbar_init(&S.xbar[i], 64);   // every lane of both warps
         for (int i = 0; i < kQueue; ++i) {
             mbar_init(&S.item_full[i], 1);
@@ -339,21 +343,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         int pv_pending = -1, pv_kvs = 0, pv_last = 0;   // tile waiting for its PV
         bool ok = true;
         // O = P V: P (bf16) from TMEM, V from shared memory.
+        // Descriptors are built once; a K step only moves the start address
+        // field (bits 0-13, in 16-byte units), which never carries here.
+        const uint64_t kv_desc0 = umma_desc(smem_u32(S.kv[0]), 16, 1024);
+        const uint64_t kv_desc1 = umma_desc(smem_u32(S.kv[1]), 16, 1024);
+        const uint64_t v_desc0 = umma_desc(smem_u32(S.kv[0] + 32768), 16384, 1024);
+        const uint64_t v_desc1 = umma_desc(smem_u32(S.kv[1] + 32768), 16384, 1024);
+        const uint64_t q_desc0 = umma_desc(smem_u32(S.q[0]), 16, 1024);
+        const uint64_t q_desc1 = umma_desc(smem_u32(S.q[1]), 16, 1024);
         auto issue_pv = [&](int t, int kvs, int last_of_item) -> bool {
-            const int os = t & 1;
-            if (*abort_flag || !mbar_wait(&S.p_full, t & 1, P.status)) return false;
-            if (t >= 2 && (*abort_flag || !mbar_wait(&S.o_empty[os], ((t >> 1) - 1) & 1, P.status)))
+            const int pb = t & 1;
+            if (*abort_flag || !mbar_wait(&S.p_full[pb], (t >> 1) & 1, P.status)) return false;
+            // the epilogue has read the previous tile's O
+            if (t >= 1 && (*abort_flag || !mbar_wait(&S.o_empty, (t - 1) & 1, P.status)))
                 return false;
             tc_fence_after();
-            const uint32_t va = smem_u32(S.kv[kvs] + 32768);
+            const uint64_t vd = kvs ? v_desc1 : v_desc0;
+            const uint32_t d = tmem + kColO, a = tmem + kColP + pb * 64;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t bd = umma_desc(va + kk * 2048, 16384, 1024);
-                umma_bf16_ts(tmem + kColO + os * 128, tmem + kColP + kk * 8, bd, idesc_pv,
-                             kk > 0 ? 1u : 0u);
-            }
-            umma_commit(&S.o_full[os]);
-            umma_commit(&S.p_empty);
+            for (int kk = 0; kk < 8; ++kk)
+                umma_bf16_ts(d, a + kk * 8, vd + static_cast<uint64_t>(kk * 128), idesc_pv, kk > 0 ? 1u : 0u);
+            umma_commit(&S.o_full);
+            umma_commit(&S.p_empty[pb]);
             if (last_of_item) umma_commit(&S.kv_empty[kvs]);
             return true;
         };
@@ -365,25 +376,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int kvs = ki & 1;
             if (*abort_flag || !mbar_wait(&S.kv_full[kvs], (ki >> 1) & 1, P.status)) { ok = false; break; }
             ++ki;
-            const uint32_t ka = smem_u32(S.kv[kvs]);
+            const uint64_t kd = kvs ? kv_desc1 : kv_desc0;
             for (int t0 = 0; t0 < x.n; t0 += kTileRows, ++qt) {
                 const int qs = qt & 1;
                 if (*abort_flag || !mbar_wait(&S.q_full[qs], (qt >> 1) & 1, P.status)) { ok = false; break; }
                 fence_proxy_async_smem();   // pass B's Q rows were written by cp.async
-                // One S buffer: the previous tile's S must have been read.
-                if (qt >= 1 && (*abort_flag || !mbar_wait(&S.s_empty, (qt - 1) & 1, P.status))) {
+                // S[sb] is free once the softmax has read the tile two back.
+                const int sb = qt & 1;
+                if (qt >= 2 && (*abort_flag || !mbar_wait(&S.s_empty[sb], ((qt >> 1) - 1) & 1, P.status))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t qa = smem_u32(S.q[qs]);
+                const uint64_t qd = qs ? q_desc1 : q_desc0;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t ad = umma_desc(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bd = umma_desc(ka + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                    umma_bf16_ss(tmem + kColS, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                    const uint64_t off = static_cast<uint64_t>((kk >> 2) * 1024 + (kk & 3) * 2);
+                    umma_bf16_ss(tmem + kColS + sb * 128, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&S.s_full);
+                umma_commit(&S.s_full[sb]);
                 umma_commit(&S.q_empty[qs]);
                 // PV of the previous tile runs behind this tile's QK.
                 if (pv_pending >= 0 && !issue_pv(pv_pending, pv_kvs, pv_last)) { ok = false; break; }
@@ -395,8 +406,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && pv_pending >= 0 && !issue_pv(pv_pending, pv_kvs, pv_last)) ok = false;
         if (!ok) *abort_flag = 1;
         // Every MMA issued must finish before TMEM is released.
-        if (qt > 0) mbar_wait(&S.s_full, (qt - 1) & 1, nullptr);
-        if (pv_pending >= 0) mbar_wait(&S.o_full[pv_pending & 1], (pv_pending >> 1) & 1, nullptr);
+        if (qt > 0) mbar_wait(&S.s_full[(qt - 1) & 1], ((qt - 1) >> 1) & 1, nullptr);
+        if (pv_pending >= 0) mbar_wait(&S.o_full, pv_pending & 1, nullptr);
     } else if (warp >= 4 && warp < kEpiWarp0) {
         // ------------------------------------------------ softmax
         // Warps 4-7 and 8-11 share the TMEM lanes of warp % 4 and split each
@@ -458,11 +469,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!fetch(xn)) { ok = false; break; }
                     if (xn.n > 0) load_tile(xn, 0, row_nx, shift_nx);
                 }
-                bool have = !*abort_flag && mbar_wait(&S.s_full, qt & 1, P.status);
+                const int sb = qt & 1;
+                bool have = !*abort_flag && mbar_wait(&S.s_full[sb], (qt >> 1) & 1, P.status);
                 have = __all_sync(0xffffffffu, have);
                 if (!have) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t sa = lane_addr + kColS;
+                const uint32_t sa = lane_addr + kColS + sb * 128;
                 int lim = 127;                         // last visible column of the row
                 uint32_t a[32], b[32];
                 tmem_ld32r(sa + ch * 64, a);
@@ -498,27 +510,42 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // S is in registers: the next tile's QK may overwrite it.
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&S.s_empty);
+                if (lane == 0) mbar_arrive(&S.s_empty[sb]);
                 float l = 0.f;
                 uint32_t pk[32];                        // 64 probabilities as bf16 pairs
+                if (MODE == 1) {
+                    // every column is visible; a padding lane gets 2^-inf = 0
+                    const float sh = valid ? shift : INFINITY;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int c0 = ch * 64 + 2 * e;
-                    const uint32_t *src = e < 16 ? a : b;
-                    const int k = (2 * e) & 31;
-                    float p0 = fast_exp2(__uint_as_float(src[k]) * sl2 - shift);
-                    float p1 = fast_exp2(__uint_as_float(src[k + 1]) * sl2 - shift);
-                    p0 = (valid && c0 <= lim) ? p0 : 0.f;
-                    p1 = (valid && c0 + 1 <= lim) ? p1 : 0.f;
-                    l += p0 + p1;
-                    pk[e] = pack_bf16x2(p0, p1);
+                    for (int e = 0; e < 32; ++e) {
+                        const uint32_t *src = e < 16 ? a : b;
+                        const int k = (2 * e) & 31;
+                        const float p0 = fast_exp2(fmaf(__uint_as_float(src[k]), sl2, -sh));
+                        const float p1 = fast_exp2(fmaf(__uint_as_float(src[k + 1]), sl2, -sh));
+                        l += p0 + p1;
+                        pk[e] = pack_bf16x2(p0, p1);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int c0 = ch * 64 + 2 * e;
+                        const uint32_t *src = e < 16 ? a : b;
+                        const int k = (2 * e) & 31;
+                        float p0 = fast_exp2(__uint_as_float(src[k]) * sl2 - shift);
+                        float p1 = fast_exp2(__uint_as_float(src[k + 1]) * sl2 - shift);
+                        p0 = (valid && c0 <= lim) ? p0 : 0.f;
+                        p1 = (valid && c0 + 1 <= lim) ? p1 : 0.f;
+                        l += p0 + p1;
+                        pk[e] = pack_bf16x2(p0, p1);
+                    }
                 }
-                // P's columns are free once the previous tile's PV has read them.
-                bool pfree = !*abort_flag && (qt == 0 || mbar_wait(&S.p_empty, (qt - 1) & 1, P.status));
+                // P[pb]'s columns are free once the PV two tiles back has read them.
+                const int pb = qt & 1;
+                bool pfree = !*abort_flag && (qt < 2 || mbar_wait(&S.p_empty[pb], ((qt >> 1) - 1) & 1, P.status));
                 pfree = __all_sync(0xffffffffu, pfree);
                 if (!pfree) { ok = false; break; }
                 tc_fence_after();
-                tmem_st32(lane_addr + kColP + ch * 32, pk);
+                tmem_st32(lane_addr + kColP + pb * 64 + ch * 32, pk);
                 if (zero_v) {
                     bool kok = !*abort_flag && mbar_wait(&S.kv_full[kvs], kv_par, P.status);
                     kok = __all_sync(0xffffffffu, kok);
@@ -536,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&S.p_full);
+                if (lane == 0) mbar_arrive(&S.p_full[pb]);
                 if (valid) atomicAdd(P.l_acc + row * P.H_q + x.g * kG + h, l);
                 if (MODE == 0 && ch == 0 && valid) P.m_arr[row * P.H_q + x.g * kG + h] = shift;
             }
@@ -581,7 +608,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             Item xn;
             xn.n = -1;
             for (int t0 = 0; t0 < x.n; t0 += kTileRows, ++qt) {
-                const int os = qt & 1;
                 const long long row = row_nx;
                 const bool valid = row >= 0;
                 if (t0 + kTileRows < x.n) {
@@ -596,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const long long rr = __shfl_sync(0xffffffffu, row, r4 * 8);
                     dst4[r4] = rr >= 0 ? P.o_acc + (rr * P.H_kv + x.g) * (kDim * kG) : nullptr;
                 }
-                bool have = !*abort_flag && mbar_wait(&S.o_full[os], (qt >> 1) & 1, P.status);
+                bool have = !*abort_flag && mbar_wait(&S.o_full, qt & 1, P.status);
                 have = __all_sync(0xffffffffu, have);
                 if (!have) { ok = false; break; }
                 tc_fence_after();
@@ -607,14 +633,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t a[32], b[32];
-                    tmem_ld32r(lane_addr + kColO + os * 128 + half * 64, a);
-                    tmem_ld32r(lane_addr + kColO + os * 128 + half * 64 + 32, b);
+                    tmem_ld32r(lane_addr + kColO + half * 64, a);
+                    tmem_ld32r(lane_addr + kColO + half * 64 + 32, b);
                     tmem_wait_ld(a);
                     tmem_tie(b);
                     if (half == 1) {
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&S.o_empty[os]);
+                        if (lane == 0) mbar_arrive(&S.o_empty);
                     }
                     if (valid) {
 #pragma unroll
@@ -677,9 +703,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 // scattered.  No grid-wide scan: each range owns fixed slices of the arrays.
 constexpr int kBuildThreads = 512;
 
+// Counters and cursors live in shared memory when nb_max <= this (64 KiB),
+// else in the workspace.
+constexpr int kBuildSmemBlocks = 8192;
+
 __global__ void __launch_bounds__(kBuildThreads) bucket_build_kernel(const PrefillArgs P) {
     __shared__ int warp_c[kBuildThreads / 32], warp_i[kBuildThreads / 32];
     __shared__ int carry_c, carry_i;
+    extern __shared__ int build_smem[];             // [2][nb_max] when it fits
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const long long r = blockIdx.x;
     const int rng = static_cast<int>(r % P.n_ranges);
@@ -692,8 +723,13 @@ __global__ void __launch_bounds__(kBuildThreads) bucket_build_kernel(const Prefi
     }
     const int i0 = rng * kRange, i1 = min(P.Sq, i0 + kRange);
     const long long n_e = static_cast<long long>(i1 - i0) * P.K;
-    int *cnt = P.bucket_cnt + r * P.nb_max;
-    int *cur = P.bucket_cur + r * P.nb_max;
+    const bool in_smem = P.nb_max <= kBuildSmemBlocks;
+    int *cnt = in_smem ? build_smem : P.bucket_cnt + r * P.nb_max;
+    int *cur = in_smem ? build_smem + P.nb_max : P.bucket_cur + r * P.nb_max;
+    if (in_smem) {
+        for (int j = tid; j < 2 * P.nb_max; j += kBuildThreads) build_smem[j] = 0;
+        __syncthreads();
+    }
     const int32_t *ids = P.ids;
     auto entry = [&](long long e, long long &row) -> int {
         const int i = i0 + static_cast<int>(e / P.K);
@@ -729,6 +765,7 @@ __global__ void __launch_bounds__(kBuildThreads) bucket_build_kernel(const Prefi
         const int ex_c = pc + ic - c, ex_i = pi + ii - ni;
         if (j < P.nb_max) {
             const long long bk = r * P.nb_max + j;
+            if (in_smem) P.bucket_cnt[bk] = c;       // read by item_table_kernel
             P.bucket_off[bk] = static_cast<int>(region + ex_c);
             P.item_off[bk] = ex_i;
             for (int q = 0; q < ni; ++q) P.item_bucket[r * P.items_per_range + ex_i + q] = j;
@@ -738,6 +775,7 @@ __global__ void __launch_bounds__(kBuildThreads) bucket_build_kernel(const Prefi
         __syncthreads();
     }
     if (tid == 0) P.range_count[r] = carry_i;
+    __syncthreads();
     __syncthreads();
     for (long long e = tid; e < n_e; e += kBuildThreads) {
         long long row;
@@ -818,36 +856,58 @@ __global__ void bucket_shift_kernel(const PrefillArgs P) {
     }
 }
 
-// out = accumulator / sum, bf16.  One warp per (row, group): lane = (head,
-// 32 dims = four 16-byte chunks of the fp16 accumulator).
-__global__ void finalize_kernel(const PrefillArgs P) {
-    const int lane = threadIdx.x & 31;
-    const int h = lane >> 2, qd = lane & 3;
-    const long long total = static_cast<long long>(P.B) * P.Sq * P.H_kv;
-    for (long long pair = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-         pair < total; pair += (static_cast<long long>(gridDim.x) * blockDim.x) >> 5) {
-        const long long row = pair / P.H_kv;
-        const int g = static_cast<int>(pair % P.H_kv);
-        const int b = static_cast<int>(row / P.Sq);
-        int L;
-        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(P.out) + (row * P.H_q + g * kG + h) * kDim + qd * 32;
-        if (!seq_ok(P, b, L)) {
-            for (int d = 0; d < 32; ++d) out[d] = __float2bfloat16(NAN);
-            continue;
+// out = accumulator / sum, bf16.  A thread takes 16-byte chunks of the fp16
+// accumulator (8 dims of one head) in order, four at a time, so every warp
+// reads 2 KiB contiguous and the loads of four chunks are in flight at once.
+__global__ void __launch_bounds__(256) finalize_kernel(const PrefillArgs P) {
+    const long long pairs = static_cast<long long>(P.B) * P.Sq * P.H_kv;
+    const long long chunks = pairs * (kDim * kG / 8);        // 128 chunks per (row, group)
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    const uint4 *acc = reinterpret_cast<const uint4 *>(P.o_acc);
+    __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(P.out);
+    for (long long c0 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; c0 < chunks;
+         c0 += 4 * stride) {
+        uint4 v[4];
+        float l[4];
+        bool ok[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const long long c = c0 + u * stride;
+            ok[u] = c < chunks;
+            if (!ok[u]) continue;
+            const long long pair = c >> 7;
+            const int q = static_cast<int>(c & 127), h = q & 7;
+            const long long row = pair / P.H_kv;
+            const int g = static_cast<int>(pair % P.H_kv);
+            v[u] = acc[c];
+            l[u] = P.l_acc[row * P.H_q + g * kG + h];
         }
-        const float inv = 1.f / P.l_acc[row * P.H_q + g * kG + h];
-        const uint4 *acc = reinterpret_cast<const uint4 *>(P.o_acc + pair * (kDim * kG));
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const uint4 v = acc[(qd * 4 + c) * kG + h];      // dims 8(4qd+c) .. +7 of head h
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-            uint32_t o4[4];
+        for (int u = 0; u < 4; ++u) {
+            if (!ok[u]) continue;
+            const long long c = c0 + u * stride;
+            const long long pair = c >> 7;
+            const int q = static_cast<int>(c & 127), h = q & 7, cd = q >> 3;
+            const long long row = pair / P.H_kv;
+            const int g = static_cast<int>(pair % P.H_kv);
+            const int b = static_cast<int>(row / P.Sq);
+            int L;
+            uint4 o;
+            if (!seq_ok(P, b, L)) {
+                const uint32_t nan2 = pack_bf16x2(NAN, NAN);
+                o = make_uint4(nan2, nan2, nan2, nan2);
+            } else {
+                const float inv = 1.f / l[u];
+                const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                uint32_t o4[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w4[e]));
-                o4[e] = pack_bf16x2(f.x * inv, f.y * inv);
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w4[e]));
+                    o4[e] = pack_bf16x2(f.x * inv, f.y * inv);
+                }
+                o = make_uint4(o4[0], o4[1], o4[2], o4[3]);
             }
-            *reinterpret_cast<uint4 *>(out + c * 8) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+            *reinterpret_cast<uint4 *>(out + (row * P.H_q + g * kG + h) * kDim + cd * 8) = o;
         }
     }
 }
@@ -1006,7 +1066,12 @@ cudaError_t launch_prefill_attention(const PrefillArgs &a0, uint8_t *ws, const P
     const int sms = device_sm_count();
     {
         TraceScope t(s, "prefill_bucket");
-        bucket_build_kernel<<<static_cast<unsigned>(L.n_ranges_total), kBuildThreads, 0, s>>>(a);
+        const size_t bsm = L.nb_max <= kBuildSmemBlocks ? static_cast<size_t>(2 * L.nb_max) * sizeof(int) : 0;
+        if (bsm > 48 * 1024 &&
+            (e = cudaFuncSetAttribute(bucket_build_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(bsm))) != cudaSuccess)
+            return e;
+        bucket_build_kernel<<<static_cast<unsigned>(L.n_ranges_total), kBuildThreads, bsm, s>>>(a);
         range_scan_kernel<<<1, 1024, 0, s>>>(a);
         item_table_kernel<<<static_cast<unsigned>(L.n_ranges_total), 256, 0, s>>>(a);
     }
@@ -1019,7 +1084,7 @@ cudaError_t launch_prefill_attention(const PrefillArgs &a0, uint8_t *ws, const P
     if ((e = launch_pass<1>(tq, tk, tv, a, s, "prefill_attn_kv_outer")) != cudaSuccess) return e;
     {
         TraceScope t(s, "prefill_finalize");
-        finalize_kernel<<<sms * 8, 256, 0, s>>>(a);
+        finalize_kernel<<<sms * 16, 256, 0, s>>>(a);
     }
     {
         TraceScope t(s, "prefill_exact_rows");
