@@ -304,7 +304,24 @@ def measure_index_variants(w, dev, steps, warmup):
         key_bytes = ntok * kh * w.d_idx * keys.element_size() + (ntok * kh * 4 if scale is not None else 0)
         idx_bytes = key_bytes + w.B * Hi * w.d_idx * 2 + nb * Hi * 4
         gbs = idx_bytes / (per[idx_name] / 1e3) / 1e9
+        fused_ms = None
+        if fmt == msa.INDEX_KEYS_BF16:
+            # the same step as one launch (msa_decode_step takes bf16 keys, one row per index head)
+            for _ in range(warmup):
+                eng.decode_step(q_idx, keys, w.q, w.k, w.v, w.lens, w.kv_offsets, stream)
+            torch.cuda.synchronize()
+            st = msa.msa_read_device_status(eng.ws_step, stream)
+            if st != 0:
+                raise RuntimeError(f"{name} fused: device status {msa.STATUS_NAMES.get(st, st)}")
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(steps):
+                eng.decode_step(q_idx, keys, w.q, w.k, w.v, w.lens, w.kv_offsets, stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            fused_ms = e0.elapsed_time(e1) / steps
         out[name] = {"index_heads": Hi, "key_rows_per_token": kh,
+                     "fused_step_ms": fused_ms,
                      "key_dtype": "e4m3" if scale is not None else "bf16",
                      "ms_per_step": ev0.elapsed_time(ev1) / steps, "kernel_ms": per,
                      "index_bytes": idx_bytes, "index_gbs": gbs, "index_frac_of_hbm": gbs / peak,

@@ -115,7 +115,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     Smem &S = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int H = P.H_kv, G = P.H_q / P.H_kv, K = P.K;
+    // H groups (attention items); HI index heads (scores, top-k), group g
+    // reading index head g / (H / HI)
+    const int H = P.H_kv, HI = P.n_idx, G = P.H_q / P.H_kv, K = P.K;
     const int nbs = score_stride(P.nb_max);
     volatile int *abort_flag = &S.abort_flag;
 
@@ -151,9 +153,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else if (blockIdx.x == 0) {
                 // rejected sequence: -1 / -inf selection, NaN output, status word
                 set_status(P.status, kStatusBadLens);
-                for (int q = 0; q < H * K; ++q) {
-                    P.ids[static_cast<long long>(b) * H * K + q] = -1;
-                    P.out_scores[static_cast<long long>(b) * H * K + q] = -INFINITY;
+                for (int q = 0; q < HI * K; ++q) {
+                    P.ids[static_cast<long long>(b) * HI * K + q] = -1;
+                    P.out_scores[static_cast<long long>(b) * HI * K + q] = -INFINITY;
                 }
                 __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(P.out) + static_cast<long long>(b) * P.H_q * kDim;
                 for (int e = 0; e < P.H_q * kDim; ++e) o[e] = __float2bfloat16(NAN);
@@ -195,15 +197,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!have) { *abort_flag = 1; break; }
             const int b = S.red_b[slot], j = S.red_j[slot];
             float m = -INFINITY;
-            if (lane < H)
-                for (int r = lane; r < 16; r += H) m = fmaxf(m, S.red[slot][r]);
+            if (lane < HI)
+                for (int r = lane; r < 16; r += HI) m = fmaxf(m, S.red[slot][r]);
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.red_empty[slot]);
             if (b < 0) break;                       // the consumers are done
             bool last = false;
-            if (lane < H) {
-                P.scores[((long long)b * H + lane) * nbs + j] = m;
-                const int target = H * ((P.lens[b] + kBlock - 1) / kBlock);
+            if (lane < HI) {
+                P.scores[((long long)b * HI + lane) * nbs + j] = m;
+                const int target = HI * ((P.lens[b] + kBlock - 1) / kBlock);
                 last = atom_add_acq_rel_gpu(P.seq_done + b, 1) + 1 == target;
             }
             if (__any_sync(0xffffffffu, last) && lane == 0) {
@@ -235,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tensormap(&tmV);
         const uint64_t pol = l2_policy_evict_first();
         const __nv_bfloat16 *kbase = static_cast<const __nv_bfloat16 *>(P.k_idx);
-        const int tps = 128 / H;                 // tokens per index stage
+        const int tps = 128 / HI;                // tokens per index stage
         int n = 0, it = 0;                        // work entries pushed, stages issued
         bool index_left = true, ok = true;
         auto push = [&](int4 w) -> bool {
@@ -321,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int n_kept = min(K, nb);
                 if (!push(make_int4(kWorkAttn, bg, n_kept, 0))) { ok = false; break; }
                 // K and V tiles of every kept block, the next id loaded ahead
-                const int32_t *idrow = P.ids + static_cast<long long>(bg) * K;
+                const int32_t *idrow = P.ids + (static_cast<long long>(b) * HI + g / (H / HI)) * K;
                 int jn = __ldcg(idrow);
                 for (int sl = 0; sl < n_kept && ok; ++sl) {
                     const int j = jn;
@@ -357,9 +359,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int t0s = 0; t0s < ntok; t0s += tps) {
                     int slot;
                     if (!stage(slot)) { ok = false; break; }
-                    const uint32_t bytes = static_cast<uint32_t>(min(tps, ntok - t0s)) * H * kDim * 2;
+                    const uint32_t bytes = static_cast<uint32_t>(min(tps, ntok - t0s)) * HI * kDim * 2;
                     mbar_arrive_expect_tx(&S.full[slot], bytes);
-                    bulk_g2s(S.ring[slot], kbase + (t_first + t0s) * H * kDim, bytes, &S.full[slot], pol);
+                    bulk_g2s(S.ring[slot], kbase + (t_first + t0s) * HI * kDim, bytes, &S.full[slot], pol);
                 }
                 t_idle = now_ns();
                 continue;
@@ -400,10 +402,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++cb;
     };
     const int c16 = tid & 15, r16 = tid >> 4;     // index rows: 16-byte chunk, row slot 0..15
-    const int gi = r16 % H;                        // group of this thread's index rows
+    const int gi = r16 % HI;                       // index head of this thread's index rows
     const int gq = lane >> 2, tq = lane & 3;
     const int r0 = warp * 16;                      // attention: this warp's 16 tokens
-    const int tps = 128 / H;
+    const int tps = 128 / HI;
     const float sl2 = P.softmax_scale * kLog2e;
     const __nv_bfloat16 *qibase = static_cast<const __nv_bfloat16 *>(P.q_idx);
     float qf[8];
@@ -430,8 +432,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int own = nb - 1;                    // decode: the query is token L-1
         unsigned long long *keys = reinterpret_cast<unsigned long long *>(&S.om[warp][0][0]);
         int *sel = reinterpret_cast<int *>(&S.om[warp][2][0]);
-        for (int g = warp; g < H; g += kWarps) {
-            const long long bg = static_cast<long long>(b) * H + g;
+        for (int g = warp; g < HI; g += kWarps) {   // index heads
+            const long long bg = static_cast<long long>(b) * HI + g;
             const float *sc = P.scores + bg * nbs;
             int n = 0;
             if (nb <= K) {
@@ -497,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // ---- index unit: block j of sequence b, every group
             const int b = w.y, j = w.z, ntok = w.w;
             if (b != cur_b) {
-                const uint4 qv = *reinterpret_cast<const uint4 *>(qibase + ((long long)b * H + gi) * kDim + c16 * 8);
+                const uint4 qv = *reinterpret_cast<const uint4 *>(qibase + ((long long)b * HI + gi) * kDim + c16 * 8);
                 qf[0] = bf16lo(qv.x); qf[1] = bf16hi(qv.x);
                 qf[2] = bf16lo(qv.y); qf[3] = bf16hi(qv.y);
                 qf[4] = bf16lo(qv.z); qf[5] = bf16hi(qv.z);
@@ -506,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             float runmax = -INFINITY;
             for (int t0 = 0; t0 < ntok; t0 += tps) {
-                const int rows_valid = min(tps, ntok - t0) * H;
+                const int rows_valid = min(tps, ntok - t0) * HI;
                 int slot;
                 if (wait_stage(slot)) {
                     const uint8_t *sb = S.ring[slot];
@@ -664,7 +666,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-size_t decode_fused_layout(int B, int H_q, int H_kv, int K, int max_kv_len, DecodeFusedLayout *L) {
+size_t decode_fused_layout(int B, int H_q, int H_kv, int n_idx, int K, int max_kv_len,
+                           DecodeFusedLayout *L) {
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
     const size_t nb_max = score_stride((max_kv_len + kBlock - 1) / kBlock);
     const size_t items = static_cast<size_t>(B) * H_kv;
@@ -676,7 +679,7 @@ size_t decode_fused_layout(int B, int H_q, int H_kv, int K, int max_kv_len, Deco
     L->seq_done = o; o += up(static_cast<size_t>(B) * 4);
     L->aq_flag = o;  o += up(items * 4);
     L->zero_hi = o;
-    L->scores = o;   o += up(static_cast<size_t>(B) * H_kv * nb_max * 4);
+    L->scores = o;   o += up(static_cast<size_t>(B) * n_idx * nb_max * 4);
     L->aq_item = o;  o += up(items * 4);
     L->total = o;
     (void)H_q;

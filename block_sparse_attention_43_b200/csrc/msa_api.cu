@@ -483,20 +483,22 @@ msa_status_t msa_sparse_attention_backward(const msa_shape_t *shape, const void 
     return launch_attn_bwd(a, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
 }
 
-// The fused decode step takes one bf16 index key per group, q_len 1 and
-// groups of at most 8 heads (one n8 tile of the attention products).
+// The fused decode step takes bf16 index keys, one row per index head (any
+// index-head count the shape allows), q_len 1 and groups of at most 8 heads
+// (one n8 tile of the attention products).
 static msa_status_t check_decode_step(const msa_shape_t *s) {
     msa_status_t st = check_shape(s);
     if (st != MSA_OK) return st;
-    if (s->q_len != 1 || index_heads(s) != s->num_kv_heads ||
-        s->index_key_format != MSA_INDEX_KEYS_BF16 || s->num_q_heads / s->num_kv_heads > 8)
+    if (s->q_len != 1 || s->index_key_format != MSA_INDEX_KEYS_BF16 ||
+        s->num_q_heads / s->num_kv_heads > 8)
         return MSA_ERR_UNSUPPORTED;
     return MSA_OK;
 }
 
 static DecodeFusedLayout decode_step_layout(const msa_shape_t *s) {
     DecodeFusedLayout L;
-    decode_fused_layout(s->batch, s->num_q_heads, s->num_kv_heads, s->top_k, s->max_kv_len, &L);
+    decode_fused_layout(s->batch, s->num_q_heads, s->num_kv_heads, index_heads(s), s->top_k,
+                        s->max_kv_len, &L);
     return L;
 }
 
@@ -538,6 +540,7 @@ static msa_status_t decode_step_impl(const msa_shape_t *shape, const void *q_idx
     a.aq_flag = reinterpret_cast<int *>(ws + L.aq_flag);
     a.B = shape->batch; a.H_q = shape->num_q_heads; a.H_kv = shape->num_kv_heads;
     a.K = shape->top_k; a.nb_max = nb_max_of(shape); a.max_kv_len = shape->max_kv_len;
+    a.n_idx = index_heads(shape);
     a.softmax_scale = softmax_scale;
     return launch_decode_fused(a, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
 }

@@ -172,31 +172,33 @@ bool encode_q_rows_map(CUtensorMap *map, const void *q, int H_q, long long rows,
 // scores, top-k per (sequence, index head) and sparse attention.
 constexpr int kCtrStride = 32;
 struct DecodeFusedArgs {
-    const void *q_idx;      // [B][H_kv][128]
-    const void *k_idx;      // [T][H_kv][128]
+    const void *q_idx;      // [B][n_idx][128]
+    const void *k_idx;      // [T][n_idx][128]
     const void *q;          // [B][H_q][128]
     const void *k_cache;
     const void *v_cache;
     const int32_t *lens;
     KvMap kv;
-    int32_t *ids;           // [B][H_kv][K]
-    float *out_scores;      // [B][H_kv][K]
+    int32_t *ids;           // [B][n_idx][K]
+    float *out_scores;      // [B][n_idx][K]
     void *out;              // [B][H_q][128]
     int *status;
     // workspace views
-    float *scores;          // [B][H_kv][nb_max] block scores
+    float *scores;          // [B][n_idx][nb_max] block scores
     int *seq_done;          // [B] index units finished
     int *aq_item;           // [B*H_kv] published attention items (b*H_kv + g)
     int *aq_flag;           // [B*H_kv] 1 once the item above is published
     int *ctr;               // one 128-byte line each (stride kCtrStride ints): next index unit,
                             // allocated items, next item claimed, items published
     int B, H_q, H_kv, K, nb_max, max_kv_len;
+    int n_idx;              // index heads; group g reads the selection of g / (H_kv / n_idx)
     float softmax_scale;
 };
 struct DecodeFusedLayout {
     size_t scores, ctr, seq_done, aq_item, aq_flag, zero_lo, zero_hi, total;
 };
-size_t decode_fused_layout(int B, int H_q, int H_kv, int K, int max_kv_len, DecodeFusedLayout *L);
+size_t decode_fused_layout(int B, int H_q, int H_kv, int n_idx, int K, int max_kv_len,
+                           DecodeFusedLayout *L);
 cudaError_t launch_decode_fused(const DecodeFusedArgs &a, cudaStream_t s);
 
 // Backward of the sparse branch (attn_bwd.cu): one CTA per (row, group).

@@ -211,9 +211,12 @@ MSA_API msa_status_t msa_sparse_attention_backward(const msa_shape_t *shape, con
  * sequence starts as soon as its own index scores are done, overlapping the
  * index streaming of the later sequences (MSA's decode cost is that
  * streaming: "百万token上下文提速近10倍..." section 四).
- * Requirements on top of the shape rules: q_len == 1, one bf16 index key per
- * group (num_index_heads == num_kv_heads or 0, index_key_format BF16), and
- * num_q_heads / num_kv_heads <= 8; otherwise MSA_ERR_UNSUPPORTED.  The
+ * Requirements on top of the shape rules: q_len == 1, bf16 index keys with
+ * one row per index head (index_key_format BF16; any num_index_heads the
+ * shape allows, group g using the selection of index head
+ * g / (num_kv_heads / num_index_heads)), and num_q_heads / num_kv_heads <= 8;
+ * otherwise MSA_ERR_UNSUPPORTED (shared and E4M3 index keys go through
+ * msa_index_topk / msa_index_topk_fp8 and msa_sparse_attention).  The
  * launch is cooperative (one CTA per SM, all resident); it is not meant to
  * share the GPU with another kernel running at the same time.
  *   q_idx, k_idx, lens, kv_offsets, block_ids, block_scores: as msa_index_topk

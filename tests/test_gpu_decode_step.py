@@ -122,3 +122,44 @@ def test_decode_step_bad_lengths(oracle_mod):
     compare(oracle_mod, w, ids.numpy(), eng.block_scores.cpu().numpy(),
             eng.out.float().cpu().numpy(), rows=[0, 2])
 
+
+
+# (B, lens, H_q, H_kv, Hi, top_k): fewer index heads than groups (bf16 keys,
+# one row per index head); group g uses index head g / (H_kv / Hi).
+FEWER_INDEX_HEADS = [
+    (2, [4096, 300], 64, 8, 4, 16),         # the guide's 4 index heads for 8 groups
+    (4, [700, 2047, 129, 3000], 16, 8, 2, 8),
+    (3, [9000, 1, 20000], 16, 4, 1, 16),
+]
+
+
+@pytest.mark.parametrize("B,lens,H_q,H_kv,Hi,top_k", FEWER_INDEX_HEADS)
+def test_decode_step_fewer_index_heads(oracle_mod, B, lens, H_q, H_kv, Hi, top_k):
+    """The fused step with Hi < H_kv index heads: ids and scores bit-identical
+    to msa_index_topk with the same heads, outputs against the oracle run on
+    that selection."""
+    from parity import compare
+    from synthetic import bf16_bits, make_inputs
+    w = make_inputs(B=B, Sq=1, lens=lens, H_q=H_q, H_kv=H_kv, top_k=top_k, seed=61 + Hi,
+                    device=DEV)
+    q_idx = w.q_idx[:, :, :Hi].contiguous()
+    keys = w.k_idx[:, :Hi].contiguous()
+    kw = dict(batch=B, q_len=1, max_kv_len=max(lens), num_q_heads=H_q, num_kv_heads=H_kv,
+              top_k=top_k, kv_capacity=w.kv_capacity, device=DEV, num_index_heads=Hi)
+    fused = m.MSA(**kw)
+    fused.decode_step(q_idx, keys, w.q, w.k, w.v, w.lens, w.kv_offsets)
+    two = m.MSA(**kw)
+    two.index_topk(q_idx, keys, w.lens, w.kv_offsets)
+    two.sparse_attention(w.q, w.k, w.v, w.lens, w.kv_offsets)
+    torch.cuda.synchronize()
+    assert m.msa_read_device_status(fused.ws_step) == 0
+    assert two.device_status() == 0
+    ids, sc = fused.block_ids.cpu().numpy(), fused.block_scores.cpu().numpy()
+    assert ids.shape[2] == Hi
+    np.testing.assert_array_equal(ids, two.block_ids.cpu().numpy())
+    np.testing.assert_array_equal(sc, two.block_scores.cpu().numpy())
+    host = dict(q_idx=bf16_bits(q_idx), k_idx=bf16_bits(keys), q=bf16_bits(w.q),
+                k=bf16_bits(w.k), v=bf16_bits(w.v), lens=w.lens.cpu().numpy(),
+                kv_offsets=w.kv_offsets.cpu().numpy())
+    rep = compare(oracle_mod, w, ids, sc, fused.out.float().cpu().numpy(), host=host)
+    print("fused fewer index heads", (B, H_q, H_kv, Hi, top_k), rep)
