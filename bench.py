@@ -180,15 +180,22 @@ def measure_prefill(name, dev, steps, warmup, seq_len=None):
     return res
 
 
-def measure_backward(name, dev, steps, warmup):
-    """Times msa_sparse_attention_backward on a prefill workload's own
-    selection.  Useful FLOPs: 10*D per (row, head, visible kept key) -- the
-    five products S = QK^T, dP = dO V^T, dV += P^T dO, dK += dZ^T Q,
-    dQ += dZ K; reduction bytes: the fp32 dK and dV rows every (row, group,
-    kept block) adds (valid tokens x 128 dims x 4 B x 2)."""
+def measure_backward(name, dev, steps, warmup, seq_len=None):
+    """Times one msa_sparse_attention_backward call (the forward recomputed
+    for the log-sum-exp, Delta, buckets, the block-outer kernel and the dQ
+    conversion) on a prefill workload's own selection, with CUDA events on
+    its stream; per-kernel times come from the library's trace.  Useful
+    FLOPs: 10*D per (row, head, visible kept key) -- the five products
+    S = QK^T, dP = dO V^T, dV += P^T dO, dK += dS^T Q, dQ += dS K."""
     import block_sparse_attention_43_b200 as msa
-    from synthetic import make_workload
-    w = make_workload(name, dev)
+    from synthetic import WORKLOADS, make_inputs, make_workload
+    if seq_len is None:
+        w = make_workload(name, dev)
+    else:
+        c = WORKLOADS[name]
+        w = make_inputs(B=c["B"], Sq=seq_len, lens=[seq_len] * c["B"], H_q=c["H_q"],
+                        H_kv=c["H_kv"], top_k=c["top_k"], seed=c["seed"], device=dev,
+                        name=f"{name}@{seq_len}")
     eng = msa.MSA(batch=w.B, q_len=w.Sq, max_kv_len=max(w.lens_host), num_q_heads=w.H_q,
                   num_kv_heads=w.H_kv, top_k=w.top_k, kv_capacity=w.kv_capacity, device=dev)
     stream = torch.cuda.Stream(device=dev)
@@ -213,23 +220,35 @@ def measure_backward(name, dev, steps, warmup):
     ids = eng.block_ids.cpu().numpy()
     fwd_useful = prefill_useful_flops(w, ids)             # 4*D per (row, head, key)
     useful = fwd_useful * 10 // 4
-    keys_per_group = fwd_useful // (4 * w.D * (w.H_q // w.H_kv))
-    red_bytes = keys_per_group * w.D * 4 * 2
+    kept = int((ids >= 0).sum()) * (w.H_q // w.H_kv)      # (row, head, kept block)
     msa.msa_trace_enable(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
     for _ in range(steps):
         step()
+    ev1.record(stream)
     torch.cuda.synchronize()
     trace = msa.msa_trace_read()
     msa.msa_trace_enable(False)
-    ms = float(np.mean([t for n, t in trace if n == "sparse_attention_backward"]))
+    ms = ev0.elapsed_time(ev1) / steps
+    per = {}
+    for n, t in trace:
+        per[n] = per.get(n, 0.0) + t / steps
+    blocks_ms = per.get("backward_blocks", float("nan"))
     _, tf_burst, _, kind = measured_peaks()
+    tflops = useful / (ms / 1e3) / 1e12
     res = {"workload": w.name, "rows": w.B * w.Sq, "H_q": w.H_q, "H_kv": w.H_kv, "top_k": w.top_k,
-           "ms": ms, "useful_tflop": useful / 1e12, "tflops": useful / (ms / 1e3) / 1e12,
-           "frac_of_bf16_burst": useful / (ms / 1e3) / 1e12 / tf_burst,
-           "dk_dv_reduction_bytes": red_bytes, "reduction_gbs": red_bytes / (ms / 1e3) / 1e9,
-           "bound": "fp32 dK/dV reductions (one 128-row block per row and kept block)",
+           "ms": ms, "useful_tflop": useful / 1e12, "tflops": tflops,
+           "frac_of_bf16_burst": tflops / tf_burst,
+           "kernels_ms": {k: round(v, 4) for k, v in sorted(per.items())},
+           "blocks_kernel": {"ms": blocks_ms,
+                             "tflops": useful / (blocks_ms / 1e3) / 1e12,
+                             "frac_of_bf16_burst": useful / (blocks_ms / 1e3) / 1e12 / tf_burst},
+           "dq_reduction_bytes": kept * w.D * 4,
+           "note": "ms covers the whole call, the forward recompute included; useful FLOPs "
+                   "count the backward's five products only",
            "peak_kind": kind}
-    del eng, w
+    del eng, w, ws
     torch.cuda.empty_cache()
     return res
 
@@ -811,6 +830,7 @@ def main():
     backward = None
     if not args.no_backward and world == 1:
         backward = measure_backward("prefill_2k", dev, 20, 3)
+        backward["at_32k_rows"] = measure_backward("prefill_128k", dev, 5, 2, seq_len=32768)
 
     prefill = None
     configs = None

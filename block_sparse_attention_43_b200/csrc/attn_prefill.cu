@@ -699,7 +699,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------- helpers
 // Buckets of one (sequence, group, row range), built by one CTA: rows that
 // kept block j (j != own) are counted, given offsets in the range's own
-// region of bucket_rows, split into work items of <= kItemRows rows, and
+// region of bucket_rows, split into work items of <= item_rows rows, and
 // scattered.  No grid-wide scan: each range owns fixed slices of the arrays.
 constexpr int kBuildThreads = 512;
 
@@ -751,7 +751,7 @@ __global__ void __launch_bounds__(kBuildThreads) bucket_build_kernel(const Prefi
     for (int base = 0; base < P.nb_max; base += kBuildThreads) {
         const int j = base + tid;
         const int c = j < P.nb_max ? cnt[j] : 0;
-        const int ni = (c + kItemRows - 1) / kItemRows;
+        const int ni = (c + P.item_rows - 1) / P.item_rows;
         int ic = c, ii = ni;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -832,8 +832,8 @@ __global__ void item_table_kernel(const PrefillArgs P) {
         const int chunk = static_cast<int>(li) - P.item_off[bk];
         const int cnt = P.bucket_cnt[bk];
         int4 *d = reinterpret_cast<int4 *>(P.item_desc) + 2 * (base + li);
-        d[0] = make_int4(b, g, j, min(kItemRows, cnt - chunk * kItemRows));
-        d[1] = make_int4(P.bucket_off[bk] + chunk * kItemRows, L, 0, 0);
+        d[0] = make_int4(b, g, j, min(P.item_rows, cnt - chunk * P.item_rows));
+        d[1] = make_int4(P.bucket_off[bk] + chunk * P.item_rows, L, 0, 0);
     }
 }
 
@@ -896,8 +896,11 @@ __global__ void __launch_bounds__(256) finalize_kernel(const PrefillArgs P) {
             if (!seq_ok(P, b, L)) {
                 const uint32_t nan2 = pack_bf16x2(NAN, NAN);
                 o = make_uint4(nan2, nan2, nan2, nan2);
+                if (P.lse && cd == 0) P.lse[row * P.H_q + g * kG + h] = NAN;
             } else {
                 const float inv = 1.f / l[u];
+                if (P.lse && cd == 0)
+                    P.lse[row * P.H_q + g * kG + h] = P.m_arr[row * P.H_q + g * kG + h] + log2f(l[u]);
                 const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
                 uint32_t o4[4];
 #pragma unroll
@@ -978,6 +981,7 @@ __global__ void exact_rows_kernel(const PrefillArgs P) {
             const uint2 wv = make_uint2(pack_bf16x2(o4[0] * inv, o4[1] * inv),
                                         pack_bf16x2(o4[2] * inv, o4[3] * inv));
             *reinterpret_cast<uint2 *>(out) = wv;
+            if (P.lse && lane == 0) P.lse[idx] = mx + log2f(l);
         }
     }
 }
@@ -994,9 +998,73 @@ cudaError_t launch_pass(const CUtensorMap &tq, const CUtensorMap &tk, const CUte
     return cudaGetLastError();
 }
 
+cudaError_t run_buckets(const PrefillArgs &a, const PrefillLayout &L, cudaStream_t s, const char *name) {
+    TraceScope t(s, name);
+    const size_t bsm = L.nb_max <= kBuildSmemBlocks ? static_cast<size_t>(2 * L.nb_max) * sizeof(int) : 0;
+    cudaError_t e;
+    if (bsm > 48 * 1024 &&
+        (e = cudaFuncSetAttribute(bucket_build_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(bsm))) != cudaSuccess)
+        return e;
+    bucket_build_kernel<<<static_cast<unsigned>(L.n_ranges_total), kBuildThreads, bsm, s>>>(a);
+    range_scan_kernel<<<1, 1024, 0, s>>>(a);
+    item_table_kernel<<<static_cast<unsigned>(L.n_ranges_total), 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 bool prefill_attention_supported(int H_q, int H_kv) { return H_q / H_kv == kG; }
+
+size_t prefill_bucket_layout(int B, int Sq, int H_kv, int K, int max_kv_len, int item_rows,
+                             size_t base, PrefillLayout *L) {
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    *L = PrefillLayout{};
+    L->nb_max = (max_kv_len + 127) / 128;
+    L->n_ranges = (Sq + kRange - 1) / kRange;
+    L->n_ranges_total = static_cast<long long>(B) * H_kv * L->n_ranges;
+    L->rows_per_range = Sq < kRange ? Sq : kRange;
+    L->n_buckets = L->n_ranges_total * L->nb_max;
+    const size_t per_range_rows = static_cast<size_t>(L->rows_per_range) * (K > 1 ? K - 1 : 1);
+    L->item_rows = item_rows;
+    L->items_per_range = static_cast<int>(L->nb_max + per_range_rows / item_rows + 1);
+    size_t o = base;
+    L->cnt = o;          o += up(static_cast<size_t>(L->n_buckets) * 4);
+    L->cur = o;          o += up(static_cast<size_t>(L->n_buckets) * 4);
+    L->zero_end = o;
+    L->off = o;          o += up(static_cast<size_t>(L->n_buckets) * 4);
+    L->item_off = o;     o += up(static_cast<size_t>(L->n_buckets) * 4);
+    L->item_bucket = o;  o += up(static_cast<size_t>(L->n_ranges_total) * L->items_per_range * 4);
+    L->range_count = o;  o += up(static_cast<size_t>(L->n_ranges_total) * 8);
+    L->range_item_off = o; o += up(static_cast<size_t>(L->n_ranges_total + 1) * 8);
+    L->rows = o;         o += up(static_cast<size_t>(L->n_ranges_total) * per_range_rows * 4);
+    L->item_desc = o;    o += up(static_cast<size_t>(L->n_ranges_total) * L->items_per_range * 32);
+    L->total = o;
+    return o;
+}
+
+cudaError_t launch_prefill_buckets(PrefillArgs &a, uint8_t *ws, const PrefillLayout &L,
+                                   long long *item_total, cudaStream_t s) {
+    a.bucket_cnt = reinterpret_cast<int *>(ws + L.cnt);
+    a.bucket_cur = reinterpret_cast<int *>(ws + L.cur);
+    a.bucket_off = reinterpret_cast<int *>(ws + L.off);
+    a.item_off = reinterpret_cast<int *>(ws + L.item_off);
+    a.item_bucket = reinterpret_cast<int *>(ws + L.item_bucket);
+    a.range_count = reinterpret_cast<long long *>(ws + L.range_count);
+    a.range_item_off = reinterpret_cast<long long *>(ws + L.range_item_off);
+    a.bucket_rows = reinterpret_cast<int *>(ws + L.rows);
+    a.item_desc = reinterpret_cast<int *>(ws + L.item_desc);
+    a.item_total = item_total;
+    a.nb_max = L.nb_max;
+    a.n_ranges = L.n_ranges;
+    a.n_ranges_total = L.n_ranges_total;
+    a.rows_per_range = L.rows_per_range;
+    a.items_per_range = L.items_per_range;
+    a.item_rows = L.item_rows;
+    cudaError_t e = cudaMemsetAsync(ws + L.cnt, 0, L.zero_end - L.cnt, s);
+    if (e != cudaSuccess) return e;
+    return run_buckets(a, L, s, "backward_bucket");
+}
 
 size_t prefill_workspace_layout(int B, int Sq, int H_q, int H_kv, int K, int max_kv_len,
                                 PrefillLayout *L) {
@@ -1008,6 +1076,7 @@ size_t prefill_workspace_layout(int B, int Sq, int H_q, int H_kv, int K, int max
     L->rows_per_range = Sq < kRange ? Sq : kRange;
     L->n_buckets = L->n_ranges_total * L->nb_max;
     const size_t per_range_rows = static_cast<size_t>(L->rows_per_range) * (K > 1 ? K - 1 : 1);
+    L->item_rows = kItemRows;
     L->items_per_range = static_cast<int>(L->nb_max + per_range_rows / kItemRows + 1);
     size_t o = kWsHeaderBytes;
     L->cnt = o;          o += up(static_cast<size_t>(L->n_buckets) * 4);
@@ -1055,6 +1124,7 @@ cudaError_t launch_prefill_attention(const PrefillArgs &a0, uint8_t *ws, const P
     a.n_ranges_total = L.n_ranges_total;
     a.rows_per_range = L.rows_per_range;
     a.items_per_range = L.items_per_range;
+    a.item_rows = L.item_rows;
 
     CUtensorMap tq, tk, tv;
     if (!encode_q_rows_map(&tq, a.q, a.H_q, static_cast<long long>(a.B) * a.Sq, kTileRows) ||
@@ -1064,18 +1134,7 @@ cudaError_t launch_prefill_attention(const PrefillArgs &a0, uint8_t *ws, const P
     cudaError_t e = cudaMemsetAsync(ws + L.cnt, 0, L.zero_end - L.cnt, s);
     if (e != cudaSuccess) return e;
     const int sms = device_sm_count();
-    {
-        TraceScope t(s, "prefill_bucket");
-        const size_t bsm = L.nb_max <= kBuildSmemBlocks ? static_cast<size_t>(2 * L.nb_max) * sizeof(int) : 0;
-        if (bsm > 48 * 1024 &&
-            (e = cudaFuncSetAttribute(bucket_build_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      static_cast<int>(bsm))) != cudaSuccess)
-            return e;
-        bucket_build_kernel<<<static_cast<unsigned>(L.n_ranges_total), kBuildThreads, bsm, s>>>(a);
-        range_scan_kernel<<<1, 1024, 0, s>>>(a);
-        item_table_kernel<<<static_cast<unsigned>(L.n_ranges_total), 256, 0, s>>>(a);
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = run_buckets(a, L, s, "prefill_bucket")) != cudaSuccess) return e;
     if ((e = launch_pass<0>(tq, tk, tv, a, s, "prefill_attn_own_block")) != cudaSuccess) return e;
     {
         TraceScope t(s, "prefill_bucket_shift");

@@ -79,6 +79,8 @@ __global__ void __launch_bounds__(kThreads, kStages == 1 ? 3 : 1)
     if (!valid) {
         if (split == 0) {
             for (int e = tid; e < G * kDim; e += kThreads) out[e] = __float2bfloat16(NAN);
+            if (P.lse)
+                for (int e = tid; e < G; e += kThreads) P.lse[row * P.H_q + static_cast<long long>(g) * G + e] = NAN;
             if (tid == 0 && i == 0 && g == 0) set_status(P.status, kStatusBadLens);
         }
         return;
@@ -362,6 +364,8 @@ __global__ void __launch_bounds__(kThreads, kStages == 1 ? 3 : 1)
             v.z = pack_bf16x2(o[4] * inv, o[5] * inv);
             v.w = pack_bf16x2(o[6] * inv, o[7] * inv);
             *reinterpret_cast<uint4 *>(out + h * kDim + d0) = v;
+            if (P.lse && d0 == 0)
+                P.lse[row * P.H_q + static_cast<long long>(g) * G + h] = aborted ? NAN : mref + log2f(l);
         } else {
             float *pr = part + split * rec;
             if (d0 == 0) { pr[h] = mx; pr[G + h] = aborted ? NAN : l; }
@@ -426,6 +430,7 @@ __global__ void __launch_bounds__(kThreads, kStages == 1 ? 3 : 1)
         v.z = pack_bf16x2(o[4] * inv, o[5] * inv);
         v.w = pack_bf16x2(o[6] * inv, o[7] * inv);
         *reinterpret_cast<uint4 *>(out + h * kDim + d0) = v;
+        if (P.lse && d0 == 0) P.lse[row * P.H_q + static_cast<long long>(g) * G + h] = mref + log2f(l);
     }
 }
 

@@ -300,7 +300,7 @@ msa_status_t sparse_attention_impl(const msa_shape_t *shape, const void *q, cons
                                    const void *v_cache, const int32_t *block_ids,
                                    const int32_t *lens, const KvMap &kv, float softmax_scale,
                                    void *out, void *workspace, size_t workspace_bytes,
-                                   msa_stream_t stream) {
+                                   msa_stream_t stream, float *lse = nullptr) {
     if (!q || !k_cache || !v_cache || !block_ids || !lens || !out) return MSA_ERR_INVALID_ARG;
     if (!(softmax_scale == softmax_scale) || softmax_scale == INFINITY || softmax_scale == -INFINITY)
         return MSA_ERR_INVALID_ARG;
@@ -321,11 +321,12 @@ msa_status_t sparse_attention_impl(const msa_shape_t *shape, const void *q, cons
         p.H_kv = shape->num_kv_heads; p.K = shape->top_k; p.max_kv_len = shape->max_kv_len;
         p.n_idx = index_heads(shape);
         p.softmax_scale = softmax_scale;
+        p.lse = lse;
         return launch_prefill_attention(p, ws, L.pre, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
     }
     AttnRowsArgs a;
     a.q = q; a.k_cache = k_cache; a.v_cache = v_cache; a.ids = block_ids; a.lens = lens;
-    a.kv = kv; a.out = out;
+    a.kv = kv; a.out = out; a.lse = lse;
     a.partials = reinterpret_cast<float *>(ws + L.partials_off);
     a.tickets = reinterpret_cast<int *>(ws + L.tickets_off);
     a.status = reinterpret_cast<int *>(ws);
@@ -448,9 +449,17 @@ msa_status_t msa_kv_append(const msa_shape_t *shape, int32_t n_new, const void *
                                                                                      : MSA_ERR_CUDA;
 }
 
+// The backward's workspace: the forward's (recomputed first, from byte 0),
+// then the output, statistics, dQ accumulator and buckets of the backward.
+static size_t bwd_layout(const msa_shape_t *s, AttnBwdLayout *L) {
+    return attn_bwd_layout(s->batch, s->q_len, s->num_q_heads, s->num_kv_heads, s->top_k,
+                           s->max_kv_len, attn_layout(s).total, L);
+}
+
 size_t msa_sparse_attention_backward_workspace_size(const msa_shape_t *shape) {
     if (check_shape(shape) != MSA_OK) return 0;
-    return kWsHeaderBytes;
+    AttnBwdLayout L;
+    return bwd_layout(shape, &L);
 }
 
 msa_status_t msa_sparse_attention_backward(const msa_shape_t *shape, const void *q,
@@ -470,9 +479,18 @@ msa_status_t msa_sparse_attention_backward(const msa_shape_t *shape, const void 
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(d_out) ||
         !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
         return MSA_ERR_MISALIGNED;
-    if ((st = check_ws(workspace, workspace_bytes, kWsHeaderBytes)) != MSA_OK) return st;
+    AttnBwdLayout L;
+    const size_t need = bwd_layout(shape, &L);
+    if ((st = check_ws(workspace, workspace_bytes, need)) != MSA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (clear_header(workspace, kWsHeaderBytes, s) != cudaSuccess) return MSA_ERR_CUDA;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    // The forward, recomputed: its output and log-sum-exp go to the backward's
+    // regions (it clears the header and owns bytes 4..31 of it).
+    const KvMap kv = packed_map(shape, kv_offsets);
+    if ((st = sparse_attention_impl(shape, q, k_cache, v_cache, block_ids, lens, kv, softmax_scale,
+                                    ws + L.o, workspace, workspace_bytes, stream,
+                                    reinterpret_cast<float *>(ws + L.lse))) != MSA_OK)
+        return st;
     AttnBwdArgs a;
     a.q = q; a.k_cache = k_cache; a.v_cache = v_cache; a.dout = d_out; a.ids = block_ids;
     a.lens = lens; a.kv = packed_map(shape, kv_offsets); a.dq = dq; a.dk = dk; a.dv = dv;
@@ -480,7 +498,7 @@ msa_status_t msa_sparse_attention_backward(const msa_shape_t *shape, const void 
     a.B = shape->batch; a.Sq = shape->q_len; a.H_q = shape->num_q_heads;
     a.H_kv = shape->num_kv_heads; a.n_idx = index_heads(shape); a.K = shape->top_k;
     a.max_kv_len = shape->max_kv_len; a.softmax_scale = softmax_scale;
-    return launch_attn_bwd(a, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+    return launch_attn_bwd(a, ws, L, s) == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
 }
 
 // The fused decode step takes bf16 index keys, one row per index head (any

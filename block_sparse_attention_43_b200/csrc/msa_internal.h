@@ -106,6 +106,7 @@ struct AttnRowsArgs {
     const int32_t *lens;
     KvMap kv;
     void *out;              // [B][Sq][H_q][128]
+    float *lse;             // optional [rows][H_q]: base-2 log-sum-exp (as PrefillArgs)
     float *partials;        // [B*Sq][H_kv][nsplit][attn_partial_floats(G)]
     int *tickets;           // [B*Sq][H_kv]
     int *status;
@@ -134,6 +135,9 @@ struct PrefillArgs {
     int B, Sq, H_q, H_kv, K, max_kv_len;
     int n_idx;              // index heads: group g reads ids of g / (H_kv / n_idx)
     float softmax_scale;
+    float *lse;             // optional [rows][H_q]: base-2 log-sum-exp of the
+                            // scaled logits (p = 2^(s * scale * log2 e - lse))
+    int item_rows;          // max rows per bucket work item
     // workspace views (filled by launch_prefill_attention)
     int *bucket_cnt, *bucket_cur, *bucket_off, *bucket_rows;  // per (range, block j)
     int *item_off;          // first item of each bucket, counted inside its range
@@ -154,7 +158,7 @@ struct PrefillArgs {
 struct PrefillLayout {
     size_t cnt, cur, l_acc, flags, zero_end, off, item_off, item_bucket, range_count,
         range_item_off, rows, shift, item_desc, o_acc, m_arr, total;
-    int nb_max, n_ranges, rows_per_range, items_per_range;
+    int nb_max, n_ranges, rows_per_range, items_per_range, item_rows;
     long long n_ranges_total, n_buckets;
 };
 bool prefill_attention_supported(int H_q, int H_kv);
@@ -162,6 +166,13 @@ size_t prefill_workspace_layout(int B, int Sq, int H_q, int H_kv, int K, int max
                                 PrefillLayout *L);
 cudaError_t launch_prefill_attention(const PrefillArgs &a, uint8_t *ws, const PrefillLayout &L,
                                      cudaStream_t s);
+// Buckets alone (rows that kept block j != own, as work items of at most
+// item_rows rows), laid out from byte `base` of a workspace; returns the end.
+// The item count lands in *item_total, the 32-byte descriptors in item_desc.
+size_t prefill_bucket_layout(int B, int Sq, int H_kv, int K, int max_kv_len, int item_rows,
+                             size_t base, PrefillLayout *L);
+cudaError_t launch_prefill_buckets(PrefillArgs &a, uint8_t *ws, const PrefillLayout &L,
+                                   long long *item_total, cudaStream_t s);
 // 3-D map over q [rows, H_q, 128] with a box of 64 dims x 8 heads x box_rows
 // rows, 128-byte swizzle.
 bool encode_q_rows_map(CUtensorMap *map, const void *q, int H_q, long long rows, int box_rows);
@@ -201,7 +212,9 @@ size_t decode_fused_layout(int B, int H_q, int H_kv, int n_idx, int K, int max_k
                            DecodeFusedLayout *L);
 cudaError_t launch_decode_fused(const DecodeFusedArgs &a, cudaStream_t s);
 
-// Backward of the sparse branch (attn_bwd.cu): one CTA per (row, group).
+// Backward of the sparse branch (attn_bwd.cu), organised around the KV
+// blocks.  The caller has run the forward into o and lse (the workspace
+// regions of AttnBwdLayout) on the same stream.
 struct AttnBwdArgs {
     const void *q;          // [B][Sq][H_q][128]
     const void *k_cache;
@@ -215,8 +228,26 @@ struct AttnBwdArgs {
     int *status;
     int B, Sq, H_q, H_kv, n_idx, K, max_kv_len;
     float softmax_scale;
+    // workspace views (filled by launch_attn_bwd)
+    const void *o;          // [rows][H_q][128] bf16: the recomputed forward output
+    const float *lse;       // [rows][H_q] base-2 log-sum-exp of the scaled logits
+    float *delta;           // [rows][H_q] dO . O
+    float *dq_acc;          // [rows][H_q][128] fp32, already scaled
+    const int *bucket_rows; // bucket entries -> flattened row
+    const int *item_desc;   // bucket work items (32 bytes each)
+    const long long *item_total;
+    long long *item_next;   // claim counter
 };
-cudaError_t launch_attn_bwd(const AttnBwdArgs &a, cudaStream_t s);
+struct AttnBwdLayout {
+    size_t o, lse, delta, dq_acc, total;
+    PrefillLayout bk;       // the backward's own buckets
+};
+// Lays the backward's regions out from byte `base` of the workspace (the
+// forward's layout ends there); returns the total size.
+size_t attn_bwd_layout(int B, int Sq, int H_q, int H_kv, int K, int max_kv_len, size_t base,
+                       AttnBwdLayout *L);
+cudaError_t launch_attn_bwd(const AttnBwdArgs &a, uint8_t *ws, const AttnBwdLayout &L,
+                            cudaStream_t s);
 
 struct KvAppendArgs {
     const void *src[3];

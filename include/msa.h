@@ -182,17 +182,23 @@ MSA_API msa_status_t msa_sparse_attention(const msa_shape_t *shape, const void *
  *   Delta = sum_t P_t dP_t, dZ_t = P_t (dP_t - Delta),
  *   dq = softmax_scale * sum_t dZ_t k_t,
  *   dk_t += softmax_scale * dZ_t q,   dv_t += P_t d_out.
- * The forward softmax is recomputed (no saved statistics are needed).
+ * The forward is recomputed inside the call (no saved statistics are
+ * needed): its output gives Delta = d_out . out, and it also yields each
+ * (row, head)'s log-sum-exp.  The products then run around the kept blocks:
+ * each block's dk and dv are summed on chip over all rows that kept it and
+ * added once per work item; dq is summed in an fp32 workspace buffer.
  *   q, k_cache, v_cache, block_ids, lens, kv_offsets: as msa_sparse_attention
  *   d_out        device bf16 [B, q_len, H_q, head_dim], gradient of out
- *   dq           device bf16 [B, q_len, H_q, head_dim]  (written)
+ *   dq           device bf16 [B, q_len, H_q, head_dim]  (written; NaN for
+ *                sequences with bad lengths and after a device timeout)
  *   dk, dv       device float [kv_capacity, H_kv, head_dim]: the gradients of
  *                this call are ADDED (fp32 atomics, so their summation order
- *                and last bits vary by run); start them at zero.
+ *                and last bits vary by run); start them at zero.  Keys that
+ *                no row reaches are not written.
  *   workspace    >= msa_sparse_attention_backward_workspace_size bytes
- * This is a first, row-oriented implementation (one CTA per row and group):
- * every (row, kept block) adds a 128 x 128 block to dk and dv, which bounds
- * it at large q_len. */
+ *                (the forward's workspace, then the recomputed output, two
+ *                floats per (row, head), the fp32 dq sum and work lists:
+ *                about rows x H_q x 776 bytes beyond the forward's) */
 MSA_API size_t msa_sparse_attention_backward_workspace_size(const msa_shape_t *shape);
 MSA_API msa_status_t msa_sparse_attention_backward(const msa_shape_t *shape, const void *q,
                                                    const void *k_cache, const void *v_cache,

@@ -169,3 +169,23 @@ def to_host(m):
     sc = m.block_scores.cpu().numpy()
     out = m.out.float().cpu().numpy()
     return ids, sc, out
+
+
+def oracle_rows_backward(oracle_mod, q, k, v, dout, ids, pos, scale, parts=8):
+    """Backward of independent rows (row i at position pos[i]) over one shared
+    cache: each row is its own single-row sequence at offset 0.  The oracle's
+    threads each own whole (sequence, group) jobs and assume sequences do not
+    share cache rows, so the rows go in `parts` single-threaded calls on
+    separate outputs, run side by side, and the dK, dV parts are summed."""
+    from concurrent.futures import ThreadPoolExecutor
+    n = len(pos)
+    cuts = np.linspace(0, n, parts + 1).astype(int)
+
+    def one(a, b):
+        return oracle_mod.sparse_attention_backward(
+            q[a:b], k, v, dout[a:b], ids[a:b], (pos[a:b] + 1).astype(np.int32),
+            np.zeros(b - a, np.int64), scale=scale, n_threads=1)
+
+    with ThreadPoolExecutor(parts) as ex:
+        res = list(ex.map(lambda ab: one(*ab), [(a, b) for a, b in zip(cuts[:-1], cuts[1:]) if b > a]))
+    return (np.concatenate([r[0] for r in res]), sum(r[1] for r in res), sum(r[2] for r in res))

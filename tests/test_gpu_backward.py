@@ -3,11 +3,14 @@ blocks) through the C ABI against the CPU oracle's exact derivative, on the
 same bf16 inputs and the same selection.
 
 Tolerance: relative L2 <= 5e-3 (the forward's bound) and max-abs <= 2 % of
-the largest reference magnitude, per gradient.  The kernel rounds P and dZ to
-bf16 as operands of the products (at most 2^-9 relative each, about 1.1e-3
-RMS for round-to-nearest) and writes dQ as bf16 (another 2^-9); dK and dV
-are fp32 sums of those products, so the rounding adds in quadrature to about
-2e-3 RMS, inside 5e-3.
+the largest reference magnitude, per gradient.  The kernel rounds P to bf16
+(the operand of dV = P^T dO, and the P that dS = P (dP - Delta) is formed
+from) and dS to bf16 (the operand of dK and dQ): at most 2^-9 relative each,
+about 1.1e-3 RMS for round-to-nearest, about 1.6e-3 for dS's two roundings;
+Delta = dO.O is taken from the recomputed bf16 output, whose error enters dS
+only scaled by |O| / |v| < 1; dQ is written as bf16 (another 1.1e-3).  dK and
+dV are fp32 sums of those products, so the rounding adds in quadrature to
+about 2-2.5e-3 RMS, inside 5e-3.
 """
 import numpy as np
 import pytest
@@ -70,6 +73,7 @@ def _run(oracle_mod, w, n_idx=None, padded_nan=False):
 
 CASES = [
     # (B, Sq, lens, H_q, H_kv, top_k)
+    (1, 2048, [2048], 8, 2, 4),            # the 2k-row prefill shape
     (1, 300, [300], 8, 2, 4),              # full prefill, ragged last block
     (2, 64, [500, 64], 16, 4, 3),          # chunked prefill after a cached prefix
     (1, 1000, [1000], 64, 8, 16),          # groups of 8, every block kept
@@ -104,3 +108,49 @@ def test_backward_ignores_nan_padding(oracle_mod):
         for b, L in enumerate(lens):
             t[b * 1024 + L:(b + 1) * 1024] = float("nan")
     print(_run(oracle_mod, w, padded_nan=True))
+
+
+def test_backward_32k_rows_sampled(oracle_mod):
+    """Groups of 8 at 32,768 rows (the 128k prefill recipe at a quarter of its
+    length): dK and dV of whole key blocks, and dQ of the rows that reach
+    them, against the oracle.  A row's gradient terms depend only on its own
+    q, dO and kept blocks, so the rows that kept block j in group g, run
+    through the oracle as single-row sequences (length = position + 1) over
+    the same cache, give block j's exact dK and dV in group g."""
+    from parity import oracle_rows_backward
+    from synthetic import bf16_bits, make_inputs
+    Sq, H_q, H_kv, G = 32768, 64, 8, 8
+    w = make_inputs(B=1, Sq=Sq, lens=[Sq], H_q=H_q, H_kv=H_kv, top_k=16, seed=732, device=DEV)
+    eng = m.MSA(batch=1, q_len=Sq, max_kv_len=Sq, num_q_heads=H_q, num_kv_heads=H_kv, top_k=16,
+                kv_capacity=w.kv_capacity, device=DEV)
+    eng.index_topk(w.q_idx, w.k_idx, w.lens, w.kv_offsets)
+    g = torch.Generator(device=DEV).manual_seed(78)
+    dout = torch.randn(w.q.shape, generator=g, device=DEV).to(torch.bfloat16)
+    dq = torch.empty_like(w.q)
+    dk = torch.zeros(w.k.shape, dtype=torch.float32, device=DEV)
+    dv = torch.zeros(w.v.shape, dtype=torch.float32, device=DEV)
+    ws = m.alloc_workspace(m.msa_sparse_attention_backward_workspace_size(eng.shape), DEV)
+    m.msa_sparse_attention_backward(eng.shape, w.q, w.k, w.v, eng.block_ids, w.lens,
+                                    w.kv_offsets, w.scale, dout, dq, dk, dv, ws)
+    torch.cuda.synchronize()
+    assert m.msa_read_device_status(ws) == 0
+    ids = eng.block_ids.cpu().numpy().reshape(Sq, H_kv, 16)
+    qh = bf16_bits(w.q).reshape(Sq, H_q, 128)
+    dh = bf16_bits(dout).reshape(Sq, H_q, 128)
+    kh, vh = bf16_bits(w.k), bf16_bits(w.v)
+    gq = dq.float().cpu().numpy().reshape(Sq, H_q, 128)
+    gk, gv = dk.cpu().numpy(), dv.cpu().numpy()
+    # the last block (its own rows only), a late block and an earlier one
+    for grp, j in [(0, 255), (3, 200), (7, 150)]:
+        rows = np.nonzero((ids[:, grp, :] == j).any(axis=1))[0]
+        n = rows.size
+        hs = slice(grp * G, (grp + 1) * G)
+        rq, rk, rv = oracle_rows_backward(oracle_mod, qh[rows, hs][:, None].copy(),
+                                  kh[:, grp:grp + 1].copy(), vh[:, grp:grp + 1].copy(),
+                                  dh[rows, hs][:, None].copy(), ids[rows, grp][:, None, :].copy(),
+                                  rows, w.scale)
+        t = slice(j * 128, (j + 1) * 128)
+        rep = dict(rows=n, dk=_check(f"dk[{j},{grp}]", gk[t, grp], rk[t, 0]),
+                   dv=_check(f"dv[{j},{grp}]", gv[t, grp], rv[t, 0]),
+                   dq=_check(f"dq[rows of {j},{grp}]", gq[rows, hs], rq.reshape(n, G, 128)))
+        print(grp, j, rep)

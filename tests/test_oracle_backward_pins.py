@@ -141,3 +141,25 @@ def test_backward_with_fewer_index_heads_equals_replicated_ids(oracle_mod):
     np.testing.assert_array_equal(dq2, dq4)
     np.testing.assert_array_equal(dk2, dk4)
     np.testing.assert_array_equal(dv2, dv4)
+
+
+def test_oracle_rows_helper_matches_full_oracle(oracle_mod):
+    """oracle_rows_backward (tests/parity.py), whose split single-row calls
+    the 32k-row GPU test uses, gives the same dQ, dK and dV as one
+    oracle call on the whole prefill (checked on the CPU here, no GPU used)."""
+    from parity import host_inputs, oracle_rows_backward
+    Sq, H_q = 700, 8
+    w = make_inputs(B=1, Sq=Sq, lens=[Sq], H_q=H_q, H_kv=1, top_k=3, seed=41, device="cpu")
+    a = host_inputs(w)
+    ids = oracle_mod.index_topk(a["q_idx"], a["k_idx"], a["lens"], a["kv_offsets"],
+                                top_k=w.top_k)["block_ids"]
+    dout = bf16_bits(torch.randn(w.q.shape, generator=torch.Generator().manual_seed(4))
+                     .to(torch.bfloat16))
+    rq, rk, rv = oracle_mod.sparse_attention_backward(a["q"], a["k"], a["v"], dout, ids, a["lens"],
+                                                      a["kv_offsets"], scale=w.scale)
+    sq, sk, sv = oracle_rows_backward(oracle_mod, a["q"].reshape(Sq, 1, H_q, 128), a["k"],
+                                      a["v"], dout.reshape(Sq, 1, H_q, 128),
+                                      ids.reshape(Sq, 1, -1), np.arange(Sq), w.scale, parts=4)
+    assert np.allclose(sq.reshape(rq.shape), rq, rtol=1e-12, atol=1e-12)
+    assert np.allclose(sk, rk, rtol=1e-10, atol=1e-12)
+    assert np.allclose(sv, rv, rtol=1e-10, atol=1e-12)
