@@ -303,14 +303,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const uint32_t id_kk = umma_idesc_bf16(128, 128);            // A, B K-major
             const uint32_t id_kb = id_kk | (1u << 16);                   // B MN-major
+            const uint32_t id_mk = id_kk | (1u << 15);                   // A MN-major
             const uint32_t id_mm = id_kk | (1u << 15) | (1u << 16);      // A and B MN-major
             const uint32_t kv0 = smem_u32(S.kv), ds0 = smem_u32(S.ds);
             // Descriptors are built once; a k-step only moves the start address.
             const uint64_t k_kd = umma_desc(kv0, 16, 1024);              // K_j: tokens x dims
-            const uint64_t k_mn = umma_desc(kv0, 16384, 1024);           // K_j as dims-contiguous B
+            const uint64_t k_mn = umma_desc(kv0, 16384, 1024);           // K_j^T: dims x tokens, transposed read
             const uint64_t v_kd = umma_desc(kv0 + 32768, 16, 1024);      // V_j: tokens x dims
-            const uint64_t ds_kd = umma_desc(ds0, 16, 1024);             // dS^T: tokens x pairs
-            const uint64_t ds_mn = umma_desc(ds0, 16384, 1024);          // dS (pairs x tokens), transposed read
+            const uint64_t ds_kd = umma_desc(ds0, 16, 1024);             // dS: tokens (N) x pairs (K)
+            const uint64_t ds_mn = umma_desc(ds0, 16384, 1024);          // dS^T: tokens (K) x pairs (N)
             // Stage 1's descriptors are stage 0's moved by 64 KiB (4096 16-byte units).
             const uint32_t qa = smem_u32(S.qdo[0]);
             const uint64_t q_kd0 = umma_desc(qa, 16, 1024), q_mn0 = umma_desc(qa, 16384, 1024);
@@ -328,21 +329,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (x.n == 0) continue;
                 if (!wait(&S.kv_full, ki & 1) || !wait(&S.kv_ready, ki & 1)) { ok = false; break; }
                 const int ntile = (x.n + TR - 1) / TR;
+                // S^T of tile q (Q from stage q & 1).  S^T's columns hold the
+                // previous tile's P^T until that tile's dV is done.
+                auto issue_s = [&](int q) -> bool {
+                    const int sq = q & 1;
+                    if (!wait(&S.qdo_full[sq], (q >> 1) & 1)) return false;
+                    fence_proxy_async_smem();            // Q, dO rows were written by cp.async
+                    if (q >= 1 && !wait(&S.dv_done, (q - 1) & 1)) return false;
+                    tc_fence_after();
+                    const uint64_t qk = q_kd0 + static_cast<uint64_t>(sq * 4096);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_bf16_ss(tmem + kColS, k_kd + kstep(kk), qk + kstep(kk), id_kk, kk > 0 ? 1u : 0u);
+                    umma_commit(&S.s_full);
+                    return true;
+                };
+                if (!issue_s(qt)) { ok = false; break; }
                 for (int t = 0; t < ntile; ++t, ++qt) {
                     const int st = qt & 1;
                     const uint64_t so = static_cast<uint64_t>(st * 4096);
-                    const uint64_t q_kd = q_kd0 + so, q_mn = q_mn0 + so;
-                    const uint64_t do_kd = do_kd0 + so, do_mn = do_mn0 + so;
-                    if (!wait(&S.qdo_full[st], (qt >> 1) & 1)) { ok = false; break; }
-                    fence_proxy_async_smem();           // Q, dO rows were written by cp.async
-                    // S^T's columns hold the previous tile's P^T until its dV is done.
-                    if (qt >= 1 && !wait(&S.dv_done, (qt - 1) & 1)) { ok = false; break; }
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16_ss(tmem + kColS, k_kd + kstep(kk), q_kd + kstep(kk), id_kk, kk > 0 ? 1u : 0u);
-                    umma_commit(&S.s_full);
-                    // dP^T's columns hold the previous tile's dQ until the epilogue has read it.
+                    const uint64_t q_mn = q_mn0 + so, do_kd = do_kd0 + so, do_mn = do_mn0 + so;
+                    // dP^T's columns hold the previous tile's dQ^T until the epilogue has read it.
                     if (qt >= 1 && !wait(&S.dq_empty, (qt - 1) & 1)) { ok = false; break; }
                     tc_fence_after();
 #pragma unroll
@@ -360,17 +367,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      (t > 0 || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(&S.dv_done);
+                    // The next tile's S^T goes ahead of this tile's dQ and dK, so
+                    // the softmax warps start on it while those two run.
+                    if (t + 1 < ntile && !issue_s(qt + 1)) { ok = false; break; }
                     if (!wait(&S.ds_ready, qt & 1)) { ok = false; break; }
                     tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)        // dQ = dS K_j, into dP^T's columns
-                        umma_bf16_ss(tmem + kColDP, ds_mn + static_cast<uint64_t>(kk * 128),
-                                     k_mn + static_cast<uint64_t>(kk * 128), id_mm, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < 8; ++kk)        // dQ^T = K_j^T dS^T, into dP^T's columns
+                        umma_bf16_ss(tmem + kColDP, k_mn + static_cast<uint64_t>(kk * 128),
+                                     ds_mn + static_cast<uint64_t>(kk * 128), id_mm, kk > 0 ? 1u : 0u);
                     umma_commit(&S.dq_full);
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)        // dK += dS^T Q
-                        umma_bf16_ss(tmem + kColDK, ds_kd + kstep(kk), q_mn + static_cast<uint64_t>(kk * 128),
-                                     id_kb, (t > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 8; ++kk)        // dK^T += Q^T dS
+                        umma_bf16_ss(tmem + kColDK, q_mn + static_cast<uint64_t>(kk * 128), ds_kd + kstep(kk),
+                                     id_mk, (t > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&S.ds_empty);
                     umma_commit(&S.qdo_empty[st]);
                     if (t == ntile - 1) {
@@ -561,13 +571,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) *abort_flag = 1;
     } else if (warp >= kEpiWarp0) {
         // ------------------------------------------------ epilogue
-        // Per tile: lane m = pair (tile row m / G, head m % G) reads its dQ
-        // row (128 fp32) and adds it to the accumulator with vector
-        // reductions.  Per item: lane m = token m of the block adds its dV
-        // and dK rows to the caller's buffers.
+        // dQ^T (per tile) and dK^T (per item) have lane = dim, column = pair
+        // or token: each column's 32 dims of a warp leave as one coalesced
+        // 128-byte fp32 reduction (a full line; 16-byte pieces of separate
+        // rows would each cost a whole 32-byte sector operation at L2).  dV
+        // (per item) has lane = token and goes out as 16-byte vector
+        // reductions along its row.  Pair p = tile row p / G, head p % G.
+        constexpr int NRR = (TR + 31) / 32;                  // tile rows per lane
         const int w = warp & 3;
-        const int m = w * 32 + lane;
-        const int r = m / G, h = m % G;
+        const int d = w * 32 + lane;                          // dim (dQ^T, dK^T) or token (dV)
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(w * 32) << 16);
         int qt = 0, ki = 0, n = 0;
         bool ok = true;
@@ -580,57 +592,99 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; e += 4) red_add_v4(dst + e, v[e], v[e + 1], v[e + 2], v[e + 3]);
         };
+        // Accumulator row bases of tile rows lane, lane + 32, ... (0: no row).
+        auto row_bases = [&](const BItem &it, int t, unsigned long long (&rb)[NRR]) {
+#pragma unroll
+            for (int i = 0; i < NRR; ++i) {
+                const int rr = lane + 32 * i;
+                rb[i] = 0;
+                if (rr < TR && t * TR + rr < it.n)
+                    rb[i] = reinterpret_cast<unsigned long long>(
+                        P.dq_acc + (item_row(P, it, t * TR + rr) * P.H_q + static_cast<long long>(it.g) * G) * kDim);
+            }
+        };
         while (ok) {
             if (!next_item(n++, true, x)) { ok = false; break; }
             if (x.n < 0) break;
             if (x.n == 0) continue;
             const int ntile = (x.n + TR - 1) / TR;
-            long long row_nx = r < x.n ? item_row(P, x, r) : -1;
+            unsigned long long rb_nx[NRR];
+            row_bases(x, 0, rb_nx);
             for (int t = 0; t < ntile; ++t, ++qt) {
-                const long long row = row_nx;
-                if (t + 1 < ntile) row_nx = (t + 1) * TR + r < x.n ? item_row(P, x, (t + 1) * TR + r) : -1;
-                float *dst = row >= 0 ? P.dq_acc + (row * P.H_q + static_cast<long long>(x.g) * G + h) * kDim
-                                      : nullptr;
+                unsigned long long rb[NRR];
+#pragma unroll
+                for (int i = 0; i < NRR; ++i) rb[i] = rb_nx[i];
+                if (t + 1 < ntile) row_bases(x, t + 1, rb_nx);
                 if (!wait_all(&S.dq_full, qt & 1)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t a[32], b[32];
-                tmem_ld32r(lane_addr + kColDP, a);
-                tmem_ld32r(lane_addr + kColDP + 32, b);
-                tmem_wait_ld(a);
-                tmem_tie(b);
-                if (dst) { red_row(dst, a); red_row(dst + 32, b); }
-                tmem_ld32r(lane_addr + kColDP + 64, a);
-                tmem_ld32r(lane_addr + kColDP + 96, b);
-                tmem_wait_ld(a);
-                tmem_tie(b);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&S.dq_empty);
-                if (dst) { red_row(dst + 64, a); red_row(dst + 96, b); }
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t a[32], b[32];
+                    tmem_ld32r(lane_addr + kColDP + half * 64, a);
+                    tmem_ld32r(lane_addr + kColDP + half * 64 + 32, b);
+                    tmem_wait_ld(a);
+                    tmem_tie(b);
+                    if (half == 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&S.dq_empty);
+                    }
+#pragma unroll
+                    for (int r2 = 0; r2 < 64 / G; ++r2) {        // the half's tile rows
+                        const int rr = half * (64 / G) + r2;
+                        const unsigned long long base = __shfl_sync(0xffffffffu, rb[rr / 32], rr % 32);
+                        if (!base) continue;
+                        float *dst = reinterpret_cast<float *>(base) + d;
+#pragma unroll
+                        for (int hh = 0; hh < G; ++hh) {
+                            const int e = r2 * G + hh;
+                            asm volatile("red.global.add.f32 [%0], %1;" ::"l"(dst + hh * kDim),
+                                         "f"(__uint_as_float(e < 32 ? a[e] : b[e - 32]))
+                                         : "memory");
+                        }
+                    }
+                }
             }
             if (!ok) break;
             if (!wait_all(&S.acc_full, ki & 1)) { ok = false; break; }
             tc_fence_after();
-            // Tokens past the sequence's end (own block only) get no gradient.
-            const bool tv = x.j * 128 + m < x.L;
-            const long long trow = kv_block_row(P.kv, x.b, x.j, P.status) + m;
-            float *dvp = P.dv + (trow * P.H_kv + x.g) * kDim;
-            float *dkp = P.dk + (trow * P.H_kv + x.g) * kDim;
+            const long long trow0 = kv_block_row(P.kv, x.b, x.j, P.status);
+            const int nvalid = x.L - x.j * 128;             // tokens inside the sequence
+            {   // dV: lane = token d of the block
+                float *dvp = P.dv + ((trow0 + d) * P.H_kv + x.g) * kDim;
 #pragma unroll 1
-            for (int q4 = 0; q4 < 4; ++q4) {                    // dV, then dK, 64 columns at a time
-                const uint32_t col = (q4 < 2 ? kColDV : kColDK) + (q4 & 1) * 64;
-                float *dst = (q4 < 2 ? dvp : dkp) + (q4 & 1) * 64;
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t a[32], b[32];
+                    tmem_ld32r(lane_addr + kColDV + hf * 64, a);
+                    tmem_ld32r(lane_addr + kColDV + hf * 64 + 32, b);
+                    tmem_wait_ld(a);
+                    tmem_tie(b);
+                    if (d < nvalid) { red_row(dvp + hf * 64, a); red_row(dvp + hf * 64 + 32, b); }
+                }
+            }
+            // dK^T: lane = dim d, column = token
+#pragma unroll 1
+            for (int hf = 0; hf < 2; ++hf) {
                 uint32_t a[32], b[32];
-                tmem_ld32r(lane_addr + col, a);
-                tmem_ld32r(lane_addr + col + 32, b);
+                tmem_ld32r(lane_addr + kColDK + hf * 64, a);
+                tmem_ld32r(lane_addr + kColDK + hf * 64 + 32, b);
                 tmem_wait_ld(a);
                 tmem_tie(b);
-                if (q4 == 3) {
+                if (hf == 1) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S.acc_empty);
                 }
-                if (tv) { red_row(dst, a); red_row(dst + 32, b); }
+#pragma unroll
+                for (int e = 0; e < 64; ++e) {
+                    const int tk = hf * 64 + e;
+                    if (tk < nvalid) {
+                        float *dst = P.dk + ((trow0 + tk) * P.H_kv + x.g) * kDim + d;
+                        asm volatile("red.global.add.f32 [%0], %1;" ::"l"(dst),
+                                     "f"(__uint_as_float(e < 32 ? a[e] : b[e - 32]))
+                                     : "memory");
+                    }
+                }
             }
             ++ki;
         }
