@@ -68,6 +68,9 @@ def parse():
                     help="override the prefill length (profiling captures of a smaller case)")
     ap.add_argument("--decode-len", type=int, default=None,
                     help="override the decode context length (profiling captures of a smaller case)")
+    ap.add_argument("--backward-rows", type=int, default=None,
+                    help="only time the backward on the prefill_128k recipe at this many rows "
+                         "(profiling captures); prints its JSON object")
     return ap.parse_args()
 
 
@@ -733,6 +736,12 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.backward_rows is not None:
+        torch.cuda.set_device(0)
+        r = measure_backward("prefill_128k", torch.device("cuda", 0), args.steps, max(args.warmup, 1),
+                             seq_len=args.backward_rows)
+        print(json.dumps(r), flush=True)
+        return
     if args.workload.startswith("prefill"):
         return run_prefill_headline(args)
     import block_sparse_attention_43_b200 as msa
@@ -829,8 +838,15 @@ def main():
 
     backward = None
     if not args.no_backward and world == 1:
-        backward = measure_backward("prefill_2k", dev, 20, 3)
-        backward["at_32k_rows"] = measure_backward("prefill_128k", dev, 5, 2, seq_len=32768)
+        # the 128k prefill recipe at 32,768 rows (the largest backward that
+        # keeps the default run short) and the 2k-row prefill
+        big = measure_backward("prefill_128k", dev, 5, 2, seq_len=32768)
+        _, tf_burst, _, kind = measured_peaks()
+        big["roofline"] = {"bound": "tensor", "kernel": "whole backward call (forward recompute included)",
+                           "achieved": big["tflops"], "peak": tf_burst, "peak_kind": kind + " burst",
+                           "unit": "TFLOP/s", "frac": big["frac_of_bf16_burst"]}
+        backward = {"prefill_128k_at_32k_rows": big,
+                    "prefill_2k": measure_backward("prefill_2k", dev, 20, 3)}
 
     prefill = None
     configs = None

@@ -53,6 +53,12 @@ constexpr int kSoftWarps = 8;
 constexpr int kEpiWarps = 4;
 constexpr int kEpiWarp0 = 4 + kSoftWarps;   // first epilogue warp
 constexpr int kTilesPerItem = 16;           // bucket items hold up to 16 tiles of rows
+#ifndef MSA_BWD_RANGE_ROWS
+#define MSA_BWD_RANGE_ROWS 8192
+#endif
+// Bucket items are claimed range by range; a range's Q, dO and dQ
+// accumulator rows (8 KiB per row and group) should stay in L2 meanwhile.
+constexpr int kRangeRows = MSA_BWD_RANGE_ROWS;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -778,7 +784,8 @@ size_t attn_bwd_layout(int B, int Sq, int H_q, int H_kv, int K, int max_kv_len, 
     L->delta = o;   o += up(pairs * 4);
     L->dq_acc = o;  o += up(pairs * kDim * 4);
     const int G = H_q / H_kv;
-    o = prefill_bucket_layout(B, Sq, H_kv, K, max_kv_len, kTilesPerItem * (128 / G), o, &L->bk);
+    o = prefill_bucket_layout(B, Sq, H_kv, K, max_kv_len, kTilesPerItem * (128 / G), kRangeRows, o,
+                              &L->bk);
     L->total = o;
     return o;
 }

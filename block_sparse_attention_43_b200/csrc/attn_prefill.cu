@@ -721,7 +721,7 @@ __global__ void __launch_bounds__(kBuildThreads) bucket_build_kernel(const Prefi
         if (tid == 0) P.range_count[r] = 0;
         return;
     }
-    const int i0 = rng * kRange, i1 = min(P.Sq, i0 + kRange);
+    const int i0 = rng * P.rows_per_range, i1 = min(P.Sq, i0 + P.rows_per_range);
     const long long n_e = static_cast<long long>(i1 - i0) * P.K;
     const bool in_smem = P.nb_max <= kBuildSmemBlocks;
     int *cnt = in_smem ? build_smem : P.bucket_cnt + r * P.nb_max;
@@ -1017,13 +1017,13 @@ cudaError_t run_buckets(const PrefillArgs &a, const PrefillLayout &L, cudaStream
 bool prefill_attention_supported(int H_q, int H_kv) { return H_q / H_kv == kG; }
 
 size_t prefill_bucket_layout(int B, int Sq, int H_kv, int K, int max_kv_len, int item_rows,
-                             size_t base, PrefillLayout *L) {
+                             int range_rows, size_t base, PrefillLayout *L) {
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
     *L = PrefillLayout{};
     L->nb_max = (max_kv_len + 127) / 128;
-    L->n_ranges = (Sq + kRange - 1) / kRange;
+    L->n_ranges = (Sq + range_rows - 1) / range_rows;
     L->n_ranges_total = static_cast<long long>(B) * H_kv * L->n_ranges;
-    L->rows_per_range = Sq < kRange ? Sq : kRange;
+    L->rows_per_range = Sq < range_rows ? Sq : range_rows;
     L->n_buckets = L->n_ranges_total * L->nb_max;
     const size_t per_range_rows = static_cast<size_t>(L->rows_per_range) * (K > 1 ? K - 1 : 1);
     L->item_rows = item_rows;

@@ -166,11 +166,12 @@ size_t prefill_workspace_layout(int B, int Sq, int H_q, int H_kv, int K, int max
                                 PrefillLayout *L);
 cudaError_t launch_prefill_attention(const PrefillArgs &a, uint8_t *ws, const PrefillLayout &L,
                                      cudaStream_t s);
-// Buckets alone (rows that kept block j != own, as work items of at most
-// item_rows rows), laid out from byte `base` of a workspace; returns the end.
-// The item count lands in *item_total, the 32-byte descriptors in item_desc.
+// Buckets alone (rows that kept block j != own, per range of range_rows
+// query rows, as work items of at most item_rows rows), laid out from byte
+// `base` of a workspace; returns the end.  The item count lands in
+// *item_total, the 32-byte descriptors in item_desc.
 size_t prefill_bucket_layout(int B, int Sq, int H_kv, int K, int max_kv_len, int item_rows,
-                             size_t base, PrefillLayout *L);
+                             int range_rows, size_t base, PrefillLayout *L);
 cudaError_t launch_prefill_buckets(PrefillArgs &a, uint8_t *ws, const PrefillLayout &L,
                                    long long *item_total, cudaStream_t s);
 // 3-D map over q [rows, H_q, 128] with a box of 64 dims x 8 heads x box_rows
