@@ -22,9 +22,10 @@
 //   - between index units a CTA takes published attention items, one per
 //     (sequence, group): the K/V tiles of its kept blocks (TMA, 128-byte
 //     swizzle) stream through the same ring, S^T = K Q^T and O^T = V^T P^T
-//     run on mma.sync for the group's heads with a running softmax across
-//     the blocks, and the CTA writes the group's output itself (no partial
-//     records, no merge across CTAs).
+//     run on mma.sync for the group's heads (one n8 tile per 8 heads, groups
+//     of up to 16) with a running softmax across the blocks, and the CTA
+//     writes the group's output itself (no partial records, no merge across
+//     CTAs).
 // An attention item is claimed (one atomicAdd) only while the claim counter
 // is below the published count; a claim that overtakes its publisher stays
 // pending while the CTA streams more index units.  Once a CTA has no index
@@ -33,6 +34,8 @@
 // keeps queueing its own CTA's top-k requests, and it ends only after its
 // bookkeeper has finished every unit it handed out, so no request is left
 // behind.  Every wait is bounded.
+#include <type_traits>
+
 #include "msa_device.cuh"
 #include "msa_internal.h"
 #include "topk_warp.cuh"
@@ -542,124 +545,151 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Warp w takes tokens 16w..16w+15 of each block, with a running
         // (max, sum, O^T) per head across the blocks; the blocks arrive in
         // ascending id order, so only the last one (the own block) is partial.
+        // The group's heads sit on the 8-wide side of the products: NT = 1
+        // n8 tile for groups of up to 8 heads, 2 for groups of 16.
         const int bg = w.y, n_kept = w.z;
         const int b = bg / H, g = bg % H;
         const int L = P.lens[b];
         const int last_valid = L - ((L - 1) / kBlock) * kBlock;
-        uint32_t qb[8][2];                          // Q^T of the group's heads (zero past G)
-        {
-            const __nv_bfloat16 *qh = static_cast<const __nv_bfloat16 *>(P.q) +
-                                      ((long long)b * P.H_q + (long long)g * G + gq) * kDim + tq * 2;
+        auto attn_item = [&](auto ntc) {
+            constexpr int NT = decltype(ntc)::value;
+            uint32_t qb[NT][8][2];                  // Q^T of heads 8 nt + gq (zero past G)
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                qb[kk][0] = gq < G ? *reinterpret_cast<const uint32_t *>(qh + kk * 16) : 0u;
-                qb[kk][1] = gq < G ? *reinterpret_cast<const uint32_t *>(qh + kk * 16 + 8) : 0u;
-            }
-        }
-        float m2[2] = {-INFINITY, -INFINITY}, l2[2] = {0.f, 0.f};
-        float acc[8][4];
+            for (int nt = 0; nt < NT; ++nt) {
+                const int hq = nt * 8 + gq;
+                const __nv_bfloat16 *qh = static_cast<const __nv_bfloat16 *>(P.q) +
+                                          ((long long)b * P.H_q + (long long)g * G + hq) * kDim + tq * 2;
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
-        for (int sl = 0; sl < n_kept; ++sl) {
-            int sk, sv;
-            const bool hk = wait_stage(sk);
-            const bool hv = wait_stage(sv);
-            if (!(hk && hv)) break;
-            const int nvalid = sl == n_kept - 1 ? last_valid : kBlock;
-            const uint32_t kb = smem_u32(S.ring[sk]), vb = smem_u32(S.ring[sv]);
-            if (nvalid < r0 + 16) {
-                // value rows past the query: weight 0, but padding may hold NaN
-                for (int e = lane; e < 16 * 16; e += 32) {
-                    const int r = r0 + (e >> 4), c = e & 15;
-                    if (r >= nvalid)
-                        *reinterpret_cast<uint4 *>(S.ring[sv] + (c >> 3) * 16384 + r * 128 + (c & 7) * 16) =
-                            make_uint4(0, 0, 0, 0);
+                for (int kk = 0; kk < 8; ++kk) {
+                    qb[nt][kk][0] = hq < G ? *reinterpret_cast<const uint32_t *>(qh + kk * 16) : 0u;
+                    qb[nt][kk][1] = hq < G ? *reinterpret_cast<const uint32_t *>(qh + kk * 16 + 8) : 0u;
                 }
-                fence_proxy_async_smem();          // before the next TMA write of this stage
-                __syncwarp();
             }
-            float sv4[4] = {0.f, 0.f, 0.f, 0.f};
+            float m2[NT][2], l2[NT][2];
+            float acc[NT][8][4];
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const int chunk = ((kk & 3) << 1) | (lane >> 4);
-                uint32_t a4[4];
-                ldsm_x4(kb + (kk >> 2) * 16384 + swz128(r0 + (lane & 15), chunk), a4[0], a4[1], a4[2], a4[3]);
-                mma_bf16_16816(sv4, a4, qb[kk][0], qb[kk][1]);
+            for (int nt = 0; nt < NT; ++nt) {
+                m2[nt][0] = m2[nt][1] = -INFINITY;
+                l2[nt][0] = l2[nt][1] = 0.f;
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[nt][mt][e] = 0.f;
             }
-            float p[4];
+            for (int sl = 0; sl < n_kept; ++sl) {
+                int sk, sv;
+                const bool hk = wait_stage(sk);
+                const bool hv = wait_stage(sv);
+                if (!(hk && hv)) break;
+                const int nvalid = sl == n_kept - 1 ? last_valid : kBlock;
+                const uint32_t kb = smem_u32(S.ring[sk]), vb = smem_u32(S.ring[sv]);
+                if (nvalid < r0 + 16) {
+                    // value rows past the query: weight 0, but padding may hold NaN
+                    for (int e = lane; e < 16 * 16; e += 32) {
+                        const int r = r0 + (e >> 4), c = e & 15;
+                        if (r >= nvalid)
+                            *reinterpret_cast<uint4 *>(S.ring[sv] + (c >> 3) * 16384 + r * 128 + (c & 7) * 16) =
+                                make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();      // before the next TMA write of this stage
+                    __syncwarp();
+                }
+                float sv4[NT][4];
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                const float x0 = r0 + gq < nvalid ? sv4[c] * sl2 : -INFINITY;
-                const float x1 = r0 + gq + 8 < nvalid ? sv4[2 + c] * sl2 : -INFINITY;
-                float cm = fmaxf(x0, x1);
-                cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 4));
-                cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 8));
-                cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 16));
-                const float mnew = fmaxf(m2[c], cm);
-                const float mref = mnew == -INFINITY ? 0.f : mnew;
-                const float alpha = exp2f(m2[c] - mref);
-                m2[c] = mnew;
-                p[c] = exp2f(x0 - mref);
-                p[2 + c] = exp2f(x1 - mref);
-                l2[c] = l2[c] * alpha + p[c] + p[2 + c];
+                for (int nt = 0; nt < NT; ++nt) sv4[nt][0] = sv4[nt][1] = sv4[nt][2] = sv4[nt][3] = 0.f;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const int chunk = ((kk & 3) << 1) | (lane >> 4);
+                    uint32_t a4[4];
+                    ldsm_x4(kb + (kk >> 2) * 16384 + swz128(r0 + (lane & 15), chunk), a4[0], a4[1], a4[2], a4[3]);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(sv4[nt], a4, qb[nt][kk][0], qb[nt][kk][1]);
+                }
+                uint32_t pb0[NT], pb1[NT];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    float p[4];
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const float x0 = r0 + gq < nvalid ? sv4[nt][c] * sl2 : -INFINITY;
+                        const float x1 = r0 + gq + 8 < nvalid ? sv4[nt][2 + c] * sl2 : -INFINITY;
+                        float cm = fmaxf(x0, x1);
+                        cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 4));
+                        cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 8));
+                        cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 16));
+                        const float mnew = fmaxf(m2[nt][c], cm);
+                        const float mref = mnew == -INFINITY ? 0.f : mnew;
+                        const float alpha = exp2f(m2[nt][c] - mref);
+                        m2[nt][c] = mnew;
+                        p[c] = exp2f(x0 - mref);
+                        p[2 + c] = exp2f(x1 - mref);
+                        l2[nt][c] = l2[nt][c] * alpha + p[c] + p[2 + c];
+#pragma unroll
+                        for (int mt = 0; mt < 8; ++mt) {
+                            acc[nt][mt][c] *= alpha;
+                            acc[nt][mt][2 + c] *= alpha;
+                        }
+                    }
+                    pb0[nt] = movmatrix_t(pack_bf16x2(p[0], p[1]));
+                    pb1[nt] = movmatrix_t(pack_bf16x2(p[2], p[3]));
+                }
+                const int mi = lane >> 3;
+                const int r = r0 + ((mi >> 1) << 3) + (lane & 7);
 #pragma unroll
                 for (int mt = 0; mt < 8; ++mt) {
-                    acc[mt][c] *= alpha;
-                    acc[mt][2 + c] *= alpha;
+                    const int d = mt * 16 + ((mi & 1) << 3);
+                    uint32_t a4[4];
+                    ldsm_x4_t(vb + (d >> 6) * 16384 + swz128(r, (d & 63) >> 3), a4[0], a4[1], a4[2], a4[3]);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(acc[nt][mt], a4, pb0[nt], pb1[nt]);
                 }
+                release_stage(sk);
+                release_stage(sv);
             }
-            const uint32_t pb0 = movmatrix_t(pack_bf16x2(p[0], p[1]));
-            const uint32_t pb1 = movmatrix_t(pack_bf16x2(p[2], p[3]));
-            const int mi = lane >> 3;
-            const int r = r0 + ((mi >> 1) << 3) + (lane & 7);
+            // Per n8 tile: per-warp partials to shared memory (heads 2tq + c
+            // of the tile), then the 8 warps merged and the heads written.
 #pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-                const int d = mt * 16 + ((mi & 1) << 3);
-                uint32_t a4[4];
-                ldsm_x4_t(vb + (d >> 6) * 16384 + swz128(r, (d & 63) >> 3), a4[0], a4[1], a4[2], a4[3]);
-                mma_bf16_16816(acc[mt], a4, pb0, pb1);
-            }
-            release_stage(sk);
-            release_stage(sv);
-        }
-        // per-warp partials to shared memory: heads 2tq + c
+            for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            float l = l2[c];
-            l += __shfl_xor_sync(0xffffffffu, l, 4);
-            l += __shfl_xor_sync(0xffffffffu, l, 8);
-            l += __shfl_xor_sync(0xffffffffu, l, 16);
-            const int h = 2 * tq + c;
-            if (gq == 0) { S.mw[warp][h] = m2[c]; S.lw[warp][h] = l; }
+                for (int c = 0; c < 2; ++c) {
+                    float l = l2[nt][c];
+                    l += __shfl_xor_sync(0xffffffffu, l, 4);
+                    l += __shfl_xor_sync(0xffffffffu, l, 8);
+                    l += __shfl_xor_sync(0xffffffffu, l, 16);
+                    const int h = 2 * tq + c;
+                    if (gq == 0) { S.mw[warp][h] = m2[nt][c]; S.lw[warp][h] = l; }
 #pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-                S.om[warp][h][mt * 16 + gq] = acc[mt][c];
-                S.om[warp][h][mt * 16 + gq + 8] = acc[mt][2 + c];
-            }
-        }
-        cbar();
-        if (!*abort_flag) {
-            // merge the 8 warps and write the group's heads
-            __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(P.out) + ((long long)b * P.H_q + (long long)g * G) * kDim;
-            for (int e = tid; e < G * kDim; e += kConsumers) {
-                const int h = e / kDim, d = e % kDim;
-                float M = -INFINITY;
-#pragma unroll
-                for (int w8 = 0; w8 < kWarps; ++w8) M = fmaxf(M, S.mw[w8][h]);
-                const float Mr = M == -INFINITY ? 0.f : M;
-                float o = 0.f, l = 0.f;
-#pragma unroll
-                for (int w8 = 0; w8 < kWarps; ++w8) {
-                    const float f = exp2f(S.mw[w8][h] - Mr);
-                    o += S.om[w8][h][d] * f;
-                    l += S.lw[w8][h] * f;
+                    for (int mt = 0; mt < 8; ++mt) {
+                        S.om[warp][h][mt * 16 + gq] = acc[nt][mt][c];
+                        S.om[warp][h][mt * 16 + gq + 8] = acc[nt][mt][2 + c];
+                    }
                 }
-                out[e] = __float2bfloat16(o / l);
+                cbar();
+                const int nh = min(8, G - nt * 8);            // heads of this tile
+                if (!*abort_flag) {
+                    __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(P.out) +
+                                         ((long long)b * P.H_q + (long long)g * G + nt * 8) * kDim;
+                    for (int e = tid; e < nh * kDim; e += kConsumers) {
+                        const int h = e / kDim, d = e % kDim;
+                        float M = -INFINITY;
+#pragma unroll
+                        for (int w8 = 0; w8 < kWarps; ++w8) M = fmaxf(M, S.mw[w8][h]);
+                        const float Mr = M == -INFINITY ? 0.f : M;
+                        float o = 0.f, l = 0.f;
+#pragma unroll
+                        for (int w8 = 0; w8 < kWarps; ++w8) {
+                            const float f = exp2f(S.mw[w8][h] - Mr);
+                            o += S.om[w8][h][d] * f;
+                            l += S.lw[w8][h] * f;
+                        }
+                        out[e] = __float2bfloat16(o / l);
+                    }
+                }
+                cbar();                             // om, mw, lw and bcast are reused
             }
-        }
-        cbar();                                     // om, mw, lw and bcast are reused
+        };
+        if (G > 8) attn_item(std::integral_constant<int, 2>{});
+        else attn_item(std::integral_constant<int, 1>{});
     }
     hand_over(-1, 0, 0.f);                          // end of the bookkeeper's stream
 }

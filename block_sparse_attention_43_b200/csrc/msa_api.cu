@@ -502,13 +502,13 @@ msa_status_t msa_sparse_attention_backward(const msa_shape_t *shape, const void 
 }
 
 // The fused decode step takes bf16 index keys, one row per index head (any
-// index-head count the shape allows), q_len 1 and groups of at most 8 heads
-// (one n8 tile of the attention products).
+// index-head count the shape allows), q_len 1 and groups of at most 16 heads
+// (one or two n8 tiles of the attention products).
 static msa_status_t check_decode_step(const msa_shape_t *s) {
     msa_status_t st = check_shape(s);
     if (st != MSA_OK) return st;
     if (s->q_len != 1 || s->index_key_format != MSA_INDEX_KEYS_BF16 ||
-        s->num_q_heads / s->num_kv_heads > 8)
+        s->num_q_heads / s->num_kv_heads > 16)
         return MSA_ERR_UNSUPPORTED;
     return MSA_OK;
 }

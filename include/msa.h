@@ -220,7 +220,7 @@ MSA_API msa_status_t msa_sparse_attention_backward(const msa_shape_t *shape, con
  * Requirements on top of the shape rules: q_len == 1, bf16 index keys with
  * one row per index head (index_key_format BF16; any num_index_heads the
  * shape allows, group g using the selection of index head
- * g / (num_kv_heads / num_index_heads)), and num_q_heads / num_kv_heads <= 8;
+ * g / (num_kv_heads / num_index_heads)), and num_q_heads / num_kv_heads <= 16;
  * otherwise MSA_ERR_UNSUPPORTED (shared and E4M3 index keys go through
  * msa_index_topk / msa_index_topk_fp8 and msa_sparse_attention).  The
  * launch is cooperative (one CTA per SM, all resident); it is not meant to

@@ -139,11 +139,11 @@ def test_index_variant_shapes_are_checked(m):
 
 
 def test_decode_step_rejects_unsupported_shapes(m):
-    """q_len > 1, groups of 16 heads, shared or E4M3 index keys: the
-    workspace query returns 0 and the call returns MSA_ERR_UNSUPPORTED.
-    Fewer index heads than groups (bf16, one key row per index head) are
+    """q_len > 1, shared or E4M3 index keys: the workspace query returns 0
+    and the call returns MSA_ERR_UNSUPPORTED.  Fewer index heads than groups
+    (bf16, one key row per index head) and groups of 16 heads are
     accepted."""
-    for kw in (dict(q_len=2), dict(num_q_heads=32), dict(index_key_format=m.INDEX_KEYS_BF16_SHARED),
+    for kw in (dict(q_len=2), dict(index_key_format=m.INDEX_KEYS_BF16_SHARED),
                dict(index_key_format=m.INDEX_KEYS_FP8)):
         base = dict(batch=1, q_len=1, max_kv_len=1000, num_q_heads=16, num_kv_heads=2, top_k=4,
                     kv_capacity=1000)
@@ -159,6 +159,9 @@ def test_decode_step_rejects_unsupported_shapes(m):
     fewer = m.make_shape(batch=3, q_len=1, max_kv_len=1000, num_q_heads=16, num_kv_heads=2,
                          top_k=4, kv_capacity=3000, num_index_heads=1)
     assert m.msa_decode_step_workspace_size(fewer) > 256
+    g16 = m.make_shape(batch=3, q_len=1, max_kv_len=1000, num_q_heads=32, num_kv_heads=2,
+                       top_k=4, kv_capacity=3000)
+    assert m.msa_decode_step_workspace_size(g16) > 256
     # paged: a pool that is not whole pages, or a table row too short for max_kv_len
     for cap, pps in ((3000, 8), (3072, 7)):
         s = m.make_shape(batch=3, q_len=1, max_kv_len=1000, num_q_heads=16, num_kv_heads=2,

@@ -44,7 +44,7 @@ def _run_and_compare(oracle_mod, w, rows=None):
 
 
 # (B, lens, H_q, H_kv, top_k): ragged lengths, a block-aligned length, fewer
-# blocks than k, a single token, one group, 16 groups, group sizes 1..8.
+# blocks than k, a single token, one group, 16 groups, group sizes 1..16.
 CASES = [
     (3, [5000, 128, 1], 16, 2, 4),
     (2, [4096, 4097], 64, 8, 16),
@@ -54,6 +54,8 @@ CASES = [
     (2, [6000, 6001], 16, 4, 1),
     (1, [3 * 128 + 5], 8, 8, 16),
     (7, [300, 129000, 5, 4096, 77777, 1024, 65], 32, 4, 64),
+    (3, [9000, 129, 40000], 32, 2, 16),                # groups of 16 (two n8 tiles)
+    (2, [5000, 300], 128, 8, 8),                       # groups of 16, 8 groups
 ]
 
 
