@@ -256,10 +256,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// m16n8k16 with f16 operands and fp32 accumulation (products of two f16
+// values are exact in fp32, as those of two bf16 values are).
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                              uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // Shared E4M3 keys, one block per consumer warp: the widening makes each block
 // worth ~1000 instructions per warp, so blocks are not split across warps
 // (no cross-warp reduction, no CTA barrier); the CTA's k-th block goes to
 // stage k % 8 and warp k % 8, so eight blocks are in flight per SM.
+// Every E4M3 value is an f16 value, so when a sequence's index queries are f16
+// values too (bf16 values inside f16's range, checked per warp and sequence),
+// the products run on f16 operands and each pair of codes costs one
+// conversion; otherwise the codes are widened to bf16 (three more steps).
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 1)
     index_shared_fp8_kernel(const IndexDecodeVarArgs P) {
@@ -314,6 +329,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int gq = lane >> 2, tq = lane & 3;
     const __nv_bfloat16 *qbase = static_cast<const __nv_bfloat16 *>(P.q_idx);
     uint32_t qf[8][NT][2];
+    uint32_t qh16[8][NT][2];                    // the same queries as f16 pairs
+    bool f16ok = false;
     int cur_b = -1;
     for (int it = warp;; it += kWarps) {
         const long long uu = blockIdx.x + static_cast<long long>(it) * gridDim.x;
@@ -337,6 +354,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     qf[kk][nt][0] = h < H ? *reinterpret_cast<const uint32_t *>(qh) : 0u;
                     qf[kk][nt][1] = h < H ? *reinterpret_cast<const uint32_t *>(qh + 2) : 0u;
                 }
+            bool exact = true;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const float lo = bf16lo(qf[kk][nt][e]), hi = bf16hi(qf[kk][nt][e]);
+                        const __half2 h2 = __floats2half2_rn(lo, hi);
+                        exact = exact && __low2float(h2) == lo && __high2float(h2) == hi;
+                        qh16[kk][nt][e] = *reinterpret_cast<const uint32_t *>(&h2);
+                    }
+            f16ok = __all_sync(0xffffffffu, exact);
             cur_b = b;
         }
         // Row scales of this thread's 16 tokens (2 per 16-token tile).
@@ -370,15 +400,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
+            if (f16ok) {
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                uint32_t a[4];
-                a[0] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w0[kk] & 0xFFFFu));
-                a[1] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w1[kk] & 0xFFFFu));
-                a[2] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w0[kk] >> 16));
-                a[3] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w1[kk] >> 16));
+                for (int kk = 0; kk < 8; ++kk) {
+                    uint32_t a[4];
+                    a[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[kk] & 0xFFFFu));
+                    a[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] & 0xFFFFu));
+                    a[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[kk] >> 16));
+                    a[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] >> 16));
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a, qf[kk][nt][0], qf[kk][nt][1]);
+                    for (int nt = 0; nt < NT; ++nt) mma_f16_16816(s[nt], a, qh16[kk][nt][0], qh16[kk][nt][1]);
+                }
+            } else {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    uint32_t a[4];
+                    a[0] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w0[kk] & 0xFFFFu));
+                    a[1] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w1[kk] & 0xFFFFu));
+                    a[2] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w0[kk] >> 16));
+                    a[3] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w1[kk] >> 16));
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a, qf[kk][nt][0], qf[kk][nt][1]);
+                }
             }
             // rows past the length hold stale bytes: masked here
             const bool v0 = tok < ntok, v1 = tok + 8 < ntok;
