@@ -96,3 +96,16 @@ def test_prefill_variants(oracle_mod, fmt, B, Sq, lens, H_q, H_kv, Hi, top_k):
                     device=DEV)
     rep = _run(w, Hi, FORMATS[fmt], 2)
     print(fmt, (B, Sq, H_kv, Hi), rep)
+
+
+def test_decode_shared_fp8_queries_outside_f16(oracle_mod):
+    """Shared E4M3 keys take f16 products when a sequence's index queries are
+    f16 values.  Sequence 0's queries here are scaled by 2^17 (exact in bf16,
+    beyond f16's range), so its warps widen the codes to bf16 instead;
+    sequence 1 keeps the f16 form.  Both must match the oracle."""
+    from synthetic import make_inputs
+    w = make_inputs(B=2, Sq=1, lens=[6000, 3000], H_q=64, H_kv=8, top_k=16, seed=77, device=DEV,
+                    needles=2, amp=4.0)
+    w.q_idx[0] *= 2.0 ** 17
+    assert w.q_idx[0].float().abs().max().item() > 65504.0
+    print(_run(w, 8, FORMATS["fp8_shared"], 3))
