@@ -516,15 +516,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (MODE == 1) {
                     // every column is visible; a padding lane gets 2^-inf = 0
                     const float sh = valid ? shift : INFINITY;
+                    // four independent sums: the adds are not one serial chain
+                    float l1 = 0.f, l2 = 0.f, l3 = 0.f;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
+                    for (int e = 0; e < 32; e += 2) {
                         const uint32_t *src = e < 16 ? a : b;
                         const int k = (2 * e) & 31;
                         const float p0 = fast_exp2(fmaf(__uint_as_float(src[k]), sl2, -sh));
                         const float p1 = fast_exp2(fmaf(__uint_as_float(src[k + 1]), sl2, -sh));
-                        l += p0 + p1;
+                        const float p2 = fast_exp2(fmaf(__uint_as_float(src[k + 2]), sl2, -sh));
+                        const float p3 = fast_exp2(fmaf(__uint_as_float(src[k + 3]), sl2, -sh));
+                        l += p0;
+                        l1 += p1;
+                        l2 += p2;
+                        l3 += p3;
                         pk[e] = pack_bf16x2(p0, p1);
+                        pk[e + 1] = pack_bf16x2(p2, p3);
                     }
+                    l = (l + l1) + (l2 + l3);
                 } else {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {

@@ -332,9 +332,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tmem_wait_ld(va);
                             tmem_tie(vb);
                             if (full) {
+                                // four independent max chains instead of one serial one
+                                float m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-                                for (int e = 0; e < 32; ++e)
+                                for (int e = 0; e < 32; e += 4) {
                                     m = fmax3(m, __uint_as_float(va[e]), __uint_as_float(vb[e]));
+                                    m1 = fmax3(m1, __uint_as_float(va[e + 1]), __uint_as_float(vb[e + 1]));
+                                    m2 = fmax3(m2, __uint_as_float(va[e + 2]), __uint_as_float(vb[e + 2]));
+                                    m3 = fmax3(m3, __uint_as_float(va[e + 3]), __uint_as_float(vb[e + 3]));
+                                }
+                                m = fmax3(m, m1, fmaxf(m2, m3));
                             } else {
 #pragma unroll
                                 for (int e = 0; e < 32; ++e) {
