@@ -16,7 +16,8 @@
 //             base-2 log-sum-exp of every (row, head)
 //   prep      Delta = dO.O per (row, head); clears the fp32 dQ accumulator
 //   buckets   rows that kept block j (j != own) as work items, built by the
-//             forward's prefill bucket kernels
+//             forward's prefill bucket kernels (the forward's own items when
+//             it ran the block-outer prefill path: groups of 8)
 //   main      per work item -- one key block j of one (sequence, group) and
 //             the rows that use it -- K_j and V_j are loaded once; per tile of
 //             128/G rows x G heads = 128 (row, head) pairs:
@@ -775,7 +776,7 @@ cudaError_t launch_blocks(const CUtensorMap &tk, const CUtensorMap &tv, const At
 }  // namespace
 
 size_t attn_bwd_layout(int B, int Sq, int H_q, int H_kv, int K, int max_kv_len, size_t base,
-                       AttnBwdLayout *L) {
+                       const PrefillLayout *fwd, AttnBwdLayout *L) {
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
     const size_t pairs = static_cast<size_t>(B) * Sq * H_q;
     size_t o = up(base);
@@ -784,8 +785,13 @@ size_t attn_bwd_layout(int B, int Sq, int H_q, int H_kv, int K, int max_kv_len, 
     L->delta = o;   o += up(pairs * 4);
     L->dq_acc = o;  o += up(pairs * kDim * 4);
     const int G = H_q / H_kv;
-    o = prefill_bucket_layout(B, Sq, H_kv, K, max_kv_len, kTilesPerItem * (128 / G), kRangeRows, o,
-                              &L->bk);
+    const int item_rows = kTilesPerItem * (128 / G);
+    L->reuse = fwd && fwd->item_rows == item_rows && fwd->rows_per_range == (Sq < kRangeRows ? Sq : kRangeRows);
+    L->fwd_rows = L->reuse ? fwd->rows : 0;
+    L->fwd_desc = L->reuse ? fwd->item_desc : 0;
+    L->bk = PrefillLayout{};
+    if (!L->reuse)
+        o = prefill_bucket_layout(B, Sq, H_kv, K, max_kv_len, item_rows, kRangeRows, o, &L->bk);
     L->total = o;
     return o;
 }
@@ -815,10 +821,18 @@ cudaError_t launch_attn_bwd(const AttnBwdArgs &a0, uint8_t *ws, const AttnBwdLay
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    if ((e = launch_prefill_buckets(pb, ws, L.bk, hdr, s)) != cudaSuccess) return e;
-    a.bucket_rows = pb.bucket_rows;
-    a.item_desc = pb.item_desc;
-    a.item_total = hdr;
+    if (L.reuse) {
+        // the forward's bucket items (same rows per item and range): its
+        // item count sits in header bytes 8..15
+        a.bucket_rows = reinterpret_cast<const int *>(ws + L.fwd_rows);
+        a.item_desc = reinterpret_cast<const int *>(ws + L.fwd_desc);
+        a.item_total = reinterpret_cast<const long long *>(ws + 8);
+    } else {
+        if ((e = launch_prefill_buckets(pb, ws, L.bk, hdr, s)) != cudaSuccess) return e;
+        a.bucket_rows = pb.bucket_rows;
+        a.item_desc = pb.item_desc;
+        a.item_total = hdr;
+    }
     a.item_next = hdr + 1;
     switch (a.H_q / a.H_kv) {
     case 1: e = launch_blocks<1>(tk, tv, a, s); break;

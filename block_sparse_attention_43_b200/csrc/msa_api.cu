@@ -452,8 +452,9 @@ msa_status_t msa_kv_append(const msa_shape_t *shape, int32_t n_new, const void *
 // The backward's workspace: the forward's (recomputed first, from byte 0),
 // then the output, statistics, dQ accumulator and buckets of the backward.
 static size_t bwd_layout(const msa_shape_t *s, AttnBwdLayout *L) {
+    const AttnLayout F = attn_layout(s);
     return attn_bwd_layout(s->batch, s->q_len, s->num_q_heads, s->num_kv_heads, s->top_k,
-                           s->max_kv_len, attn_layout(s).total, L);
+                           s->max_kv_len, F.total, use_prefill_path(s) ? &F.pre : nullptr, L);
 }
 
 size_t msa_sparse_attention_backward_workspace_size(const msa_shape_t *shape) {

@@ -241,12 +241,16 @@ struct AttnBwdArgs {
 };
 struct AttnBwdLayout {
     size_t o, lse, delta, dq_acc, total;
-    PrefillLayout bk;       // the backward's own buckets
+    PrefillLayout bk;       // the backward's own buckets (unless reused)
+    bool reuse;             // the forward's prefill buckets are the same items
+    size_t fwd_rows, fwd_desc;
 };
 // Lays the backward's regions out from byte `base` of the workspace (the
-// forward's layout ends there); returns the total size.
+// forward's layout ends there); returns the total size.  fwd: the forward's
+// prefill layout when it ran the block-outer path (its bucket items are
+// reused when they are the backward's), else nullptr.
 size_t attn_bwd_layout(int B, int Sq, int H_q, int H_kv, int K, int max_kv_len, size_t base,
-                       AttnBwdLayout *L);
+                       const PrefillLayout *fwd, AttnBwdLayout *L);
 cudaError_t launch_attn_bwd(const AttnBwdArgs &a, uint8_t *ws, const AttnBwdLayout &L,
                             cudaStream_t s);
 
