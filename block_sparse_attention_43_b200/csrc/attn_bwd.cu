@@ -26,11 +26,14 @@
 //               P^T  = 2^(S^T scale log2 e - lse)  bf16, back into S^T's columns
 //               dS^T = scale P^T (dP^T - Delta)    bf16, shared memory
 //               dV  += P^T dO                      A from TMEM, summed over the item
-//               dK  += dS^T Q                      summed over the item
-//               dQ   = dS K_j                      A = dS^T read transposed
-//             dQ of each tile is added to the accumulator with fp32 vector
+//               dQ^T = K_j^T dS^T                  dims x pairs
+//               dK^T += Q^T dS                     dims x tokens, summed over the item
+//             (dQ and dK are formed transposed so that a warp's reduction
+//             covers 32 consecutive dims of one row: whole 128-byte lines).
+//             dQ of each tile is added to the accumulator with fp32
 //             reductions; dK and dV leave TMEM once per item, not once per
-//             (row, block)
+//             (row, block); the next tile's S^T is issued ahead of the
+//             current tile's dQ and dK
 //   finalize  dq = accumulator, bf16
 // The own block of each row is processed as items of the consecutive rows
 // whose own block it is (causal mask); every product is tcgen05.mma
@@ -41,7 +44,7 @@
 // rows and statistics with cp.async (zero-filled past the item's rows);
 // warps 4-11 compute P and dS, two warps per TMEM lane quarter with 64 pair
 // columns each; warps 12-15 drain dQ per tile and dK, dV per item.  TMEM
-// columns: S^T / P^T 0-127, dP^T / dQ 128-255, dV 256-383, dK 384-511.
+// columns: S^T / P^T 0-127, dP^T / dQ^T 128-255, dV 256-383, dK^T 384-511.
 #include "msa_device.cuh"
 #include "msa_internal.h"
 

@@ -181,3 +181,23 @@ def test_block_count_bound(m):
     ok = m.make_shape(batch=4096, q_len=1, max_kv_len=(1 << 26) - 128, num_q_heads=64,
                       num_kv_heads=8, top_k=16, kv_capacity=1 << 27)
     assert m.msa_index_topk_workspace_size(ok) > 0
+
+
+def test_backward_workspace_layout(m):
+    """The backward's workspace is the forward's, then per (row, head) the
+    recomputed output (256 B), log-sum-exp and Delta (4 B each) and the fp32
+    dQ sum (512 B), each region rounded to 256 B, then the backward's own
+    bucket lists -- except with groups of 8 on the block-outer prefill path,
+    whose forward items are reused and add nothing."""
+    up = lambda x: (x + 255) // 256 * 256
+    for H_q, H_kv, Sq in ((64, 8, 4096), (8, 2, 2048), (64, 8, 1)):
+        s = m.make_shape(batch=2, q_len=Sq, max_kv_len=8192, num_q_heads=H_q, num_kv_heads=H_kv,
+                         top_k=16, kv_capacity=16384)
+        fwd = m.msa_sparse_attention_workspace_size(s)
+        bwd = m.msa_sparse_attention_backward_workspace_size(s)
+        pairs = 2 * Sq * H_q
+        regions = up(pairs * 256) + 2 * up(pairs * 4) + up(pairs * 512)
+        if H_q // H_kv == 8 and Sq > 1:
+            assert bwd == up(fwd) + regions
+        else:
+            assert bwd > up(fwd) + regions
