@@ -906,6 +906,9 @@ __global__ void __launch_bounds__(256) finalize_kernel(const PrefillArgs P) {
                 const uint32_t nan2 = pack_bf16x2(NAN, NAN);
                 o = make_uint4(nan2, nan2, nan2, nan2);
                 if (P.lse && cd == 0) P.lse[row * P.H_q + g * kG + h] = NAN;
+                // once per sequence: its first row's first chunk
+                if (q == 0 && g == 0 && row == static_cast<long long>(b) * P.Sq)
+                    set_status(P.status, kStatusBadLens);
             } else {
                 const float inv = 1.f / l[u];
                 if (P.lse && cd == 0)

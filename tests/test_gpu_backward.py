@@ -154,3 +154,39 @@ def test_backward_32k_rows_sampled(oracle_mod):
                    dv=_check(f"dv[{j},{grp}]", gv[t, grp], rv[t, 0]),
                    dq=_check(f"dq[rows of {j},{grp}]", gq[rows, hs], rq.reshape(n, G, 128)))
         print(grp, j, rep)
+
+
+@pytest.mark.parametrize("H_q,H_kv", [(64, 8), (16, 4)])
+def test_backward_bad_lengths(oracle_mod, H_q, H_kv):
+    """A sequence whose length is out of range: the call raises the status
+    word, writes NaN into that sequence's dq and leaves its keys' dk, dv
+    alone; the other sequence's gradients still match the oracle."""
+    from synthetic import bf16_bits, make_inputs
+    w = make_inputs(B=2, Sq=300, lens=[600, 900], H_q=H_q, H_kv=H_kv, top_k=4, seed=74,
+                    device=DEV)
+    eng = m.MSA(batch=2, q_len=300, max_kv_len=900, num_q_heads=H_q, num_kv_heads=H_kv, top_k=4,
+                kv_capacity=w.kv_capacity, device=DEV)
+    eng.index_topk(w.q_idx, w.k_idx, w.lens, w.kv_offsets)
+    g = torch.Generator(device=DEV).manual_seed(79)
+    dout = torch.randn(w.q.shape, generator=g, device=DEV).to(torch.bfloat16)
+    dq = torch.empty_like(w.q)
+    dk = torch.zeros(w.k.shape, dtype=torch.float32, device=DEV)
+    dv = torch.zeros(w.v.shape, dtype=torch.float32, device=DEV)
+    ws = m.alloc_workspace(m.msa_sparse_attention_backward_workspace_size(eng.shape), DEV)
+    bad = torch.tensor([600, 5000], dtype=torch.int32, device=DEV)     # 5000 > max_kv_len
+    m.msa_sparse_attention_backward(eng.shape, w.q, w.k, w.v, eng.block_ids, bad, w.kv_offsets,
+                                    w.scale, dout, dq, dk, dv, ws)
+    torch.cuda.synchronize()
+    assert m.msa_read_device_status(ws) == 6
+    gq = dq.float().cpu().numpy()
+    assert np.isnan(gq[1]).all() and np.isfinite(gq[0]).all()
+    offs = w.kv_offsets.cpu().numpy()
+    gk, gv = dk.cpu().numpy(), dv.cpu().numpy()
+    assert (gk[offs[1]:] == 0).all() and (gv[offs[1]:] == 0).all()
+    ids = eng.block_ids.cpu().numpy()
+    rq, rk, rv = oracle_mod.sparse_attention_backward(
+        bf16_bits(w.q)[:1], bf16_bits(w.k), bf16_bits(w.v), bf16_bits(dout)[:1], ids[:1],
+        np.array([600], np.int32), offs[:1], scale=w.scale)
+    _check("dq", gq[0].reshape(rq.shape), rq)
+    _check("dk", gk, rk)
+    _check("dv", gv, rv)

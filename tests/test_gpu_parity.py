@@ -231,3 +231,20 @@ def test_bad_lengths_set_device_status(msa_lib):
     # A clean call clears the word again.
     eng.index_topk(w.q_idx, w.k_idx, w.lens, w.kv_offsets)
     assert m.msa_read_device_status(eng.ws_index) == 0
+
+
+def test_bad_lengths_prefill_path(msa_lib):
+    """The block-outer prefill path (groups of 8) reports an out-of-range
+    length the same way: status word raised, NaN output for that sequence,
+    the other sequence finite."""
+    import block_sparse_attention_43_b200 as m
+    from synthetic import make_inputs
+    w = make_inputs(B=2, Sq=300, lens=[600, 900], H_q=64, H_kv=8, top_k=4, seed=6, device=DEV)
+    eng = m.MSA(batch=2, q_len=300, max_kv_len=900, num_q_heads=64, num_kv_heads=8, top_k=4,
+                kv_capacity=w.kv_capacity, device=DEV)
+    eng.index_topk(w.q_idx, w.k_idx, w.lens, w.kv_offsets)
+    bad = torch.tensor([600, 5000], dtype=torch.int32, device=DEV)     # 5000 > max_kv_len
+    eng.sparse_attention(w.q, w.k, w.v, bad, w.kv_offsets)
+    assert m.msa_read_device_status(eng.ws_attn) == 6
+    out = eng.out.float().cpu()
+    assert torch.isnan(out[1]).all() and torch.isfinite(out[0]).all()
