@@ -168,7 +168,9 @@ def sparse_attention_backward(q, k, v, dout, block_ids, lens, kv_offsets, *, blo
                               scale=None, num_index_heads=None, n_threads=None):
     """Backward of the sparse branch.  Shapes as sparse_attention, plus dout
     [B,Sq,H_q,D] (uint16 bf16 bits).  Returns (dq [B*Sq,H_q,D], dk [T,H_kv,D],
-    dv [T,H_kv,D]), float64; dk/dv are zero on keys no row kept."""
+    dv [T,H_kv,D]), float64; dk/dv are zero on keys no row kept.  Each thread
+    owns whole (sequence, group) jobs and adds into dk/dv without locks, so
+    with n_threads > 1 the sequences must not share cache rows."""
     q = _c(q, np.uint16)
     k = _c(k, np.uint16)
     v = _c(v, np.uint16)
