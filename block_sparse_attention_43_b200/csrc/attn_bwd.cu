@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             prefetch_tensormap(&tmK);
             prefetch_tensormap(&tmV);
-            int ki = 0;
+            int ki = 0, last_issued = -1;
             bool ok = true;
             for (int n = 0; ok; ++n) {
                 const int slot = n % kQueue;
@@ -290,6 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_3d(S.kv + 16384, &tmK, 64, x.g, tok, &S.kv_full);
                 tma_load_3d(S.kv + 32768, &tmV, 0, x.g, tok, &S.kv_full);
                 tma_load_3d(S.kv + 49152, &tmV, 64, x.g, tok, &S.kv_full);
+                last_issued = ki;
                 const int nvalid = x.L - x.j * 128;      // tokens of the block inside the sequence
                 if (nvalid < 128) {
                     if (*abort_flag || !mbar_wait(&S.kv_full, ki & 1, P.status)) {
@@ -307,6 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++ki;
             }
             if (!ok) *abort_flag = 1;
+            // The last K/V copy lands before the CTA can end, abort or not.
+            if (last_issued >= 0) mbar_wait(&S.kv_full, last_issued & 1, nullptr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (lane 0)
